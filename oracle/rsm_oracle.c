@@ -1,0 +1,169 @@
+/*
+ * rsm_oracle.c -- TEST INFRASTRUCTURE ONLY.
+ *
+ * A plain, slow, sequential fp64 CPU restatement of the Raven routing-state-model (RSM) mixer.
+ * It exists to check the CUDA library; only tests/, __graft_entry__.smoke() and bench.py's CPU
+ * baseline leg may load it. It shares no code, header, table or constant with the CUDA path.
+ *
+ * What it computes, per batch b, head h, token t (one token at a time, no chunking):
+ *   1. S_t = the K slots with the largest router logits, ordered by (logit desc, slot index asc).
+ *      Raven README (github.com/xiaol/SelectingMemory), "How Raven Works": the router keeps the
+ *      TopK of sigmoid(r_proj(x)); sigmoid is monotone, so the order is the order of the logits.
+ *      paperlayer.ai summary of "Raven: High-Recall Sequence Modeling with Sparse Memory Routing",
+ *      section 4.1: only the top-K entries are kept, the rest are zero.
+ *   2. s_i = sigmoid(logit_i) for i in S_t (README, "How Raven Works").
+ *   3. decay a_i = exp(s_i * f) with f the per-head (Mamba2) or per-slot (GLA) log-decay
+ *      (README, "How Raven Works" and "Model Structure": Mamba2 or GLA decay).
+ *   4. for i in S_t: H[i,:] = a_i * H[i,:] + (1 - a_i) * k_i * v ; other rows are not touched
+ *      (README, "How Raven Works"; "Raven Part 1 -- Memory as a Set of Slots", "Method": a slot
+ *      with zero routing is carried over unchanged).
+ *   5. o_t = sum_i q_i * H[i,:], read after the write (README, "How Raven Works").
+ *
+ * Layouts (row-major, contiguous): q, k, logits [B,T,H,M]; v [B,T,H,Dv]; f [B,T,H] (per head)
+ * or [B,T,H,M] (per slot); H0, HT [B,H,M,Dv]; o [B,T,H,Dv]; idx, score [B,T,H,K].
+ * Inputs are the exact fp32 values the device sees (bf16 inputs are widened exactly beforehand).
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* Slot a ranks ahead of slot b: larger logit first, the lower index on an exact tie.
+ * Comparisons are on the fp32 values (widened to fp64, which preserves order and equality;
+ * -0.0 and +0.0 compare equal and fall to the index rule). */
+static int rsmo_ahead(const float* row, int a, int b) {
+  double xa = (double)row[a], xb = (double)row[b];
+  if (xa > xb) return 1;
+  if (xa < xb) return 0;
+  return a < b;
+}
+
+/* TopK by insertion sort of all M slot indices under rsmo_ahead; the first K are kept. */
+void rsmo_topk(const float* row, int M, int K, int32_t* idx_out) {
+  int* ord = (int*)malloc(sizeof(int) * (size_t)M);
+  for (int i = 0; i < M; ++i) {
+    int j = i;
+    while (j > 0 && rsmo_ahead(row, i, ord[j - 1])) {
+      ord[j] = ord[j - 1];
+      --j;
+    }
+    ord[j] = i;
+  }
+  for (int r = 0; r < K; ++r) idx_out[r] = ord[r];
+  free(ord);
+}
+
+double rsmo_sigmoid(double x) { return 1.0 / (1.0 + exp(-x)); }
+
+typedef struct {
+  int B, T, H, M, K, Dv, per_slot;
+  const float *q, *k, *v, *logits, *f;
+  const double* H0;
+  double *o, *HT;
+  int32_t* idx;
+  double* score;
+  int pair_begin, pair_end; /* range of flattened (b,h) pairs handled by one worker */
+} rsmo_job;
+
+/* One (b,h) pair, all T tokens, strictly in order. */
+static void rsmo_run_pair(const rsmo_job* J, int pair) {
+  const int b = pair / J->H, h = pair % J->H;
+  const int M = J->M, K = J->K, Dv = J->Dv, H = J->H, T = J->T;
+  double* S = (double*)malloc(sizeof(double) * (size_t)M * (size_t)Dv);
+  int32_t* sel = (int32_t*)malloc(sizeof(int32_t) * (size_t)K);
+  if (J->H0)
+    memcpy(S, J->H0 + (size_t)pair * M * Dv, sizeof(double) * (size_t)M * Dv);
+  else
+    memset(S, 0, sizeof(double) * (size_t)M * Dv);
+
+  for (int t = 0; t < T; ++t) {
+    const size_t row = ((size_t)b * T + t) * H + h; /* flattened (b,t,h) */
+    const float* q = J->q + row * M;
+    const float* k = J->k + row * M;
+    const float* lg = J->logits + row * M;
+    const float* v = J->v + row * Dv;
+    rsmo_topk(lg, M, K, sel);
+    for (int r = 0; r < K; ++r) {
+      const int i = sel[r];
+      const double s = rsmo_sigmoid((double)lg[i]);
+      const double f = J->per_slot ? (double)J->f[row * M + i] : (double)J->f[row];
+      const double a = exp(s * f);
+      const double wk = (1.0 - a) * (double)k[i];
+      double* Si = S + (size_t)i * Dv;
+      for (int d = 0; d < Dv; ++d) Si[d] = a * Si[d] + wk * (double)v[d];
+      if (J->idx) J->idx[row * K + r] = i;
+      if (J->score) J->score[row * K + r] = s;
+    }
+    if (J->o) {
+      double* o = J->o + row * Dv;
+      for (int d = 0; d < Dv; ++d) o[d] = 0.0;
+      for (int i = 0; i < M; ++i) {
+        const double qi = (double)q[i];
+        const double* Si = S + (size_t)i * Dv;
+        for (int d = 0; d < Dv; ++d) o[d] += qi * Si[d];
+      }
+    }
+  }
+  if (J->HT) memcpy(J->HT + (size_t)pair * M * Dv, S, sizeof(double) * (size_t)M * Dv);
+  free(sel);
+  free(S);
+}
+
+static void* rsmo_worker(void* arg) {
+  const rsmo_job* J = (const rsmo_job*)arg;
+  for (int p = J->pair_begin; p < J->pair_end; ++p) rsmo_run_pair(J, p);
+  return NULL;
+}
+
+/* Runs the recurrence over all (b,h) pairs; pairs are independent, so they are split over
+ * nthreads POSIX threads (nthreads <= 1 runs inline). Returns 0 on success, -1 on bad sizes. */
+int rsmo_forward(int B, int T, int H, int M, int K, int Dv, int per_slot,
+                 const float* q, const float* k, const float* v, const float* logits,
+                 const float* f, const double* H0, double* o, double* HT, int32_t* idx,
+                 double* score, int nthreads) {
+  if (B < 0 || T < 0 || H < 0 || M < 1 || K < 1 || K > M || Dv < 1) return -1;
+  const int pairs = B * H;
+  if (nthreads < 1) nthreads = 1;
+  if (nthreads > pairs) nthreads = pairs > 0 ? pairs : 1;
+  rsmo_job base = {B, T, H, M, K, Dv, per_slot, q, k, v, logits, f, H0, o, HT, idx, score, 0, pairs};
+  if (nthreads == 1) {
+    rsmo_worker(&base);
+    return 0;
+  }
+  pthread_t* th = (pthread_t*)malloc(sizeof(pthread_t) * (size_t)nthreads);
+  rsmo_job* jobs = (rsmo_job*)malloc(sizeof(rsmo_job) * (size_t)nthreads);
+  for (int w = 0; w < nthreads; ++w) {
+    jobs[w] = base;
+    jobs[w].pair_begin = (int)((long long)pairs * w / nthreads);
+    jobs[w].pair_end = (int)((long long)pairs * (w + 1) / nthreads);
+    pthread_create(&th[w], NULL, rsmo_worker, &jobs[w]);
+  }
+  for (int w = 0; w < nthreads; ++w) pthread_join(th[w], NULL);
+  free(jobs);
+  free(th);
+  return 0;
+}
+
+/* One generation step: the same update and read for a single token per (b,h), applied in
+ * place to the carried state (README, "Model Structure": fused recurrent computation for
+ * inference). Layouts: q, k, logits [B,H,M]; v [B,H,Dv]; f [B,H] or [B,H,M];
+ * state [B,H,M,Dv] (in/out); o [B,H,Dv]; idx, score [B,H,K]. */
+int rsmo_decode_step(int B, int H, int M, int K, int Dv, int per_slot, const float* q,
+                     const float* k, const float* v, const float* logits, const float* f,
+                     double* state, double* o, int32_t* idx, double* score, int nthreads) {
+  /* A step is the T = 1 case of the recurrence with the carried state as both H0 and HT. */
+  return rsmo_forward(B, 1, H, M, K, Dv, per_slot, q, k, v, logits, f, state, o, state, idx,
+                      score, nthreads);
+}
+
+/* Standalone routing: TopK indices (rank order) and sigmoid scores for rows [rows, M]. */
+int rsmo_route(const float* logits, long long rows, int M, int K, int32_t* idx, double* score) {
+  if (rows < 0 || M < 1 || K < 1 || K > M) return -1;
+  for (long long r = 0; r < rows; ++r) {
+    const float* lg = logits + r * M;
+    rsmo_topk(lg, M, K, idx + r * K);
+    for (int j = 0; j < K; ++j) score[r * K + j] = rsmo_sigmoid((double)lg[idx[r * K + j]]);
+  }
+  return 0;
+}

@@ -1,0 +1,284 @@
+"""Pins the fp64 CPU oracle to things other than itself (CPU only).
+
+* hand-derived worked examples (tests/golden/*.json, each with its citation and derivation);
+* an independent unrolled closed form on tiny inputs (oracle/brute.py, quadratic form);
+* the TopK = M limit against a masked-matrix gated-linear-attention form;
+* the one-hot cyclic router limit against the sliding-window closed form;
+* TopK against a stable library sort, with constructed ties, signed zeros and saturating logits;
+* sigmoid scores against scipy's expit;
+* the invariant that unselected slots keep their bits;
+* mutants of the oracle (planted mistakes, compiled on the CPU) must fail these pins.
+"""
+import ctypes
+import json
+import math
+import os
+import subprocess
+
+import numpy as np
+import pytest
+from scipy.special import expit
+
+from oracle import brute, oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rand_stream(rng, T, M, Dv, per_slot, fscale=1.0):
+    q = rng.standard_normal((T, M)).astype(np.float32)
+    k = rng.standard_normal((T, M)).astype(np.float32)
+    v = rng.standard_normal((T, Dv)).astype(np.float32)
+    lg = rng.standard_normal((T, M)).astype(np.float32)
+    shape = (T, M) if per_slot else (T,)
+    f = (-np.log1p(np.exp(rng.standard_normal(shape))) * fscale).astype(np.float32)
+    return q, k, v, lg, f
+
+
+def _fwd1(q, k, v, lg, f, K, H0=None):
+    """Run the C oracle on one (b,h) stream."""
+    out = oracle.forward(q[None, :, None], k[None, :, None], v[None, :, None], lg[None, :, None],
+                         f[None, :, None], K, None if H0 is None else H0[None, None], nthreads=1)
+    return out["o"][0, :, 0], out["HT"][0, 0], out["idx"][0, :, 0], out["score"][0, :, 0]
+
+
+def _rel(a, b):
+    return float(np.max(np.abs(a - b)) / max(np.sqrt(np.mean(np.square(b))), 1e-300))
+
+
+# ----------------------------------------------------------------------------- golden
+
+
+def test_golden_head_decay():
+    g = json.load(open(os.path.join(GOLDEN, "hand_head_decay_M2.json")))
+    q, k, v, lg = (np.array(g[n], np.float32) for n in ("q", "k", "v", "logits"))
+    f = np.array(g["f"], np.float32)
+    o, HT, idx, score = _fwd1(q, k, v, lg, f, g["K"])
+    assert np.array_equal(idx, np.array(g["expect_idx"]))
+    assert np.allclose(o, np.array(g["expect_o"]), atol=g["tol"], rtol=0)
+    assert np.allclose(HT, np.array(g["expect_HT"]), atol=g["tol"], rtol=0)
+    assert np.allclose(score, np.array(g["expect_score"]), atol=1e-12)
+
+
+def test_golden_slot_decay():
+    g = json.load(open(os.path.join(GOLDEN, "hand_slot_decay_M3.json")))
+    q, k, v, lg = (np.array(g[n], np.float32) for n in ("q", "k", "v", "logits"))
+    f = np.full(lg.shape, -1.0, np.float32)
+    for t, row in enumerate(g["f_slot_targets"]):
+        for i, target in enumerate(row):
+            if target is not None:
+                f[t, i] = math.log(target) / expit(float(lg[t, i]))
+    H0 = np.array(g["H0"], np.float64)
+    o, HT, idx, _ = _fwd1(q, k, v, lg, f, g["K"], H0)
+    assert np.array_equal(idx, np.array(g["expect_idx"]))
+    assert np.allclose(o, np.array(g["expect_o"]), atol=g["tol"], rtol=0)
+    assert np.allclose(HT, np.array(g["expect_HT"]), atol=g["tol"], rtol=0)
+
+
+# ----------------------------------------------------------------------------- TopK
+
+
+def _topk_rows():
+    rng = np.random.default_rng(11)
+    rows = [rng.standard_normal(64).astype(np.float32) for _ in range(50)]
+    rows += [(np.round(4 * rng.standard_normal(64)) / 4).astype(np.float32) for _ in range(50)]
+    rows.append(np.zeros(64, np.float32))                              # all equal -> 0..K-1
+    z = np.zeros(64, np.float32)
+    z[::2] = -0.0                                                      # signed zeros tie
+    rows.append(z)
+    big = (20 + rng.standard_normal(64)).astype(np.float32)           # sigmoid saturates here
+    rows.append(big)
+    near = np.full(64, 1.5, np.float32)
+    bump = rng.random(64) < 0.5
+    near[bump] = np.nextafter(np.float32(1.5), np.float32(2.0))
+    rows.append(near)                                                  # one-ulp differences
+    return np.stack(rows)
+
+
+@pytest.mark.parametrize("K", [1, 5, 16, 63, 64])
+def test_topk_matches_stable_library_sort(K):
+    rows = _topk_rows()
+    idx, score = oracle.route(rows, K)
+    assert np.array_equal(idx, brute.topk_stable(rows, K))
+
+
+def test_topk_tie_rules():
+    idx, _ = oracle.route(np.zeros((1, 32), np.float32), 7)
+    assert list(idx[0]) == list(range(7))                             # all-equal row
+    row = np.array([0.0, -0.0, 0.0, -0.0] + [-1.0] * 28, np.float32)
+    idx, _ = oracle.route(row[None], 3)
+    assert list(idx[0]) == [0, 1, 2]                                  # -0.0 == +0.0
+    row = np.full(32, 30.0, np.float32)
+    row[5] = np.nextafter(np.float32(30.0), np.float32(31.0))
+    idx, score = oracle.route(row[None], 2)
+    assert list(idx[0]) == [5, 0]                                     # order by logit, not score
+    assert score[0, 0] == score[0, 1] or abs(score[0, 0] - score[0, 1]) < 1e-12
+
+
+def test_scores_match_expit():
+    rows = _topk_rows()
+    idx, score = oracle.route(rows, 16)
+    ref = expit(np.take_along_axis(rows.astype(np.float64), idx, axis=1))
+    assert np.max(np.abs(score - ref)) < 1e-15
+
+
+# ----------------------------------------------------------------------------- recurrence
+
+
+@pytest.mark.parametrize("seed", range(6))
+@pytest.mark.parametrize("K", [1, 3, 8])
+@pytest.mark.parametrize("per_slot", [False, True])
+def test_recurrence_matches_quadratic_form(seed, K, per_slot):
+    rng = np.random.default_rng(100 + seed)
+    T, M, Dv = 9, 8, 3
+    q, k, v, lg, f = _rand_stream(rng, T, M, Dv, per_slot)
+    H0 = rng.standard_normal((M, Dv)) if seed % 2 else None
+    o, HT, idx, _ = _fwd1(q, k, v, lg, f, K, H0)
+    ob, HTb = brute.quadratic_form(q, k, v, lg, f, K, H0)
+    assert _rel(o, ob) < 1e-12
+    assert _rel(HT, HTb) < 1e-12
+    assert np.array_equal(idx, brute.topk_stable(lg, K))
+
+
+@pytest.mark.parametrize("per_slot", [False, True])
+def test_dense_limit_is_gated_linear_attention(per_slot):
+    rng = np.random.default_rng(7)
+    T, M, Dv = 12, 6, 4
+    q, k, v, lg, f = _rand_stream(rng, T, M, Dv, per_slot, fscale=0.3)
+    H0 = rng.standard_normal((M, Dv))
+    o, HT, _, _ = _fwd1(q, k, v, lg, f, M, H0)
+    od, HTd = brute.dense_masked_form(q, k, v, lg, f, H0)
+    assert _rel(o, od) < 1e-10
+    assert _rel(HT, HTd) < 1e-10
+
+
+def test_window_limit_is_sliding_window():
+    rng = np.random.default_rng(3)
+    T, M, Dv = 40, 8, 5
+    q = rng.standard_normal((T, M)).astype(np.float32)
+    v = rng.standard_normal((T, Dv)).astype(np.float32)
+    k = np.ones((T, M), np.float32)
+    lg = np.zeros((T, M), np.float32)
+    lg[np.arange(T), np.arange(T) % M] = 10.0
+    f = np.full((T,), -1e4, np.float32)
+    o, HT, idx, _ = _fwd1(q, k, v, lg, f, 1)
+    ow, HTw = brute.window_form(q, v, M)
+    assert np.array_equal(idx[:, 0], np.arange(T) % M)
+    assert _rel(o, ow) < 1e-12
+    assert _rel(HT, HTw) < 1e-12
+
+
+def test_unselected_rows_keep_bits():
+    rng = np.random.default_rng(5)
+    T, M, Dv = 30, 16, 4
+    q, k, v, lg, f = _rand_stream(rng, T, M, Dv, False)
+    lg[:, M // 2:] = -100.0
+    H0 = rng.standard_normal((M, Dv))
+    _, HT, idx, _ = _fwd1(q, k, v, lg, f, 4, H0)
+    assert idx.max() < M // 2
+    assert np.array_equal(HT[M // 2:].view(np.uint64), H0[M // 2:].view(np.uint64))
+
+
+def test_decode_step_is_one_token_forward():
+    rng = np.random.default_rng(9)
+    B, H, M, Dv, K = 2, 3, 8, 4, 3
+    q = rng.standard_normal((B, H, M)).astype(np.float32)
+    k = rng.standard_normal((B, H, M)).astype(np.float32)
+    v = rng.standard_normal((B, H, Dv)).astype(np.float32)
+    lg = rng.standard_normal((B, H, M)).astype(np.float32)
+    f = -np.abs(rng.standard_normal((B, H))).astype(np.float32)
+    st = rng.standard_normal((B, H, M, Dv))
+    out = oracle.decode_step(q, k, v, lg, f, K, st)
+    for b in range(B):
+        for h in range(H):
+            ob, HTb = brute.quadratic_form(q[b, h][None], k[b, h][None], v[b, h][None],
+                                           lg[b, h][None], f[b, h][None], K, st[b, h])
+            assert _rel(out["o"][b, h][None], ob) < 1e-12
+            assert _rel(out["state"][b, h], HTb) < 1e-12
+
+
+def test_split_sequence_resumes():
+    rng = np.random.default_rng(13)
+    T, M, Dv = 50, 16, 8
+    q, k, v, lg, f = _rand_stream(rng, T, M, Dv, True)
+    o, HT, _, _ = _fwd1(q, k, v, lg, f, 4)
+    o1, H1, _, _ = _fwd1(q[:17], k[:17], v[:17], lg[:17], f[:17], 4)
+    o2, H2, _, _ = _fwd1(q[17:], k[17:], v[17:], lg[17:], f[17:], 4, H1)
+    assert np.array_equal(np.concatenate([o1, o2]), o)
+    assert np.array_equal(H2, HT)
+
+
+def test_threads_do_not_change_results():
+    rng = np.random.default_rng(21)
+    B, T, H, M, Dv = 3, 20, 5, 16, 8
+    x = {n: rng.standard_normal(s).astype(np.float32) for n, s in
+         dict(q=(B, T, H, M), k=(B, T, H, M), v=(B, T, H, Dv), logits=(B, T, H, M)).items()}
+    f = -np.abs(rng.standard_normal((B, T, H))).astype(np.float32)
+    a = oracle.forward(x["q"], x["k"], x["v"], x["logits"], f, 4, nthreads=1)
+    b = oracle.forward(x["q"], x["k"], x["v"], x["logits"], f, 4, nthreads=4)
+    assert np.array_equal(a["o"], b["o"]) and np.array_equal(a["HT"], b["HT"])
+
+
+# ----------------------------------------------------------------------------- mutants
+
+# Each mutant plants one plausible mistake in a copy of the oracle source (compiled here, on the
+# CPU, into a scratch directory). The pins above must notice every one of them.
+MUTANTS = {
+    "read_before_write": ("if (J->o) {", "if (0) {", "for (int r = 0; r < K; ++r) {",
+                          "if (J->o) { double* o0 = J->o + row * Dv; for (int d = 0; d < Dv; ++d) o0[d] = 0.0;"
+                          " for (int i = 0; i < M; ++i) { const double* Si = S + (size_t)i * Dv;"
+                          " for (int d = 0; d < Dv; ++d) o0[d] += (double)q[i] * Si[d]; } }\n"
+                          "    for (int r = 0; r < K; ++r) {"),
+    "tie_to_higher_index": ("return a < b;", "return a > b;", None, None),
+    "decay_without_score": ("const double a = exp(s * f);", "const double a = exp(f);", None, None),
+    "write_without_one_minus_a": ("const double wk = (1.0 - a) * (double)k[i];",
+                                  "const double wk = (double)k[i];", None, None),
+    "q_k_swapped_in_read": ("const double qi = (double)q[i];", "const double qi = (double)k[i];",
+                            None, None),
+}
+
+
+def _build_mutant(tmp_path, name):
+    src = open(os.path.join(os.path.dirname(oracle.__file__), "rsm_oracle.c")).read()
+    a, b, c, d = MUTANTS[name]
+    assert a in src
+    src = src.replace(a, b, 1)
+    if c is not None:
+        assert c in src
+        src = src.replace(c, d, 1)
+    path = tmp_path / f"mut_{name}.c"
+    path.write_text(src)
+    so = tmp_path / f"mut_{name}.so"
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread", "-o", str(so),
+                           str(path), "-lm"])
+    return str(so)
+
+
+def _pins_pass_with(lib_path) -> bool:
+    saved = oracle._lib
+    try:
+        lib = ctypes.CDLL(lib_path)
+        f32p = np.ctypeslib.ndpointer(np.float32, flags="C_CONTIGUOUS")
+        vp = ctypes.c_void_p
+        lib.rsmo_forward.argtypes = [ctypes.c_int] * 7 + [f32p] * 5 + [vp] * 5 + [ctypes.c_int]
+        lib.rsmo_route.argtypes = [f32p, ctypes.c_longlong, ctypes.c_int, ctypes.c_int, vp, vp]
+        oracle._lib = lib
+        for fn, args in [(test_golden_head_decay, ()), (test_golden_slot_decay, ()),
+                         (test_topk_tie_rules, ()), (test_window_limit_is_sliding_window, ()),
+                         (test_recurrence_matches_quadratic_form, (1, 3, True)),
+                         (test_recurrence_matches_quadratic_form, (2, 3, False))]:
+            try:
+                fn(*args)
+            except AssertionError:
+                return False
+        return True
+    finally:
+        oracle._lib = saved
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_planted_mistakes(tmp_path, name):
+    assert not _pins_pass_with(_build_mutant(tmp_path, name))
+
+
+def test_pins_pass_with_the_real_oracle():
+    assert _pins_pass_with(oracle.build())
