@@ -1,0 +1,398 @@
+"""Benchmark of the RSM mixer hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one chunked prefill (rsm_forward) of the chosen workload, inputs resident in HBM
+(default: the 32K-token long-context prefill, B=1 T=32768 H=16 M=128 K=16 Dv=128, bf16 q/k/v,
+fp32 logits/state/output). The line also carries the generation-decode measurement
+(rsm_decode_step on 256 sequences x 16 heads, M=128 K=16 Dv=128, state from a 2048-token prefill).
+
+Under torchrun (N > 1) every rank runs its own replica on its own GPU with its own inputs (the
+path shards by sequence with no data exchange), timing is taken on the device with CUDA events,
+and the max over ranks is reported (weak scaling). `--impl reference` times the fp64 CPU oracle
+on bounded samples of the same workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "RSM prefill tokens/s and decode state HBM GB/s on 1 B200; % roofline"
+
+
+def load_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# --------------------------------------------------------------------------- work accounting
+
+def prefill_bytes(w) -> int:
+    """Algorithmic bytes of one prefill: every input read once, o and H_T written once."""
+    es = 2 if w.dtype == "bf16" else 4
+    th = w.B * w.T * w.H
+    b = th * (2 * w.M * es + w.Dv * es + w.M * 4)          # q, k, v, logits
+    b += th * (w.M * 4 if w.decay == "slot" else 4)        # f
+    b += th * w.Dv * 4                                     # o (fp32)
+    b += w.B * w.H * w.M * w.Dv * 4                        # H_T
+    return b
+
+
+def prefill_flops(w, chunk=64) -> int:
+    """Dense-contraction FLOPs of the chunked form: 4*M*Dv + 2*C*(M+Dv) per token-head."""
+    return w.B * w.T * w.H * (4 * w.M * w.Dv + 2 * chunk * (w.M + w.Dv))
+
+
+def decode_bytes(B, H, M, K, Dv, es=2, per_slot=False) -> tuple[int, int]:
+    """(state bytes, total bytes) of one decode step: the state is read once (M rows) and the K
+    selected rows are written; inputs q, k, v, logits, f are read and o is written."""
+    state = B * H * (M + K) * Dv * 4
+    inputs = B * H * (2 * M * es + Dv * es + M * 4 + (M * 4 if per_slot else 4) + Dv * 4)
+    return state, state + inputs
+
+
+# --------------------------------------------------------------------------- clocks
+
+CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+class ClockSampler:
+    """Samples nvidia-smi every 200 ms in the background while the timed region runs."""
+
+    def __init__(self, gpu_index: int):
+        self.path = tempfile.mktemp(prefix="clocks_", suffix=".csv")
+        self.proc = None
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={CLOCK_FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(gpu_index), "-lms", "200"], stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# --------------------------------------------------------------------------- distributed
+
+def dist_setup():
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------------- CPU oracle timing
+
+def oracle_sample(w, seconds_target: float = 12.0) -> dict:
+    """Times the fp64 CPU oracle (as it stands) on a bounded sample of the workload: all heads
+    of sequence 0 over a prefix of the tokens, sized to about `seconds_target` of CPU time."""
+    import numpy as np
+    import torch
+    from oracle import oracle
+    from sparse_routed_slot_b200.workloads import make_inputs
+
+    cores = oracle.default_threads()
+
+    def run(T):
+        x = make_inputs(1, T, w.H, w.M, w.Dv, w.torch_dtype, w.decay, seed=w.seed)
+        c = {n: t.float().numpy() for n, t in x.items()}
+        t0 = time.perf_counter()
+        oracle.forward(c["q"], c["k"], c["v"], c["logits"], c["f"], w.K, want_idx=False, nthreads=cores)
+        return time.perf_counter() - t0
+
+    T0 = min(w.T, 256)
+    dt = run(T0)
+    T1 = int(min(w.T, max(T0, T0 * seconds_target / max(dt, 1e-6))))
+    dt1 = run(T1) if T1 != T0 else dt
+    used = min(cores, w.H)
+    return {"value": T1 / dt1, "unit": "tokens/s", "cores": used, "kind": "oracle",
+            "sample": f"sequence 0, all {w.H} heads, first {T1} of {w.T} tokens, fp64, "
+                      f"{used} threads over heads; {dt1:.1f} s", "seconds": dt1, "tokens": T1}
+
+
+# --------------------------------------------------------------------------- our arm
+
+def run_ours(args, world, rank, local):
+    import torch
+    import sparse_routed_slot_b200 as rsm
+    from sparse_routed_slot_b200 import api
+    from sparse_routed_slot_b200.workloads import WORKLOADS, make_inputs
+
+    w = WORKLOADS[args.workload]
+    dev = torch.device("cuda", local)
+    peaks = load_peaks()
+    x = make_inputs(w.B, w.T, w.H, w.M, w.Dv, w.torch_dtype, w.decay, seed=w.seed + 1000 * rank, device=dev)
+    o = torch.empty(w.B, w.T, w.H, w.Dv, dtype=torch.float32, device=dev)
+    HT = torch.empty(w.B, w.H, w.M, w.Dv, dtype=torch.float32, device=dev)
+    outs = {"o": o, "HT": HT}
+    a = api._forward_args(x["q"], x["k"], x["v"], x["logits"], x["f"], w.K, None, o, HT, None, None,
+                          args.path, False)
+    ws_bytes = api.workspace_bytes(a)
+    path_used = api.selected_path(a)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+
+    def step():
+        rsm.forward(x["q"], x["k"], x["v"], x["logits"], x["f"], w.K, out=outs, workspace=ws,
+                    path=args.path)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = ClockSampler(local)
+    stream = torch.cuda.current_stream(dev)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    torch.cuda.synchronize()
+    barrier(world)
+    ev[0].record(stream)
+    for i in range(args.steps):
+        step()
+        ev[i + 1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    per = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
+    ms = sum(per) / len(per)
+    ms_max = max_over_ranks(ms, world)
+    tokens = w.B * w.T
+    value = tokens * world / (ms_max * 1e-3)
+
+    # end to end through the public call with host buffers: pinned inputs copied in, result out
+    host_in = {n: t.cpu().pin_memory() for n, t in x.items()}
+    dev_in = {n: torch.empty_like(t) for n, t in x.items()}
+    host_o = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    host_HT = torch.empty(HT.shape, dtype=HT.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = host_o.numel() * 4 + host_HT.numel() * 4
+
+    def e2e_step():
+        for n in dev_in:
+            dev_in[n].copy_(host_in[n], non_blocking=True)
+        rsm.forward(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["logits"], dev_in["f"], w.K,
+                    out=outs, workspace=ws, path=args.path)
+        host_o.copy_(o, non_blocking=True)
+        host_HT.copy_(HT, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+    del host_in, dev_in
+
+    nbytes = prefill_bytes(w)
+    achieved = nbytes / (ms * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32" if path_used == "simt" else "tf32", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "M": w.M, "K": w.K, "Dv": w.Dv,
+                   "decay": w.decay, "qkv_dtype": w.dtype, "state_dtype": "f32", "o_dtype": "f32",
+                   "path": path_used, "parallelism": f"replicas{world}",
+                   "l2": f"inputs larger than L2 ({nbytes / 1e6:.0f} MB per step, no flush)"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                     "algorithmic_bytes": nbytes, "kernel": "rsm prefill (single launch per step)",
+                     "peak_source": peaks["source"],
+                     "tensor_tflops": prefill_flops(w) / (ms * 1e-3) / 1e12},
+        "e2e": {"value": tokens * world / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": args.steps * launches_per_forward(path_used),
+        "clocks": clk,
+    }
+    if not args.no_decode:
+        line["decode"] = run_decode(args, world, rank, local, peaks)
+    if rank == 0 and not args.no_cpu:
+        line["cpu_baseline"] = oracle_sample(w)
+    return line
+
+
+def launches_per_forward(path):
+    return 1
+
+
+def run_decode(args, world, rank, local, peaks) -> dict:
+    """Generation decode: 256 sequences x 16 heads, state from a 2048-token prefill, then
+    `decode_steps` timed rsm_decode_step calls (default 256 of the 1024-step workload)."""
+    import torch
+    import sparse_routed_slot_b200 as rsm
+    from sparse_routed_slot_b200.workloads import WORKLOADS, make_inputs
+
+    w = WORKLOADS["decode_256x16"]
+    dev = torch.device("cuda", local)
+    state = torch.zeros(w.B, w.H, w.M, w.Dv, dtype=torch.float32, device=dev)
+    # prefill in groups of 32 sequences (bounded input memory)
+    for b0 in range(0, w.B, 32):
+        x = make_inputs(32, w.decode_prefill_T, w.H, w.M, w.Dv, w.torch_dtype, w.decay,
+                        seed=w.seed + b0 + 1000 * rank, device=dev)
+        out = rsm.forward(x["q"], x["k"], x["v"], x["logits"], x["f"], w.K, state=True, path=args.path)
+        state[b0:b0 + 32].copy_(out["HT"])
+        del x, out
+    nsteps = args.decode_steps
+    d = make_inputs(nsteps, w.B, w.H, w.M, w.Dv, w.torch_dtype, w.decay, seed=w.seed + 7 + 1000 * rank,
+                    device=dev)
+    o = torch.empty(w.B, w.H, w.Dv, dtype=torch.float32, device=dev)
+
+    def step(i):
+        rsm.decode_step(d["q"][i], d["k"][i], d["v"][i], d["logits"][i], d["f"][i], w.K, state, o=o)
+
+    for i in range(3):
+        step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(nsteps):
+        step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1) / nsteps, world)
+    sb, tb = decode_bytes(w.B, w.H, w.M, w.K, w.Dv, 2, w.decay == "slot")
+    state_gbs = sb / (ms * 1e-3) / 1e9
+    total_gbs = tb / (ms * 1e-3) / 1e9
+    return {"value": state_gbs * world, "unit": "GB/s (state, all GPUs)", "ms_per_step": ms,
+            "steps_timed": nsteps, "total_gbs": total_gbs * world,
+            "roofline": {"bound": "hbm", "achieved": total_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": total_gbs / peaks["hbm_gbs"], "traffic": None,
+                         "algorithmic_bytes": tb, "kernel": "rsm decode step"},
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "M": w.M, "K": w.K, "Dv": w.Dv,
+                       "prefill_T": w.decode_prefill_T, "graph": False,
+                       "l2": f"state {w.B * w.H * w.M * w.Dv * 4 / 1e6:.0f} MB > L2"}}
+
+
+# --------------------------------------------------------------------------- reference arm
+
+def run_reference(args, world, rank) -> dict | None:
+    from sparse_routed_slot_b200.workloads import WORKLOADS
+    if rank != 0:
+        return None
+    w = WORKLOADS[args.workload]
+    for _ in range(args.warmup):
+        oracle_sample(w, seconds_target=2.0)
+    vals, secs = [], 0.0
+    last = None
+    for _ in range(args.steps):
+        last = oracle_sample(w, seconds_target=6.0)
+        vals.append(last["value"])
+        secs += last["seconds"]
+    value = sum(vals) / len(vals)
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * last["tokens"] / value,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "M": w.M, "K": w.K, "Dv": w.Dv,
+                       "decay": w.decay, "qkv_dtype": w.dtype},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": last["cores"], "kind": "oracle",
+                             "sample": last["sample"]},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="long_ctx_bf16")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--path", default="auto", choices=["auto", "simt", "tensor"])
+    ap.add_argument("--decode-steps", type=int, default=256)
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        line = run_reference(args, world, rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+
+    world, rank, local = dist_setup()
+    line = run_ours(args, world, rank, local)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

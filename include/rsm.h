@@ -1,0 +1,178 @@
+/*
+ * rsm.h -- C ABI of librsm, a B200 (sm_100a) implementation of the routing-state-model (RSM)
+ * sequence mixer of Raven ("Raven: High-Recall Sequence Modeling with Sparse Memory Routing").
+ *
+ * The mixer, per batch b, head h and token t (Raven README, github.com/xiaol/SelectingMemory,
+ * "How Raven Works"):
+ *   S_t      = the K of M slots with the largest router logits (ties: lower slot index first)
+ *   s_i      = sigmoid(logit_i)                         for i in S_t, 0 otherwise
+ *   a_i      = exp(s_i * f)                             f = per-head or per-slot log-decay, f <= 0
+ *   H[i,:]   = a_i * H[i,:] + (1 - a_i) * k_i * v       for i in S_t; other rows keep their bits
+ *   o_t      = sum_i q_i * H[i,:]                       (read after the write)
+ * with a state H of M slot rows by Dv columns per (b,h). "Model Structure" of the same README
+ * names the two decay families (Mamba2: one log-decay per head and token; GLA: one per slot) and
+ * the two kernels (chunked for training/prefill, fused recurrent for generation).
+ *
+ * Conventions for every entry point:
+ *   - The caller owns all memory. Pointers are DEVICE pointers unless stated otherwise, 16-byte
+ *     aligned, row-major and contiguous in the layouts given below. The library never allocates.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream). Work is
+ *     enqueued asynchronously; argument errors are returned synchronously before any launch,
+ *     and a failed launch returns RSM_ERR_CUDA. rsm_last_error() describes the last failure of
+ *     the calling host thread.
+ *   - Logits and f must be finite and f <= 0 (a very negative finite f stands for "forget").
+ *     These are preconditions; they are checked only when RSM_FLAG_VALIDATE is set.
+ *   - Slots not selected at a step (decode) or in the whole call (prefill) are left bit-identical
+ *     in the state.
+ *   - Supported sizes: 32 <= M <= 256 with M a power of two, 1 <= K <= M, 1 <= Dv <= 256 with
+ *     Dv % 4 == 0. Other sizes return RSM_ERR_UNSUPPORTED.
+ */
+#ifndef RSM_H_
+#define RSM_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define RSM_API __attribute__((visibility("default")))
+#else
+#define RSM_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum rsm_status {
+  RSM_OK = 0,
+  RSM_ERR_INVALID_ARG = 1,  /* null pointer where one is required, bad size, misalignment */
+  RSM_ERR_UNSUPPORTED = 2,  /* valid arguments outside the sizes this build implements */
+  RSM_ERR_CUDA = 3,         /* a CUDA call or launch failed; see rsm_last_error() */
+  RSM_ERR_NONFINITE = 4,    /* RSM_FLAG_VALIDATE found a non-finite logit or a non-finite/positive f */
+  RSM_ERR_WORKSPACE = 5,    /* workspace missing or smaller than rsm_forward_workspace_size() */
+  RSM_ERR_TIMEOUT = 6       /* a bounded device wait gave up (reported by rsm_get_device_status) */
+} rsm_status;
+
+typedef enum rsm_dtype { RSM_F32 = 0, RSM_BF16 = 1 } rsm_dtype;
+
+typedef enum rsm_decay {
+  RSM_DECAY_HEAD = 0,  /* f has one value per (b,t,h): Mamba2-style scalar log-decay            */
+  RSM_DECAY_SLOT = 1   /* f has one value per (b,t,h,slot): GLA-style per-slot log-decay         */
+} rsm_decay;
+
+typedef enum rsm_path {
+  RSM_PATH_AUTO = 0,    /* tensor-core path when the shape allows it, else the CUDA-core path    */
+  RSM_PATH_SIMT = 1,    /* CUDA-core fp32 chunked path (any supported size, any input dtype)     */
+  RSM_PATH_TENSOR = 2   /* tcgen05/TMEM tensor-core path; RSM_ERR_UNSUPPORTED when not available */
+} rsm_path;
+
+enum { RSM_FLAG_VALIDATE = 1 };
+
+/* ---------------------------------------------------------------------------------------------
+ * rsm_route -- TopK routing of router logits.
+ *   Raven README "How Raven Works" (route_scores = TopK(sigmoid(r_proj(x)))); paperlayer.ai summary
+ *   section 4.1 (keep the top-K scores, set the rest to zero). Ranking is on the fp32 logits
+ *   (sigmoid is monotone and saturates in fp32); exact ties go to the lower slot index, and
+ *   -0.0 ties +0.0.
+ *   logits    [rows, M] fp32 (device)
+ *   idx_out   [rows, K] int32 (device): selected slots in rank order (logit desc, index asc)
+ *   score_out [rows, K] fp32 (device, may be NULL): sigmoid(logit) of each selected slot
+ *   rows may be 0 (nothing is launched).
+ * ------------------------------------------------------------------------------------------- */
+RSM_API rsm_status rsm_route(const float* logits, int64_t rows, int M, int K, int32_t* idx_out,
+                     float* score_out, void* stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * rsm_forward -- chunked prefill over T tokens.
+ *   The recurrence above, evaluated chunk by chunk (paperlayer.ai summary, section A.5: the
+ *   sequence is split into n chunks of length C, T = n*C, for stability and parallelism; a
+ *   ragged last chunk is allowed here). The result does not depend on the chunk length beyond
+ *   rounding.
+ *   q, k    [B,T,H,M] in qkv_dtype (fp32 or bf16)
+ *   v       [B,T,H,Dv] in qkv_dtype
+ *   logits  [B,T,H,M] fp32
+ *   f       [B,T,H] fp32 (RSM_DECAY_HEAD) or [B,T,H,M] fp32 (RSM_DECAY_SLOT)
+ *   H0      [B,H,M,Dv] fp32 initial state, or NULL for zeros. May alias HT.
+ *   o       [B,T,H,Dv] fp32 output (required)
+ *   HT      [B,H,M,Dv] fp32 final state, or NULL to skip
+ *   idx_out, score_out  [B,T,H,K] (int32, fp32), or NULL to skip: the routing of every token
+ *   workspace / workspace_bytes: device scratch of at least rsm_forward_workspace_size(args)
+ *     bytes (256-byte aligned); may be NULL when that size is 0. Its contents are not preserved.
+ *   path: which implementation to run (RSM_PATH_AUTO normally).
+ * ------------------------------------------------------------------------------------------- */
+typedef struct rsm_forward_args {
+  int B, T, H, M, K, Dv;
+  rsm_dtype qkv_dtype;
+  rsm_decay decay;
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* logits;
+  const float* f;
+  const float* H0;
+  float* o;
+  float* HT;
+  int32_t* idx_out;
+  float* score_out;
+  void* workspace;
+  size_t workspace_bytes;
+  rsm_path path;
+  int flags; /* RSM_FLAG_* */
+} rsm_forward_args;
+
+/* Bytes of device workspace rsm_forward needs for these arguments (0 when none). Depends only on
+ * the sizes, dtype, decay and path fields. Returns (size_t)-1 for arguments rsm_forward rejects. */
+RSM_API size_t rsm_forward_workspace_size(const rsm_forward_args* args);
+RSM_API rsm_status rsm_forward(const rsm_forward_args* args, void* stream);
+
+/* The implementation rsm_forward would run for these arguments: RSM_PATH_SIMT or RSM_PATH_TENSOR
+ * (RSM_PATH_AUTO resolved), or -1 for arguments rsm_forward rejects. Host-only. */
+RSM_API int rsm_forward_selected_path(const rsm_forward_args* args);
+
+/* ---------------------------------------------------------------------------------------------
+ * rsm_decode_step -- one generation token per (b,h): fused routing, sparse decay/write of the K
+ *   selected rows of the carried state in place, and the read o = q.H over all M rows.
+ *   Raven README "Model Structure" (fused recurrent computation for inference).
+ *   q, k    [B,H,M] in qkv_dtype;  v [B,H,Dv] in qkv_dtype
+ *   logits  [B,H,M] fp32;          f [B,H] or [B,H,M] fp32
+ *   state   [B,H,M,Dv] fp32, read and updated in place (only the K selected rows are written)
+ *   o       [B,H,Dv] fp32 output
+ *   idx_out, score_out [B,H,K] or NULL
+ * ------------------------------------------------------------------------------------------- */
+typedef struct rsm_decode_args {
+  int B, H, M, K, Dv;
+  rsm_dtype qkv_dtype;
+  rsm_decay decay;
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* logits;
+  const float* f;
+  float* state;
+  float* o;
+  int32_t* idx_out;
+  float* score_out;
+  int flags; /* RSM_FLAG_* */
+} rsm_decode_args;
+
+RSM_API rsm_status rsm_decode_step(const rsm_decode_args* args, void* stream);
+
+/* Human-readable name of a status code (static storage). */
+RSM_API const char* rsm_status_string(rsm_status status);
+
+/* Detail of the last failure on the calling host thread ("" if none). */
+RSM_API const char* rsm_last_error(void);
+
+/* Synchronizes `stream`, then reads and clears the library's device status word for the current
+ * device: RSM_OK, RSM_ERR_NONFINITE (validation found bad inputs) or RSM_ERR_TIMEOUT (a bounded
+ * device wait expired). Errors of the synchronization itself return RSM_ERR_CUDA. */
+RSM_API rsm_status rsm_get_device_status(void* stream);
+
+/* Library version as major*10000 + minor*100 + patch. */
+RSM_API int rsm_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RSM_H_ */

@@ -1,0 +1,25 @@
+// kernels.h -- launch functions of the librsm kernels (internal; the public ABI is rsm.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "rsm.h"
+
+namespace rsm {
+
+cudaError_t launch_route(const float* logits, int64_t rows, int M, int K, int32_t* idx_out,
+                         float* score_out, int validate, cudaStream_t stream);
+
+cudaError_t launch_decode(const rsm_decode_args& a, cudaStream_t stream);
+
+// CUDA-core fp32 chunked prefill (any supported size).
+cudaError_t launch_prefill_simt(const rsm_forward_args& a, cudaStream_t stream);
+size_t prefill_simt_smem_bytes(int M, int Dv);
+
+// tcgen05 tensor-core chunked prefill. `supported` tells whether the shape/dtype can run there.
+bool prefill_tc_supported(const rsm_forward_args& a);
+size_t prefill_tc_workspace_bytes(const rsm_forward_args& a);
+cudaError_t launch_prefill_tc(const rsm_forward_args& a, cudaStream_t stream);
+
+}  // namespace rsm

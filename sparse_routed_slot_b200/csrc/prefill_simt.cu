@@ -1,0 +1,255 @@
+// prefill_simt.cu -- chunked prefill on CUDA cores in fp32 (rsm_forward, RSM_PATH_SIMT).
+//
+// The fp32 path (1e-4 parity class) and the fallback for sizes the tensor-core path does not
+// cover. One CTA owns one (b,h) stream and one tile of DT state columns, and walks the sequence
+// in chunks of C = 32 tokens with its state tile resident in shared memory.
+//
+// Chunk algebra (paperlayer.ai summary, section A.5: chunkwise computation over T = n*C tokens),
+// with g_{t,i} the cumulative log-decay of slot i from the chunk start through token t
+// (g <= 0, non-increasing in t), w_{t,i} = k_{t,i} (1 - a_{t,i}) on the selected slots:
+//   o_t   = (q_t * e^{g_t}) . H_start  +  sum_{s<=t} A_{t,s} v_s
+//   A_{t,s} = sum_{i in S_s} q_{t,i} w_{s,i} e^{g_{t,i} - g_{s,i}}        (pairwise, sparse)
+//   H_end = e^{g_C} * H_start + sum_s (w_s * e^{g_C - g_s}) (x) v_s
+// Every exponential has a non-positive argument, so the path is exact in structure for any
+// finite decay (no overflow, underflow only of terms that are truly negligible). Rows never
+// selected in a chunk are skipped, so they keep their bits.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace rsm {
+
+namespace {
+
+constexpr int kC = 32;          // tokens per chunk
+constexpr int kThreads = 256;
+
+__host__ __device__ inline int simt_dt(int M, int Dv) {
+  const int dt = M >= 256 ? 32 : 64;
+  return Dv < dt ? Dv : dt;
+}
+
+struct SimtSmem {
+  // float offsets into the dynamic shared buffer
+  int g, q, qh, w, H, v, A, gC, D;
+  int bytes_f;     // floats used by the above
+  int sidx, touch; // byte offsets of the uint8 rank table and the int touch flags
+  int total;       // bytes
+};
+
+__host__ __device__ inline SimtSmem simt_layout(int M, int DT) {
+  SimtSmem s;
+  int off = 0;
+  s.g = off;  off += kC * M;
+  s.q = off;  off += kC * M;
+  s.qh = off; off += kC * M;
+  s.w = off;  off += kC * M;
+  s.H = off;  off += M * DT;
+  s.v = off;  off += kC * DT;
+  s.A = off;  off += kC * kC;
+  s.gC = off; off += M;
+  s.D = off;  off += M;
+  s.bytes_f = off;
+  int b = off * 4;
+  s.touch = b; b += M * 4;
+  s.sidx = b; b += kC * M;
+  s.total = (b + 15) & ~15;
+  return s;
+}
+
+template <int M, typename TIn>
+__global__ void __launch_bounds__(kThreads) prefill_simt_kernel(rsm_forward_args a, int DT) {
+  constexpr int E = M / 32;
+  extern __shared__ __align__(16) unsigned char smem[];
+  const SimtSmem L = simt_layout(M, DT);
+  float* sf = reinterpret_cast<float*>(smem);
+  float* s_g = sf + L.g;
+  float* s_q = sf + L.q;
+  float* s_qh = sf + L.qh;
+  float* s_w = sf + L.w;
+  float* s_H = sf + L.H;
+  float* s_v = sf + L.v;
+  float* s_A = sf + L.A;
+  float* s_gC = sf + L.gC;
+  float* s_D = sf + L.D;
+  int* s_touch = reinterpret_cast<int*>(smem + L.touch);
+  unsigned char* s_sidx = smem + L.sidx;
+
+  const int T = a.T, H = a.H, K = a.K, Dv = a.Dv;
+  const int pair = blockIdx.x;
+  const int b = pair / H, h = pair % H;
+  const int d0 = blockIdx.y * DT;
+  const int DTe = min(DT, Dv - d0);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const bool route_owner = blockIdx.y == 0;  // only one column tile writes the routing outputs
+  const bool validate = (a.flags & RSM_FLAG_VALIDATE) && route_owner;
+
+  const TIn* q = reinterpret_cast<const TIn*>(a.q);
+  const TIn* k = reinterpret_cast<const TIn*>(a.k);
+  const TIn* v = reinterpret_cast<const TIn*>(a.v);
+
+  // initial state tile
+  for (int p = tid; p < M * DT; p += kThreads) {
+    const int i = p / DT, dd = p % DT;
+    s_H[p] = (dd < DTe && a.H0) ? a.H0[((int64_t)pair * M + i) * Dv + d0 + dd] : 0.f;
+  }
+
+  for (int c0 = 0; c0 < T; c0 += kC) {
+    const int nrows = min(kC, T - c0);
+    for (int i = tid; i < M; i += kThreads) s_touch[i] = 0;
+    __syncthreads();
+
+    // --- routing, log-decay and write weights of the chunk's rows (one warp per row)
+    for (int t = warp; t < kC; t += kThreads / 32) {
+      if (t < nrows) {
+        const int64_t row = ((int64_t)b * T + c0 + t) * H + h;
+        float x[E];
+        load_row_logits<M>(a.logits + row * M, lane, x);
+        float fv[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e)
+          fv[e] = (a.decay == RSM_DECAY_SLOT) ? a.f[row * M + lane * E + e] : a.f[row];
+        if (validate) {
+          bool bad = false;
+#pragma unroll
+          for (int e = 0; e < E; ++e) bad |= !finite_f32(x[e]) || !finite_f32(fv[e]) || fv[e] > 0.f;
+          if (__any_sync(kFull, bad) && lane == 0) raise_status(RSM_ERR_NONFINITE);
+        }
+        int32_t* io = (route_owner && a.idx_out) ? a.idx_out + row * K : nullptr;
+        float* so = (route_owner && a.score_out) ? a.score_out + row * K : nullptr;
+        const uint32_t sel = warp_topk<M>(x, K, lane, [&](int r, int slot, int e) {
+          s_sidx[t * M + r] = (unsigned char)slot;
+          if (io) io[r] = slot;
+          if (so) so[r] = sigmoid_f32(x[e]);
+        });
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const int i = lane * E + e;
+          s_q[t * M + i] = In<TIn>::ld(q + row * M + i);
+          if (sel & (1u << e)) {
+            const float lam = sigmoid_f32(x[e]) * fv[e];
+            s_g[t * M + i] = lam;
+            s_w[t * M + i] = In<TIn>::ld(k + row * M + i) * (-expm1f(lam));
+            s_touch[i] = 1;
+          } else {
+            s_g[t * M + i] = 0.f;
+            s_w[t * M + i] = 0.f;
+          }
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const int i = lane * E + e;
+          s_q[t * M + i] = 0.f;
+          s_g[t * M + i] = 0.f;
+          s_w[t * M + i] = 0.f;
+        }
+      }
+    }
+    for (int p = tid; p < kC * DT; p += kThreads) {
+      const int t = p / DT, dd = p % DT;
+      s_v[p] = (t < nrows && dd < DTe)
+                   ? In<TIn>::ld(v + (((int64_t)b * T + c0 + t) * H + h) * Dv + d0 + dd)
+                   : 0.f;
+    }
+    __syncthreads();
+
+    // --- cumulative log-decay per slot, q scaled to the chunk start, chunk decay
+    for (int i = tid; i < M; i += kThreads) {
+      float g = 0.f;
+      for (int t = 0; t < kC; ++t) {
+        g += s_g[t * M + i];
+        s_g[t * M + i] = g;
+        s_qh[t * M + i] = s_q[t * M + i] * expf(g);
+      }
+      s_gC[i] = g;
+      s_D[i] = expf(g);
+    }
+    __syncthreads();
+
+    // --- intra-chunk weights A[t][s], s <= t (sparse over the K slots written at s)
+    for (int p = tid; p < kC * kC; p += kThreads) {
+      const int t = p / kC, s = p % kC;
+      float acc = 0.f;
+      if (s <= t && t < nrows) {
+        for (int r = 0; r < K; ++r) {
+          const int j = s_sidx[s * M + r];
+          acc = fmaf(s_q[t * M + j] * s_w[s * M + j], expf(s_g[t * M + j] - s_g[s * M + j]), acc);
+        }
+      }
+      s_A[p] = acc;
+    }
+    __syncthreads();
+
+    // --- outputs of the chunk for this column tile
+    for (int p = tid; p < kC * DT; p += kThreads) {
+      const int t = p / DT, dd = p % DT;
+      if (t < nrows && dd < DTe) {
+        float acc = 0.f;
+        const float* qh = s_qh + t * M;
+        for (int i = 0; i < M; ++i) acc = fmaf(qh[i], s_H[i * DT + dd], acc);
+        for (int s = 0; s <= t; ++s) acc = fmaf(s_A[t * kC + s], s_v[s * DT + dd], acc);
+        a.o[(((int64_t)b * T + c0 + t) * H + h) * Dv + d0 + dd] = acc;
+      }
+    }
+    // --- write weights carried to the chunk end (non-positive exponents)
+    for (int p = tid; p < kC * M; p += kThreads) {
+      const int t = p / M, i = p % M;
+      const float w = s_w[p];
+      if (w != 0.f) s_w[p] = w * expf(s_gC[i] - s_g[t * M + i]);
+    }
+    __syncthreads();
+
+    // --- state carry; slots not selected in this chunk are left untouched
+    for (int p = tid; p < M * DT; p += kThreads) {
+      const int i = p / DT, dd = p % DT;
+      if (s_touch[i]) {
+        float acc = s_D[i] * s_H[p];
+        for (int t = 0; t < kC; ++t) acc = fmaf(s_w[t * M + i], s_v[t * DT + dd], acc);
+        s_H[p] = acc;
+      }
+    }
+    __syncthreads();
+  }
+
+  if (a.HT) {
+    for (int p = tid; p < M * DT; p += kThreads) {
+      const int i = p / DT, dd = p % DT;
+      if (dd < DTe) a.HT[((int64_t)pair * M + i) * Dv + d0 + dd] = s_H[p];
+    }
+  }
+}
+
+template <int M, typename TIn>
+cudaError_t launch_simt(const rsm_forward_args& a, cudaStream_t stream) {
+  const int DT = simt_dt(M, a.Dv);
+  const SimtSmem L = simt_layout(M, DT);
+  auto kern = prefill_simt_kernel<M, TIn>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L.total);
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)(a.B * a.H), (unsigned)((a.Dv + DT - 1) / DT));
+  kern<<<grid, kThreads, L.total, stream>>>(a, DT);
+  return cudaGetLastError();
+}
+
+template <int M>
+cudaError_t launch_simt_m(const rsm_forward_args& a, cudaStream_t stream) {
+  return a.qkv_dtype == RSM_BF16 ? launch_simt<M, __nv_bfloat16>(a, stream)
+                                 : launch_simt<M, float>(a, stream);
+}
+
+}  // namespace
+
+size_t prefill_simt_smem_bytes(int M, int Dv) { return (size_t)simt_layout(M, simt_dt(M, Dv)).total; }
+
+cudaError_t launch_prefill_simt(const rsm_forward_args& a, cudaStream_t stream) {
+  if (a.B * a.H == 0) return cudaSuccess;
+  switch (a.M) {
+    case 32: return launch_simt_m<32>(a, stream);
+    case 64: return launch_simt_m<64>(a, stream);
+    case 128: return launch_simt_m<128>(a, stream);
+    case 256: return launch_simt_m<256>(a, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace rsm
