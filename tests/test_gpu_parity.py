@@ -119,7 +119,12 @@ def test_decode_steps_match_oracle(rsm, M, Dv, dtype, decay):
 # ------------------------------------------------------------------------------------ prefill
 
 
-PATHS = ["simt", "auto"]
+PATHS = ["simt", "auto", "tensor"]
+
+
+def tensor_ok(path, M, Dv, dtype, K=16):
+    """The tensor-core path covers bf16 q/k/v with M = Dv = 128 and K <= 32."""
+    return path != "tensor" or (M == 128 and Dv == 128 and dtype == torch.bfloat16 and K <= 32)
 
 
 @pytest.mark.parametrize("path", PATHS)
@@ -128,6 +133,8 @@ PATHS = ["simt", "auto"]
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 @pytest.mark.parametrize("decay", ["head", "slot"])
 def test_forward_matches_oracle(rsm, path, M, K, Dv, T, dtype, decay):
+    if not tensor_ok(path, M, Dv, dtype, K):
+        pytest.skip("shape not on the tensor-core path")
     B, H = 2, 3
     x = make_inputs(B, T, H, M, Dv, dtype, decay, seed=M + K + T, device="cuda", h0=True)
     out = rsm.forward(x["q"], x["k"], x["v"], x["logits"], x["f"], K, x["H0"], routing=True, path=path)
@@ -191,10 +198,13 @@ def test_forward_unselected_slots_keep_bits(rsm, path):
 
 
 @pytest.mark.parametrize("path", PATHS)
-def test_forward_window_limit(rsm, path):
+@pytest.mark.parametrize("M,Dv", [(64, 64), (128, 128)])
+def test_forward_window_limit(rsm, path, M, Dv):
     """K=1, a one-hot cyclic router and f = -1e4: the slot store becomes a window of the last M
     tokens, o_t = sum_{s=t-M+1..t} q_{t, s mod M} v_s (exercises extreme decays)."""
-    B, T, H, M, Dv = 1, 300, 2, 64, 64
+    if not tensor_ok(path, M, Dv, torch.bfloat16, 1):
+        pytest.skip("shape not on the tensor-core path")
+    B, T, H = 1, 300, 2
     dev = torch.device("cuda")
     g = torch.Generator(device=dev).manual_seed(4)
     q = torch.randn(B, T, H, M, generator=g, device=dev).bfloat16()
@@ -231,3 +241,65 @@ def test_workload_parity(rsm, name):
     eo, eh = rel(out["o"].cpu().numpy(), r["o"]), rel(out["HT"].cpu().numpy(), r["HT"])
     print(f"{name}: o {eo:.3e} H_T {eh:.3e}")
     assert eo <= tol and eh <= tol
+
+
+# ------------------------------------------------------------------------------------ tensor path
+
+
+@pytest.mark.parametrize("T", [1000, 4096 + 77])
+@pytest.mark.parametrize("decay", ["head", "slot"])
+def test_tensor_segments_match_oracle(rsm, T, decay):
+    """Few (b,h) streams and a long sequence: the sequence is split into segments (summary pass,
+    scan of segment states, main pass). Random initial state."""
+    B, H, M, K, Dv = 1, 2, 128, 16, 128
+    x = make_inputs(B, T, H, M, Dv, torch.bfloat16, decay, seed=T, device="cuda", h0=True)
+    out = rsm.forward(x["q"], x["k"], x["v"], x["logits"], x["f"], K, x["H0"], routing=True, path="tensor")
+    torch.cuda.synchronize()
+    c = host(x)
+    r = oracle.forward(c["q"], c["k"], c["v"], c["logits"], c["f"], K, c["H0"])
+    assert np.array_equal(out["idx"].cpu().numpy(), r["idx"])
+    eo, eh = rel(out["o"].cpu().numpy(), r["o"]), rel(out["HT"].cpu().numpy(), r["HT"])
+    print(f"T={T} {decay}: o {eo:.3e} H_T {eh:.3e}")
+    assert eo <= TOL_BF16 and eh <= TOL_BF16
+
+
+def test_tensor_segments_with_aliased_state(rsm):
+    """H0 and HT are the same buffer while several segments run in parallel."""
+    B, T, H, M, K, Dv = 1, 1500, 2, 128, 16, 128
+    x = make_inputs(B, T, H, M, Dv, torch.bfloat16, "head", seed=77, device="cuda", h0=True)
+    c = host(x)
+    st = x["H0"].clone()
+    out = rsm.forward(x["q"], x["k"], x["v"], x["logits"], x["f"], K, st, path="tensor", out={"HT": st})
+    torch.cuda.synchronize()
+    r = oracle.forward(c["q"], c["k"], c["v"], c["logits"], c["f"], K, c["H0"])
+    assert rel(out["o"].cpu().numpy(), r["o"]) <= TOL_BF16
+    assert rel(st.cpu().numpy(), r["HT"]) <= TOL_BF16
+
+
+def test_tensor_mixed_fast_and_exact_chunks(rsm):
+    """Some tokens forget almost everything (f = -1e4): their chunks take the exact path while
+    the others take the tensor-core path; results still match the oracle."""
+    B, T, H, M, K, Dv = 2, 700, 2, 128, 16, 128
+    x = make_inputs(B, T, H, M, Dv, torch.bfloat16, "head", seed=5, device="cuda", h0=True)
+    x["f"][:, 100:110] = -1e4
+    x["f"][:, 333] = -200.0
+    out = rsm.forward(x["q"], x["k"], x["v"], x["logits"], x["f"], K, x["H0"], path="tensor")
+    torch.cuda.synchronize()
+    c = host(x)
+    r = oracle.forward(c["q"], c["k"], c["v"], c["logits"], c["f"], K, c["H0"])
+    eo, eh = rel(out["o"].cpu().numpy(), r["o"]), rel(out["HT"].cpu().numpy(), r["HT"])
+    print(f"mixed: o {eo:.3e} H_T {eh:.3e}")
+    assert eo <= TOL_BF16 and eh <= TOL_BF16
+
+
+def test_tensor_path_is_selected_for_supported_shapes(rsm):
+    from sparse_routed_slot_b200 import api
+    x = make_inputs(1, 64, 1, 128, 128, torch.bfloat16, "head", seed=1, device="cuda")
+    o = torch.empty(1, 64, 1, 128, device="cuda")
+    a = api._forward_args(x["q"], x["k"], x["v"], x["logits"], x["f"], 16, None, o, None, None, None,
+                          "auto", False)
+    assert api.selected_path(a) == "tensor"
+    y = make_inputs(1, 64, 1, 128, 128, torch.float32, "head", seed=1, device="cuda")
+    a = api._forward_args(y["q"], y["k"], y["v"], y["logits"], y["f"], 16, None, o, None, None, None,
+                          "auto", False)
+    assert api.selected_path(a) == "simt"
