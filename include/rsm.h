@@ -130,6 +130,27 @@ RSM_API rsm_status rsm_forward(const rsm_forward_args* args, void* stream);
 RSM_API int rsm_forward_selected_path(const rsm_forward_args* args);
 
 /* ---------------------------------------------------------------------------------------------
+ * rsm_forward_noalloc -- rsm_forward for callers that cannot allocate device memory.
+ *   The pages have no counterpart to this call; it exists for callers with no way to allocate:
+ *   work recorded into a CUDA graph capture (an allocation would break the capture), programs
+ *   whose allocator owns every byte of the device, or runtimes with a fixed memory plan. Where
+ *   rsm_forward needs a caller-supplied workspace (long sequences split into segments), this call
+ *   uses a scratch array built into the library instead; the caller passes only the inputs and
+ *   outputs (args->workspace and args->workspace_bytes are ignored). Results are those of
+ *   rsm_forward.
+ *   Limit: the scratch holds rsm_forward_noalloc_max_scratch() bytes (16 MiB); sizes whose
+ *   workspace would exceed it return RSM_ERR_WORKSPACE with the sizes in rsm_last_error().
+ *   The array occupies device memory on every GPU that loads the library, until exit. The first
+ *   call on each device looks up the array's device address (cudaGetSymbolAddress) with that
+ *   device current; make that first call before any stream capture. All calls share the array
+ *   and it keeps the last call's contents (nothing in it needs to start at zero): calls whose
+ *   GPU work overlaps in time, on any streams or host threads of one device, race and must not
+ *   be issued. No CUDA allocation routine is called.
+ * ------------------------------------------------------------------------------------------- */
+RSM_API rsm_status rsm_forward_noalloc(const rsm_forward_args* args, void* stream);
+RSM_API size_t rsm_forward_noalloc_max_scratch(void);
+
+/* ---------------------------------------------------------------------------------------------
  * rsm_decode_step -- one generation token per (b,h): fused routing, sparse decay/write of the K
  *   selected rows of the carried state in place, and the read o = q.H over all M rows.
  *   Raven README "Model Structure" (fused recurrent computation for inference).

@@ -21,7 +21,8 @@ RSM_FLAG_VALIDATE = 1
 # Every symbol include/rsm.h declares (the CPU tests check the library exports all of them).
 EXPORTED = ("rsm_route", "rsm_forward_workspace_size", "rsm_forward", "rsm_forward_selected_path",
             "rsm_decode_step",
-            "rsm_status_string", "rsm_last_error", "rsm_get_device_status", "rsm_version")
+            "rsm_status_string", "rsm_last_error", "rsm_get_device_status", "rsm_version",
+            "rsm_forward_noalloc", "rsm_forward_noalloc_max_scratch")
 
 _vp = ctypes.c_void_p
 _int = ctypes.c_int
@@ -67,6 +68,10 @@ def load() -> ctypes.CDLL:
         lib.rsm_forward.restype = _int
         lib.rsm_forward_selected_path.argtypes = [ctypes.POINTER(ForwardArgs)]
         lib.rsm_forward_selected_path.restype = _int
+        lib.rsm_forward_noalloc.argtypes = [ctypes.POINTER(ForwardArgs), _vp]
+        lib.rsm_forward_noalloc.restype = _int
+        lib.rsm_forward_noalloc_max_scratch.argtypes = []
+        lib.rsm_forward_noalloc_max_scratch.restype = ctypes.c_size_t
         lib.rsm_decode_step.argtypes = [ctypes.POINTER(DecodeArgs), _vp]
         lib.rsm_decode_step.restype = _int
         lib.rsm_status_string.argtypes = [_int]

@@ -93,6 +93,11 @@ bool use_tensor_path(const rsm_forward_args& a) {
 
 }  // namespace
 
+namespace rsm {
+// Records a failure message for rsm_last_error() from other translation units of the library.
+rsm_status report_error(rsm_status s, const char* msg) { return fail(s, "%s", msg); }
+}  // namespace rsm
+
 extern "C" {
 
 const char* rsm_status_string(rsm_status s) {

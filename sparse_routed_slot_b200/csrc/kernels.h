@@ -22,4 +22,7 @@ bool prefill_tc_supported(const rsm_forward_args& a);
 size_t prefill_tc_workspace_bytes(const rsm_forward_args& a);
 cudaError_t launch_prefill_tc(const rsm_forward_args& a, cudaStream_t stream);
 
+// Sets the message rsm_last_error() returns on this host thread; returns `s`.
+rsm_status report_error(rsm_status s, const char* msg);
+
 }  // namespace rsm
