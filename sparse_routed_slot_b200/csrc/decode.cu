@@ -1,12 +1,13 @@
 // decode.cu -- one generation step per (b,h) (rsm_decode_step).
 //
-// Persistent CTAs (three per SM) walk the (b,h) items. For each item the fp32 state H [M, Dv] is
-// fetched with one bulk asynchronous copy into shared memory (in row blocks of at most 64 KB);
-// while it is in flight, warp 0 runs the TopK routing of the token and prepares the decay and
-// write weight of each selected slot. Then every thread applies the sparse update to the rows it
-// covers, writes back only the selected rows, and accumulates o = sum_i q_i H'[i,:] over all M
-// rows. Bytes per (b,h): M*Dv*4 read + K*Dv*4 written + the token's inputs. With three CTAs per
-// SM, one CTA's copy overlaps the others' routing and arithmetic.
+// Persistent CTAs (three per SM) walk the (b,h) items. Each item's fp32 state H [M, Dv] streams
+// through shared memory in blocks of rows fetched by bulk asynchronous copies into two buffers:
+// while one block is processed, the next block -- of this item or of the next item -- is already
+// in flight, so the copies never wait for the arithmetic. Warp 0 runs the TopK routing of an item
+// and prepares the decay and write weight of each selected slot while that item's first block is
+// still arriving. Every thread applies the sparse update to the rows it covers, writes back only
+// the selected rows, and accumulates o = sum_i q_i H'[i,:] over all M rows.
+// Bytes per (b,h): M*Dv*4 read + K*Dv*4 written + the token's inputs.
 //
 // Thread layout: CG = Dv/4 column groups of float4 by RG = floor(256/CG) row groups; thread
 // (rg, cg) covers rows rg, rg+RG, ... of column group cg (a warp reads whole 512-byte rows).
@@ -19,7 +20,7 @@ namespace rsm {
 namespace {
 
 constexpr int kDecodeThreads = 256;
-constexpr int kStageBytes = 64 * 1024;  // state rows fetched per bulk copy
+constexpr int kBlockBytes = 32 * 1024;  // state rows per bulk copy (one of two buffers)
 constexpr int kCtasPerSm = 3;
 
 RSM_DEV void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
@@ -36,44 +37,63 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(rsm_decode_args 
   const int Dv = a.Dv, K = a.K;
   const int CG = Dv >> 2;
   const int RG = kDecodeThreads / CG;
-  const int rows_per_stage = min(M, kStageBytes / (Dv * 4));
+  const int rows_blk = min(M, kBlockBytes / (Dv * 4));  // rows per block
+  const int nblk = (M + rows_blk - 1) / rows_blk;        // blocks per item
   const int tid = threadIdx.x;
   const int cg = tid % CG, rg = tid / CG;
   const bool active = rg < RG;  // threads past CG*RG only help with the small loads
   const int64_t items = (int64_t)a.B * a.H;
 
   extern __shared__ __align__(128) unsigned char dsm[];
-  float* s_state = reinterpret_cast<float*>(dsm);  // [rows_per_stage][Dv]
+  auto buf = [&](uint32_t j) { return reinterpret_cast<float*>(dsm + (j & 1) * kBlockBytes); };
   __shared__ float s_a[M], s_w[M], s_q[M];
   __shared__ unsigned char s_sel[M];
   __shared__ __align__(16) float s_v[256];
   __shared__ __align__(16) float s_red[kDecodeThreads * 4];
-  __shared__ __align__(8) uint64_t bar;
+  __shared__ __align__(8) uint64_t bar[2];
   __shared__ int s_abort;
 
   if (tid == 0) {
-    tc::mbar_init(&bar, 1);
+    tc::mbar_init(&bar[0], 1);
+    tc::mbar_init(&bar[1], 1);
     tc::fence_mbar_init();
     s_abort = 0;
   }
   __syncthreads();
-  uint32_t phase = 0;
+
+  // The CTA's blocks form one stream: (item, block) in order. Block j goes to buffer j & 1.
+  auto issue = [&](int64_t item, int blk, uint32_t j) {
+    const int r0 = blk * rows_blk;
+    const int rows = min(rows_blk, M - r0);
+    const uint32_t bytes = (uint32_t)(rows * Dv * 4);
+    tc::mbar_arrive_expect_tx(&bar[j & 1], bytes);
+    bulk_load(buf(j), a.state + (item * M + r0) * (int64_t)Dv, bytes, &bar[j & 1]);
+  };
+  uint32_t j_issue = 0, j_use = 0;  // blocks issued / consumed by this CTA
+  int64_t nx_item = blockIdx.x;
+  int nx_blk = 0;
+  auto issue_next = [&]() {
+    if (nx_item < items) {
+      issue(nx_item, nx_blk, j_issue++);
+      if (++nx_blk == nblk) {
+        nx_blk = 0;
+        nx_item += gridDim.x;
+      }
+    }
+  };
+  if (tid == 0) {
+    issue_next();
+    issue_next();
+  }
 
   for (int64_t pair = blockIdx.x; pair < items; pair += gridDim.x) {
     float* state = a.state + pair * (int64_t)M * Dv;
-    // 1. first block of state rows in flight
-    if (tid == 0) {
-      const int rows = min(rows_per_stage, M);
-      tc::mbar_arrive_expect_tx(&bar, (uint32_t)(rows * Dv * 4));
-      bulk_load(s_state, state, (uint32_t)(rows * Dv * 4), &bar);
-    }
-    // 2. small inputs
+    // 1. small inputs and the routing of this item (its first block is in flight)
     const TIn* q = reinterpret_cast<const TIn*>(a.q) + pair * M;
     const TIn* k = reinterpret_cast<const TIn*>(a.k) + pair * M;
     const TIn* v = reinterpret_cast<const TIn*>(a.v) + pair * Dv;
     for (int i = tid; i < M; i += blockDim.x) s_q[i] = In<TIn>::ld(q + i);
     for (int d = tid; d < Dv; d += blockDim.x) s_v[d] = In<TIn>::ld(v + d);
-    // 3. routing, decay and write weights of the selected slots (warp 0)
     if (tid < 32) {
       const int lane = tid;
       float x[E];
@@ -111,30 +131,24 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(rsm_decode_args 
     }
     __syncthreads();
 
-    // 4. sparse update of the selected rows, read over all rows, one block of rows at a time
+    // 2. blocks of rows: sparse update of the selected rows, read over all rows
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     const float4 vv = active ? reinterpret_cast<const float4*>(s_v)[cg] : make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int r0 = 0; r0 < M; r0 += rows_per_stage) {
-      if (r0 > 0) {
-        __syncthreads();  // everyone is done with the previous block
-        if (tid == 0) {
-          const int rows = min(rows_per_stage, M - r0);
-          tc::mbar_arrive_expect_tx(&bar, (uint32_t)(rows * Dv * 4));
-          bulk_load(s_state, state + (int64_t)r0 * Dv, (uint32_t)(rows * Dv * 4), &bar);
-        }
-      }
-      if (!tc::mbar_wait(&bar, phase & 1)) {
+    for (int blk = 0; blk < nblk; ++blk) {
+      const uint32_t j = j_use++;
+      if (!tc::mbar_wait(&bar[j & 1], (j >> 1) & 1)) {
         if (tid == 0) {
           s_abort = 1;
           raise_status(RSM_ERR_TIMEOUT);
         }
       }
-      ++phase;
-      const int rows = min(rows_per_stage, M - r0);
+      const float* sb = buf(j);
+      const int r0 = blk * rows_blk;
+      const int rows = min(rows_blk, M - r0);
       if (active) {
         for (int rr = rg; rr < rows; rr += RG) {
           const int r = r0 + rr;
-          float4 hv = reinterpret_cast<const float4*>(s_state + rr * Dv)[cg];
+          float4 hv = reinterpret_cast<const float4*>(sb + rr * Dv)[cg];
           if (s_sel[r]) {
             const float ar = s_a[r], wr = s_w[r];
             hv.x = fmaf(ar, hv.x, wr * vv.x);
@@ -150,18 +164,27 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(rsm_decode_args 
           acc.w = fmaf(qr, hv.w, acc.w);
         }
       }
+      __syncthreads();             // the buffer is consumed ...
+      if (tid == 0) issue_next();  // ... and refilled with the stream's next block
     }
     if (active) reinterpret_cast<float4*>(s_red)[rg * CG + cg] = acc;
     __syncthreads();
 
-    // 5. reduce over the row groups
+    // 3. reduce over the row groups
     for (int d = tid; d < Dv; d += blockDim.x) {
       float s = 0.f;
       for (int g = 0; g < RG; ++g) s += s_red[g * Dv + d];
       a.o[pair * Dv + d] = s;
     }
-    __syncthreads();  // shared buffers are reused by the next item
+    __syncthreads();  // small shared arrays are reused by the next item
     if (s_abort) break;
+  }
+  // a copy still in flight (only after an abort) must land before the CTA leaves
+  if (tid == 0) {
+    while (j_use < j_issue) {
+      const uint32_t j = j_use++;
+      tc::mbar_wait(&bar[j & 1], (j >> 1) & 1);
+    }
   }
 }
 
@@ -174,8 +197,7 @@ int sm_count() {
 
 template <int M>
 cudaError_t launch_m(const rsm_decode_args& a, cudaStream_t stream) {
-  const int rows = std::min(M, kStageBytes / (a.Dv * 4));
-  const int smem = rows * a.Dv * 4;
+  const int smem = 2 * kBlockBytes;
   const int64_t items = (int64_t)a.B * a.H;
   const unsigned grid = (unsigned)std::min<int64_t>(items, (int64_t)sm_count() * kCtasPerSm);
   cudaError_t e;
