@@ -129,6 +129,11 @@ RSM_API rsm_status rsm_forward(const rsm_forward_args* args, void* stream);
  * (RSM_PATH_AUTO resolved), or -1 for arguments rsm_forward rejects. Host-only. */
 RSM_API int rsm_forward_selected_path(const rsm_forward_args* args);
 
+/* Number of kernel launches one rsm_forward call makes for these arguments (for accounting and
+ * profiling: tensor path = routing records + [segment summary + segment scan +] chunk scan; SIMT
+ * path = 1; 0 when B*H == 0 or T == 0), or -1 for arguments rsm_forward rejects. Host-only. */
+RSM_API int rsm_forward_kernel_launches(const rsm_forward_args* args);
+
 /* ---------------------------------------------------------------------------------------------
  * rsm_forward_noalloc -- rsm_forward for callers that cannot allocate device memory.
  *   The pages have no counterpart to this call; it exists for callers with no way to allocate:

@@ -94,6 +94,14 @@ def selected_path(args: _lib.ForwardArgs) -> str:
     return "tensor" if p == _lib.RSM_PATH_TENSOR else "simt"
 
 
+def kernel_launches(args: _lib.ForwardArgs) -> int:
+    """Kernel launches one rsm_forward call makes for these arguments."""
+    n = _lib.load().rsm_forward_kernel_launches(ctypes.byref(args))
+    if n < 0:
+        _lib.check(_lib.load().rsm_forward(ctypes.byref(args), None))
+    return n
+
+
 def forward(q, k, v, logits, f, K: int, H0=None, *, state: bool = True, routing: bool = False,
             path: str = "auto", validate: bool = False, out=None, workspace=None):
     """Chunked prefill. q, k [B,T,H,M]; v [B,T,H,Dv]; logits [B,T,H,M] fp32; f [B,T,H] or

@@ -127,8 +127,12 @@ rsm_status rsm_route(const float* logits, int64_t rows, int M, int K, int32_t* i
   RSM_REQUIRE_PTR(logits, "logits");
   RSM_REQUIRE_PTR(idx_out, "idx_out");
   RSM_OPTIONAL_PTR(score_out, "score_out");
-  cudaError_t e = rsm::launch_route(logits, rows, M, K, idx_out, score_out, 0,
-                                    static_cast<cudaStream_t>(stream));
+  // M = 128 with K <= 32: the thread-per-row selection kernel; other sizes: one warp per row
+  cudaError_t e = rsm::route_records_supported(M, K)
+                      ? rsm::launch_route_records(logits, nullptr, rows, M, K, 0, 0, nullptr, idx_out, score_out,
+                                                  static_cast<cudaStream_t>(stream))
+                      : rsm::launch_route(logits, rows, M, K, idx_out, score_out, 0,
+                                          static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? RSM_OK : cuda_fail(e, "rsm_route launch");
 }
 
@@ -140,6 +144,12 @@ size_t rsm_forward_workspace_size(const rsm_forward_args* a) {
 int rsm_forward_selected_path(const rsm_forward_args* a) {
   if (check_forward(a) != RSM_OK) return -1;
   return use_tensor_path(*a) ? RSM_PATH_TENSOR : RSM_PATH_SIMT;
+}
+
+int rsm_forward_kernel_launches(const rsm_forward_args* a) {
+  if (check_forward(a) != RSM_OK) return -1;
+  if ((int64_t)a->B * a->H == 0 || a->T == 0) return 0;
+  return use_tensor_path(*a) ? rsm::prefill_tc_launches(*a) : 1;
 }
 
 rsm_status rsm_forward(const rsm_forward_args* a, void* stream) {

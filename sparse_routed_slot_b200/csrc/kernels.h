@@ -11,6 +11,15 @@ namespace rsm {
 cudaError_t launch_route(const float* logits, int64_t rows, int M, int K, int32_t* idx_out,
                          float* score_out, int validate, cudaStream_t stream);
 
+// Thread-per-row TopK for M = 128, K <= 32 (route_rec.cu): routing records for the tensor prefill
+// (`rec`, route_record_bytes(K) bytes per row) and/or ranked indices and scores; null outputs are
+// skipped. `f` is read only when `rec` is written (or `validate` is set).
+bool route_records_supported(int M, int K);
+int route_record_bytes(int K);
+cudaError_t launch_route_records(const float* logits, const float* f, int64_t rows, int M, int K, int decay_slot,
+                                 int validate, unsigned char* rec, int32_t* idx_out, float* score_out,
+                                 cudaStream_t stream);
+
 cudaError_t launch_decode(const rsm_decode_args& a, cudaStream_t stream);
 
 // CUDA-core fp32 chunked prefill (any supported size).
@@ -20,6 +29,7 @@ size_t prefill_simt_smem_bytes(int M, int Dv);
 // tcgen05 tensor-core chunked prefill. `supported` tells whether the shape/dtype can run there.
 bool prefill_tc_supported(const rsm_forward_args& a);
 size_t prefill_tc_workspace_bytes(const rsm_forward_args& a);
+int prefill_tc_launches(const rsm_forward_args& a);  // kernel launches of one call
 cudaError_t launch_prefill_tc(const rsm_forward_args& a, cudaStream_t stream);
 
 // Sets the message rsm_last_error() returns on this host thread; returns `s`.

@@ -3,16 +3,21 @@
 // Shapes: M = 128 slots, Dv = 128, bf16 q/k/v, K <= 32, per-head or per-slot log-decay.
 //
 // Chunk algebra (paperlayer.ai summary of the Raven paper, section A.5: T = n*C chunks of C = 64
-// tokens), for one (b,h) stream and one chunk, with g_{t,i} the cumulative log-decay of slot i from
-// the chunk start through token t (g <= 0), w_{t,i} = k_{t,i} (1 - a_{t,i}) on the selected slots
-// and 0 elsewhere, and the reference point of the exponentials at the chunk start:
-//   Qh = q * e^{g}            (|Qh| <= |q|)
-//   Wh = w * e^{-g}           (finite while every slot decays by less than e^-80 in the chunk)
+// tokens), for one (b,h) stream and one chunk, with G_{t,i} = e^{g_{t,i}} the product of the decays
+// a = e^lam of slot i from the chunk start through token t, w_{t,i} = k_{t,i} (1 - a_{t,i}) on the
+// selected slots and 0 elsewhere, and the reference point at the chunk start:
+//   Qh = q * G                (|Qh| <= |q|)
+//   Wh = w / G                (finite while every slot decays by less than e^-80 in the chunk)
 //   S  = Qh Wh^T,  A = S masked to s <= t           (intra-chunk weights, read after write)
 //   O  = Qh H_start + A V                            (chunk outputs)
-//   H_end = e^{g_end} * (H_start + Wh^T V)           (carry; rows never selected are skipped)
-// A chunk whose decay is stronger than that bound takes an exact path: A from pairwise sums with
-// non-positive exponents, and the carry with weights w * e^{g_end - g} after the state is decayed.
+//   H_end = G_end * (H_start + Wh^T V)               (carry; rows never selected are skipped)
+// G and 1/G are running products of a and 1/a down the chunk, so the tiles need no exponential
+// per element. A chunk whose decay is stronger than the bound takes an exact path: A from
+// pairwise sums with non-positive exponents, and the carry with weights w * e^{g_end - g} after
+// the state is decayed.
+//
+// The routing is not done here: a thread-per-row kernel (route_rec.cu) has already turned the
+// logits into one record per row (selection mask, selected slots, lam of each), read here.
 //
 // Operands are fp32 tiles rounded to nearest tf32 (kind::tf32), accumulated in fp32. The fp32
 // state lives in TMEM as H^T (lane = value column, column = slot); the carry accumulates into it
@@ -20,12 +25,13 @@
 // TMEM columns: [0,128) H^T, [128,256) rounded H^T, [256,320) O^T, [320,384) S (64-lane layout).
 //
 // Warp roles (one persistent CTA per SM, 12 warps):
-//   warps 0-7  row workers: for each chunk, the routing of 8 rows per warp (TopK, log-decay), a
-//              cross-warp prefix of the log-decay, then their rows of the Qh, Wh and Wh^T tiles.
-//              They route chunk n+1 while the tensor core and the TMEM workers finish chunk n.
+//   warps 0-7  row workers, 8 rows of each chunk per warp: the decays of the selected entries of
+//              their rows (one lane per entry), the per-slot product over their rows, then, once
+//              the previous chunk's MMAs have read the operand tiles, their rows of Qh, Wh, Wh^T.
+//              q, k and the records of the next chunk are loaded while this one is processed.
 //   warps 8-11 TMEM workers (one per TMEM lane quarter): outputs of chunk n-1, the decay of the
 //              state and its rounded copy, the V^T tile of chunk n, the S -> A masking. Thread 256
-//              also issues the tile loads and the MMAs.
+//              also issues the v tile loads and the MMAs.
 //
 // Long sequences with few (b,h) streams are split into segments processed in parallel: a summary
 // pass runs the state recurrence of each segment but the last from a zero state and stores
@@ -51,9 +57,9 @@ constexpr int kRWarps = 8;     // row workers
 constexpr int kRowsPerWarp = kC / kRWarps;
 constexpr int kThreads = 384;
 constexpr int kRThreads = kRWarps * 32;
-constexpr int kIssuer = kRThreads;  // first thread of the TMEM workers
-constexpr float kGMax = 80.f;       // fast-path bound on the in-chunk decay (e^80 fits fp32/tf32)
-constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kIssuer = kRThreads;       // first thread of the TMEM workers
+constexpr float kDMin = 1.80485139e-35f;  // e^-80: fast-path bound on the in-chunk decay
+constexpr int kRecMax = 176;              // routing record bytes for K = 32
 
 constexpr int kColH = 0, kColHr = 128, kColO = 256, kColS = 320, kTmemCols = 512;
 
@@ -61,16 +67,17 @@ constexpr int kColH = 0, kColHr = 128, kColO = 256, kColS = 320, kTmemCols = 512
 // swizzled format of tc.cuh; Wh^T and V^T are stored transposed because they are contracted over
 // tokens (a tf32 operand cannot be MN-major in this swizzle).
 constexpr int kOffQ = 0;                      // Qh   [64 t][128 slot]   (A of S, B of the read)
-constexpr int kOffW = kOffQ + 32768;          // Wh   [64 s][128 slot]   (B of S)
+constexpr int kOffW = kOffQ + 32768;          // Wh   [64 s][128 slot]   (B of S); exact path: dense g
 constexpr int kOffWt = kOffW + 32768;         // Wh^T [128 slot][64 s]   (B of the carry)
 constexpr int kOffVt = kOffWt + 32768;        // V^T  [128 dv][64 s]     (A of carry and A.V)
 constexpr int kOffA = kOffVt + 32768;         // A    [64 t][64 s]       (B of A.V)
-constexpr int kOffRawV = kOffA + 16384;       // v tiles from TMA, 2 x [64][128] bf16
-constexpr int kOffTot = kOffRawV + 2 * 16384; // per-warp log-decay totals, 2 x [8][128] fp32
-constexpr int kOffSidx = kOffTot + 2 * kRWarps * kM * 4;   // exact path: written slots [64][32]
-constexpr int kOffSw = kOffSidx + kC * kKMax;              // exact path: their write weights
-constexpr int kOffSmall = kOffSw + kC * kKMax * 4;
-constexpr int kSmallBytes = (2 * kM + 2 * kM + kC) * 4 + 16;  // D[2][M], touched[2][M], cnt[64], fast[2]
+constexpr int kOffRawV = kOffA + 16384;       // v tile from TMA, [64][128] bf16
+constexpr int kOffCmp = kOffRawV + 16384;     // per selected entry (a, 1/a, 1-a, lam), [64][KP] float4
+constexpr int kOffRec = kOffCmp + kC * kKMax * 16;                   // records, [8 warps][8 rows][RB]
+constexpr int kOffTot = kOffRec + kRWarps * kRowsPerWarp * kRecMax;  // per-warp slot totals, [2][8][128]
+constexpr int kOffSmall = kOffTot + 2 * kRWarps * kM * 4;
+// D[2][M], touched[2][M], mask OR [2][8][4], fast[2]
+constexpr int kSmallBytes = (2 * kM + 2 * kM + 2 * kRWarps * 4 + 2) * 4 + 8;
 constexpr int kSmemBytes = kOffSmall + kSmallBytes + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
@@ -80,17 +87,13 @@ struct Maps {
 
 struct Params {
   int B, T, H, K;
-  int decay_slot;
   const __nv_bfloat16* q;
   const __nv_bfloat16* k;
-  const float* logits;
-  const float* f;
+  const unsigned char* rec;  // routing records, rec_bytes per row, rows in [B, T, H] order
+  int rec_bytes;
   const float* H0;
   float* o;
   float* HT;
-  int32_t* idx_out;
-  float* score_out;
-  int validate;
   int nseg, seg_chunks;
   float* ws_state;  // [pairs][nseg][M][Dv]: slot 0 = start state, slot j+1 = summary of segment j
   float* ws_D;      // [pairs][nseg][M]
@@ -102,6 +105,9 @@ RSM_DEV float4 bf16x4_to_f32(uint2 r) {
                      __uint_as_float(r.y << 16), __uint_as_float(r.y & 0xffff0000u));
 }
 RSM_DEV float fget(const float4& v, int e) { return e == 0 ? v.x : e == 1 ? v.y : e == 2 ? v.z : v.w; }
+RSM_DEV float bf16_at(const __nv_bfloat16* p) {
+  return __uint_as_float((uint32_t)(*reinterpret_cast<const uint16_t*>(p)) << 16);
+}
 
 // Bounded mbarrier wait; on expiry records a timeout and raises the CTA abort flag.
 RSM_DEV void wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
@@ -126,6 +132,7 @@ RSM_DEV bool bar_rows_or(bool flag) {
       : "memory");
   return r != 0;
 }
+RSM_DEV void bar_rows() { asm volatile("bar.sync 1, %0;" ::"n"(kRThreads) : "memory"); }
 
 // Position of one chunk in the CTA's work list.
 struct Chunk {
@@ -170,6 +177,39 @@ struct Walker {
   }
 };
 
+// A row worker's inputs for one chunk: q and k of its 8 rows (4 slots per lane) and the pieces of
+// its 8 routing records (16 bytes per piece, up to 3 pieces per lane).
+struct RowInputs {
+  uint2 q[kRowsPerWarp], k[kRowsPerWarp];
+  uint4 rec[3];
+};
+
+template <bool SUMMARY>
+RSM_DEV void load_rows(const Params& p, const Chunk& c, int w, int lane, int n16, RowInputs& in) {
+#pragma unroll
+  for (int r = 0; r < kRowsPerWarp; ++r) {
+    const int t = w * kRowsPerWarp + r;
+    in.k[r] = make_uint2(0u, 0u);
+    in.q[r] = make_uint2(0u, 0u);
+    if (t < c.nrows) {
+      const int64_t row = ((int64_t)c.b * p.T + c.c0 + t) * p.H + c.h;
+      in.k[r] = reinterpret_cast<const uint2*>(p.k + row * kM)[lane];
+      if (!SUMMARY) in.q[r] = reinterpret_cast<const uint2*>(p.q + row * kM)[lane];
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < 3; ++u) {
+    const int idx = lane + 32 * u;
+    const int r = idx / n16, part = idx - r * n16;
+    const int t = w * kRowsPerWarp + r;
+    in.rec[u] = make_uint4(0u, 0u, 0u, 0u);
+    if (r < kRowsPerWarp && t < c.nrows) {
+      const int64_t row = ((int64_t)c.b * p.T + c.c0 + t) * p.H + c.h;
+      in.rec[u] = *reinterpret_cast<const uint4*>(p.rec + row * p.rec_bytes + part * 16);
+    }
+  }
+}
+
 template <bool SUMMARY>
 __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_constant__ Maps maps,
                                                                   const Params p) {
@@ -181,15 +221,15 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
   unsigned char* sVt = sm + kOffVt;
   unsigned char* sA = sm + kOffA;
   const uint16_t* sRawV = reinterpret_cast<const uint16_t*>(sm + kOffRawV);
+  float4* sCmp = reinterpret_cast<float4*>(sm + kOffCmp);
+  unsigned char* sRec = sm + kOffRec;
   float* sTot = reinterpret_cast<float*>(sm + kOffTot);
-  unsigned char* sSidx = sm + kOffSidx;
-  float* sSw = reinterpret_cast<float*>(sm + kOffSw);
-  float* sDc = reinterpret_cast<float*>(sm + kOffSmall);  // [2][M]
-  int* sTouch = reinterpret_cast<int*>(sDc + 2 * kM);      // [2][M]
-  int* sCnt = sTouch + 2 * kM;                             // [64]
-  int* sFast = sCnt + kC;                                  // [2]
+  float* sDc = reinterpret_cast<float*>(sm + kOffSmall);         // [2][M]
+  int* sTouch = reinterpret_cast<int*>(sDc + 2 * kM);             // [2][M]
+  uint32_t* sOr = reinterpret_cast<uint32_t*>(sTouch + 2 * kM);  // [2][8][4]
+  int* sFast = reinterpret_cast<int*>(sOr + 2 * kRWarps * 4);    // [2]
 
-  __shared__ __align__(8) uint64_t bar_tma[2], bar_ready, bar_s, bar_a, bar_o, bar_x;
+  __shared__ __align__(8) uint64_t bar_tma, bar_v, bar_ready, bar_s, bar_a, bar_t, bar_o, bar_x;
   __shared__ uint32_t s_tbase;
   __shared__ int s_abort;
 
@@ -199,14 +239,16 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
   const int pairs = p.B * H;
   const int segs_here = SUMMARY ? p.nseg - 1 : p.nseg;
   const int items = pairs * segs_here;
+  const int KP = K <= 16 ? 16 : 32;  // entries per row in sCmp
 
   if (warp == kRWarps) tc::tmem_alloc(&s_tbase, kTmemCols);
   if (tid == 0) {
-    tc::mbar_init(&bar_tma[0], 1);
-    tc::mbar_init(&bar_tma[1], 1);
+    tc::mbar_init(&bar_tma, 1);
+    tc::mbar_init(&bar_v, kThreads - kRThreads);
     tc::mbar_init(&bar_ready, kThreads);
     tc::mbar_init(&bar_s, 1);
     tc::mbar_init(&bar_a, kThreads - kRThreads);
+    tc::mbar_init(&bar_t, 1);
     tc::mbar_init(&bar_o, 1);
     tc::mbar_init(&bar_x, kThreads);
     tc::fence_mbar_init();
@@ -231,120 +273,99 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
   if (row_worker) {
     // =========================================================================== row workers
     const int w = warp;
-    float Dseg[4] = {1.f, 1.f, 1.f, 1.f};  // summary pass, warp 0: product of the chunk decays
+    const int RB = p.rec_bytes, n16 = RB / 16;
+    const int slot_off = 16, lam_off = 16 + ((K + 15) & ~15);
+    unsigned char* myRec = sRec + w * (kRowsPerWarp * kRecMax);  // this warp's 8 records, stride RB
+    const int mw = lane >> 3;                  // mask word holding the lane's 4 slots
+    const int sh = (lane & 7) * 4;             // bit offset of the lane's slots in that word
+    const uint32_t below = (1u << sh) - 1u;    // the word's bits of lower slots
+    const int ej = lane % KP, er = lane / KP;  // entry-parallel mapping: entry ej of row r0 + er
+    const int rpp = 32 / KP;                   // rows per entry pass
+    float Dseg[4] = {1.f, 1.f, 1.f, 1.f};      // summary pass, warp 0: product of the chunk decays
     int tseg[4] = {0, 0, 0, 0};
-    float tau = 0.f;  // last routing threshold found by this warp (a guess for the next rows)
+
+    RowInputs cur;
+    if (wk.valid()) load_rows<SUMMARY>(p, wk.get(), w, lane, n16, cur);
     for (uint32_t n = 0; wk.valid(); ++n, wk.next()) {
       const Chunk ck = wk.get();
       const int buf = n & 1;
-      // ---- stage A: routing and per-slot log-decay of this warp's 8 rows
-      float lam[kRowsPerWarp][4];
-      uint2 qv[kRowsPerWarp], kv[kRowsPerWarp];
-      float4 xv[kRowsPerWarp], fv[kRowsPerWarp];
+      // ---- records into shared memory; the next chunk's inputs start loading
+#pragma unroll
+      for (int u = 0; u < 3; ++u) {
+        const int idx = lane + 32 * u;
+        const int r = idx / n16, part = idx - r * n16;
+        if (r < kRowsPerWarp) *reinterpret_cast<uint4*>(myRec + r * RB + part * 16) = cur.rec[u];
+      }
+      RowInputs nxt;
+      {
+        Walker nx = wk;
+        nx.next();
+        if (nx.valid()) load_rows<SUMMARY>(p, nx.get(), w, lane, n16, nxt);
+      }
+      __syncwarp();
+      // ---- decay of every selected entry of the warp's rows (one lane per entry)
+      for (int r0 = 0; r0 < kRowsPerWarp; r0 += rpp) {
+        const int r = r0 + er;
+        const int t = w * kRowsPerWarp + r;
+        if (ej < K && t < ck.nrows) {
+          const float lam = *reinterpret_cast<const float*>(myRec + r * RB + lam_off + 4 * ej);
+          sCmp[t * KP + ej] = make_float4(expf(lam), expf(-lam), -expm1f(lam), lam);
+        }
+      }
+      float* tot = sTot + (buf * kRWarps + w) * kM;
+      reinterpret_cast<float4*>(tot)[lane] = make_float4(1.f, 1.f, 1.f, 1.f);
+      if (lane < 4) {
+        uint32_t om = 0u;
+#pragma unroll
+        for (int r = 0; r < kRowsPerWarp; ++r) om |= reinterpret_cast<const uint32_t*>(myRec + r * RB)[lane];
+        sOr[(buf * kRWarps + w) * 4 + lane] = om;
+      }
+      __syncwarp();
+      // per-slot product of the decays over the warp's rows, rows in order
 #pragma unroll
       for (int r = 0; r < kRowsPerWarp; ++r) {
         const int t = w * kRowsPerWarp + r;
-        const int64_t row = ((int64_t)ck.b * T + ck.c0 + t) * H + ck.h;
-        if (t < ck.nrows) {
-          xv[r] = reinterpret_cast<const float4*>(p.logits + row * kM)[lane];
-          if (p.decay_slot) {
-            fv[r] = reinterpret_cast<const float4*>(p.f + row * kM)[lane];
-          } else {
-            const float fs = p.f[row];
-            fv[r] = make_float4(fs, fs, fs, fs);
-          }
-          kv[r] = reinterpret_cast<const uint2*>(p.k + row * kM)[lane];
-          qv[r] = SUMMARY ? make_uint2(0u, 0u) : reinterpret_cast<const uint2*>(p.q + row * kM)[lane];
-        } else {
-          xv[r] = make_float4(0.f, 0.f, 0.f, 0.f);
-          fv[r] = xv[r];
-          kv[r] = make_uint2(0u, 0u);
-          qv[r] = kv[r];
+        if (lane < K && t < ck.nrows) {
+          const int slot = myRec[r * RB + slot_off + lane];
+          tot[slot] *= sCmp[t * KP + lane].x;
         }
+        __syncwarp();
       }
-      float tot[4] = {0.f, 0.f, 0.f, 0.f};
-      const bool want_routing = !SUMMARY && (p.idx_out || p.score_out);
-#pragma unroll
-      for (int r0 = 0; r0 < kRowsPerWarp; r0 += 4) {
-        // selection of four rows at a time (their reductions overlap)
-        float x[4][4];
-        uint32_t sel[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          x[r][0] = xv[r0 + r].x; x[r][1] = xv[r0 + r].y; x[r][2] = xv[r0 + r].z; x[r][3] = xv[r0 + r].w;
-        }
-        uint32_t ok = 0u;
-        if (!want_routing && K >= 2) ok = warp_select_guess_rows<kM, 4>(x, K, tau, sel);
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          const int t = w * kRowsPerWarp + r0 + r;
-#pragma unroll
-          for (int e = 0; e < 4; ++e) lam[r0 + r][e] = 0.f;
-          if (t >= ck.nrows) continue;  // warp-uniform
-          const int64_t row = ((int64_t)ck.b * T + ck.c0 + t) * H + ck.h;
-          if (p.validate) {
-            bool bad = false;
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float fe = fget(fv[r0 + r], e);
-              bad |= !finite_f32(x[r][e]) || !finite_f32(fe) || fe > 0.f;
-            }
-            if (__any_sync(kFull, bad) && lane == 0) raise_status(RSM_ERR_NONFINITE);
-          }
-          if (!(ok & (1u << r))) {
-            int32_t* io = want_routing && p.idx_out ? p.idx_out + row * K : nullptr;
-            float* so = want_routing && p.score_out ? p.score_out + row * K : nullptr;
-            const float(&xr)[4] = x[r];
-            sel[r] = warp_topk<kM>(xr, K, lane, [&](int rk, int slot, int e) {
-              if (io) io[rk] = slot;
-              if (so) so[rk] = sigmoid_f32(xr[e]);
-            });
-          }
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float s = __frcp_rn(1.f + __expf(-x[r][e]));  // router score (selected slots)
-            lam[r0 + r][e] = (sel[r] & (1u << e)) ? s * fget(fv[r0 + r], e) : 0.f;
-          }
-        }
-      }
-#pragma unroll
-      for (int r = 0; r < kRowsPerWarp; ++r)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) tot[e] += lam[r][e];
-      reinterpret_cast<float4*>(sTot + (buf * kRWarps + w) * kM)[lane] = make_float4(tot[0], tot[1], tot[2], tot[3]);
       if (bar_rows_or(*abort_flag != 0)) break;  // every row worker takes the same decision
-      float off[4] = {0.f, 0.f, 0.f, 0.f}, gend[4] = {0.f, 0.f, 0.f, 0.f};
+      // ---- in-chunk products at the warp's first row (off) and over the chunk (gend)
+      float off[4] = {1.f, 1.f, 1.f, 1.f}, gend[4] = {1.f, 1.f, 1.f, 1.f};
+      uint32_t orw = 0u;
 #pragma unroll
       for (int w2 = 0; w2 < kRWarps; ++w2) {
         const float4 t4 = reinterpret_cast<const float4*>(sTot + (buf * kRWarps + w2) * kM)[lane];
         const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          if (w2 < w) off[e] += tv[e];
-          gend[e] += tv[e];
+          if (w2 < w) off[e] *= tv[e];
+          gend[e] *= tv[e];
         }
+        orw |= sOr[(buf * kRWarps + w2) * 4 + mw];
       }
       bool ok = true;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) ok &= gend[e] >= -kGMax;
+      for (int e = 0; e < 4; ++e) ok &= gend[e] >= kDMin;
       const bool fast = __all_sync(kFull, ok);
-      // ---- the previous chunk's MMAs are done: its operand tiles are free, and the TMEM workers
-      // have finished the chunk before it (whose decay buffer this chunk reuses)
-      if (n > 0) wait_or_abort(&bar_o, (n - 1) & 1, abort_flag);
+      // ---- the previous chunk's MMAs have read the operand tiles (and the TMEM workers have
+      // finished the chunk before it, whose decay buffer this chunk reuses)
+      if (n > 0) wait_or_abort(&bar_t, (n - 1) & 1, abort_flag);
       if (w == 0) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int slot = lane * 4 + e;
-          const float D = exp2f(gend[e] * kLog2e);
-          const int touched = gend[e] != 0.f;
-          sDc[buf * kM + slot] = D;
+          const int touched = (orw >> (sh + e)) & 1u;
+          sDc[buf * kM + slot] = gend[e];
           sTouch[buf * kM + slot] = touched;
           if (SUMMARY) {
             if (ck.first) {
               Dseg[e] = 1.f;
               tseg[e] = 0;
             }
-            Dseg[e] *= D;
+            Dseg[e] *= gend[e];
             tseg[e] |= touched;
             if (ck.last) {
               const int64_t base = ((int64_t)ck.pair * p.nseg + ck.seg + 1) * kM;
@@ -356,27 +377,36 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         if (lane == 0) sFast[buf] = fast;
       }
       if (fast) {
-        // ---- stage B: this warp's rows of Qh, Wh and Wh^T
-        float g[4], Eprev[4];
+        // ---- this warp's rows of Qh, Wh and Wh^T
+        float G[4], Gi[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          g[e] = off[e];
-          Eprev[e] = exp2f(-off[e] * kLog2e);
+          G[e] = off[e];
+          Gi[e] = 1.f / off[e];
         }
         float stash[4][4];
 #pragma unroll
         for (int r = 0; r < kRowsPerWarp; ++r) {
           const int t = w * kRowsPerWarp + r;
-          const float4 q4 = bf16x4_to_f32(qv[r]);
-          const float4 k4 = bf16x4_to_f32(kv[r]);
+          const uint4 mk = *reinterpret_cast<const uint4*>(myRec + r * RB);
+          const uint32_t wd = mw == 0 ? mk.x : mw == 1 ? mk.y : mw == 2 ? mk.z : mk.w;
+          int base = __popc(wd & below) + (mw > 0 ? __popc(mk.x) : 0) + (mw > 1 ? __popc(mk.y) : 0) +
+                     (mw > 2 ? __popc(mk.z) : 0);
+          const float4 q4 = bf16x4_to_f32(cur.q[r]);
+          const float4 k4 = bf16x4_to_f32(cur.k[r]);
           float qh[4], wh[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            g[e] += lam[r][e];
-            const float E = exp2f(-g[e] * kLog2e);                 // e^{-g_t}
-            wh[e] = tc::to_tf32(fget(k4, e) * (E - Eprev[e]));     // k (1 - a) e^{-g_t}
-            Eprev[e] = E;
-            qh[e] = SUMMARY ? 0.f : tc::to_tf32(fget(q4, e) * exp2f(g[e] * kLog2e));
+            float wt = 0.f;
+            if ((wd >> (sh + e)) & 1u) {
+              const float4 c = sCmp[t * KP + base];
+              ++base;
+              G[e] *= c.x;
+              Gi[e] *= c.y;
+              wt = fget(k4, e) * c.z * Gi[e];  // k (1 - a) / G_t
+            }
+            qh[e] = SUMMARY ? 0.f : tc::to_tf32(fget(q4, e) * G[e]);
+            wh[e] = tc::to_tf32(wt);
             stash[r & 3][e] = wh[e];
           }
           if (!SUMMARY) {
@@ -401,82 +431,93 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         tc::fence_async_smem();
         mbar_arrive(&bar_ready);
       } else {
-        // ---- exact path (rare), with the TMEM workers: the Qh tile as usual, dense q (bf16, in
-        // the raw v buffer of this chunk, already converted) and dense g (in the Wh region, unused
-        // here), the listed write weights, then A and the end-referenced Wh^T, exponents <= 0
+        // ---- exact path (rare), with the TMEM workers: dense g (log domain, in the Wh region),
+        // the Qh tile, the end-referenced Wh^T and A from pairwise sums, exponents <= 0
         mbar_arrive(&bar_ready);
-        sync_x();  // X0
-        uint2* dq = reinterpret_cast<uint2*>(sm + kOffRawV + buf * (kC * kDV * 2));  // plain [64][128] bf16
-        float* dg = reinterpret_cast<float*>(sW);                                    // plain [64][128]
-        float g[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) g[e] = off[e];
+        sync_x();  // X0: every row worker is past the product totals; the TMEM workers decay H
+        float* totL = sTot + (buf * kRWarps + w) * kM;  // now: per-warp sums of lam
+        reinterpret_cast<float4*>(totL)[lane] = make_float4(0.f, 0.f, 0.f, 0.f);
+        __syncwarp();
 #pragma unroll
         for (int r = 0; r < kRowsPerWarp; ++r) {
           const int t = w * kRowsPerWarp + r;
-          const float4 q4 = bf16x4_to_f32(qv[r]);
-          const float4 k4 = bf16x4_to_f32(kv[r]);
-          float wv[4], qh[4];
-          int cnt = 0;
+          if (lane < K && t < ck.nrows) {
+            const int slot = myRec[r * RB + slot_off + lane];
+            totL[slot] += sCmp[t * KP + lane].w;
+          }
+          __syncwarp();
+        }
+        bar_rows();
+        float g[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int w2 = 0; w2 < w; ++w2) {
+          const float4 t4 = reinterpret_cast<const float4*>(sTot + (buf * kRWarps + w2) * kM)[lane];
+          g[0] += t4.x; g[1] += t4.y; g[2] += t4.z; g[3] += t4.w;
+        }
+        float* dg = reinterpret_cast<float*>(sW);  // plain [64][128]
+#pragma unroll
+        for (int r = 0; r < kRowsPerWarp; ++r) {
+          const int t = w * kRowsPerWarp + r;
+          const uint4 mk = *reinterpret_cast<const uint4*>(myRec + r * RB);
+          const uint32_t wd = mw == 0 ? mk.x : mw == 1 ? mk.y : mw == 2 ? mk.z : mk.w;
+          int base = __popc(wd & below) + (mw > 0 ? __popc(mk.x) : 0) + (mw > 1 ? __popc(mk.y) : 0) +
+                     (mw > 2 ? __popc(mk.z) : 0);
+          const float4 q4 = bf16x4_to_f32(cur.q[r]);
+          float qh[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            g[e] += lam[r][e];
-            wv[e] = fget(k4, e) * (-expm1f(lam[r][e]));
-            cnt += wv[e] != 0.f;
+            if ((wd >> (sh + e)) & 1u) {
+              g[e] += sCmp[t * KP + base].w;
+              ++base;
+            }
             qh[e] = SUMMARY ? 0.f : tc::to_tf32(fget(q4, e) * expf(g[e]));
           }
+          reinterpret_cast<float4*>(dg + t * kM)[lane] = make_float4(g[0], g[1], g[2], g[3]);
           if (!SUMMARY)
             *reinterpret_cast<float4*>(sQ + tc::swz_offset(kC, t, lane * 4)) = make_float4(qh[0], qh[1], qh[2], qh[3]);
-          dq[t * (kM / 4) + lane] = qv[r];
-          reinterpret_cast<float4*>(dg + t * kM)[lane] = make_float4(g[0], g[1], g[2], g[3]);
-          int pre = cnt;  // inclusive scan over lanes
-#pragma unroll
-          for (int d = 1; d < 32; d <<= 1) {
-            const int v = __shfl_up_sync(kFull, pre, d);
-            if (lane >= d) pre += v;
-          }
-          const int total = __shfl_sync(kFull, pre, 31);
-          pre -= cnt;
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            if (wv[e] != 0.f) {
-              sSidx[t * kKMax + pre] = (unsigned char)(lane * 4 + e);
-              sSw[t * kKMax + pre] = wv[e];
-              ++pre;
-            }
-          }
-          if (lane == 0) sCnt[t] = total;  // <= K <= 32: only selected slots have w != 0
         }
-        for (int e = tid; e < kC * kM; e += kRThreads)
-          *reinterpret_cast<float*>(sWt + tc::swz_offset(kM, e / kC, e % kC)) = 0.f;
-        sync_x();  // X1
+        // write weight of every selected entry, w = k (1 - a), into its (unused) 1/a field
+        for (int r0 = 0; r0 < kRowsPerWarp; r0 += rpp) {
+          const int r = r0 + er;
+          const int t = w * kRowsPerWarp + r;
+          if (ej < K && t < ck.nrows) {
+            const int slot = myRec[r * RB + slot_off + ej];
+            const int64_t row = ((int64_t)ck.b * T + ck.c0 + t) * H + ck.h;
+            sCmp[t * KP + ej].y = bf16_at(p.k + row * kM + slot) * sCmp[t * KP + ej].z;
+          }
+        }
+        for (int e = tid; e < kC * kM / 4; e += kRThreads)
+          reinterpret_cast<float4*>(sWt)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+        bar_rows();
         const int nrows = ck.nrows;
-        for (int e = tid; e < nrows * kKMax; e += kRThreads) {
-          const int t = e / kKMax, r = e % kKMax;
-          if (r >= sCnt[t]) continue;
-          const int i = sSidx[t * kKMax + r];
+        for (int e = tid; e < nrows * KP; e += kRThreads) {
+          const int t = e / KP, j = e % KP;
+          if (j >= K) continue;
+          const unsigned char* rt = sRec + (t / kRowsPerWarp) * (kRowsPerWarp * kRecMax) + (t % kRowsPerWarp) * RB;
+          const int i = rt[slot_off + j];
           const float gend_i = dg[(kC - 1) * kM + i];
           *reinterpret_cast<float*>(sWt + tc::swz_offset(kM, i, t)) =
-              tc::to_tf32(sSw[t * kKMax + r] * expf(gend_i - dg[t * kM + i]));
+              tc::to_tf32(sCmp[t * KP + j].y * expf(gend_i - dg[t * kM + i]));
         }
         if (!SUMMARY) {
           for (int e = tid; e < kC * kC; e += kRThreads) {
             const int t = e / kC, s = e % kC;
             float acc = 0.f;
             if (s <= t && t < nrows) {
-              const int cs = sCnt[s];
-              for (int r = 0; r < cs; ++r) {
-                const int i = sSidx[s * kKMax + r];
-                const float qti = __uint_as_float((uint32_t)reinterpret_cast<const uint16_t*>(dq)[t * kM + i] << 16);
-                acc = fmaf(qti * sSw[s * kKMax + r], expf(dg[t * kM + i] - dg[s * kM + i]), acc);
+              const unsigned char* rs = sRec + (s / kRowsPerWarp) * (kRowsPerWarp * kRecMax) + (s % kRowsPerWarp) * RB;
+              const int64_t rowt = ((int64_t)ck.b * T + ck.c0 + t) * H + ck.h;
+              for (int j = 0; j < K; ++j) {
+                const int i = rs[slot_off + j];
+                const float qti = bf16_at(p.q + rowt * kM + i);
+                acc = fmaf(qti * sCmp[s * KP + j].y, expf(dg[t * kM + i] - dg[s * kM + i]), acc);
               }
             }
             *reinterpret_cast<float*>(sA + tc::swz_offset(kC, t, s)) = tc::to_tf32(acc);
           }
         }
         tc::fence_async_smem();
-        sync_x();  // X2
+        sync_x();  // X1
       }
+      cur = nxt;
     }
   } else {
     // =========================================================================== TMEM workers
@@ -540,8 +581,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     if (issuer && wk.valid()) {
       const Chunk c = wk.get();
       ++n_tma_issued;
-      tc::mbar_arrive_expect_tx(&bar_tma[0], kC * kDV * 2);
-      tc::tma_load_4d(sm + kOffRawV, &maps.v, &bar_tma[0], 0, c.h, c.c0, c.b);
+      tc::mbar_arrive_expect_tx(&bar_tma, kC * kDV * 2);
+      tc::tma_load_4d(sm + kOffRawV, &maps.v, &bar_tma, 0, c.h, c.c0, c.b);
     }
     uint32_t n = 0;
     for (; wk.valid() && !*abort_flag; ++n, wk.next()) {
@@ -567,31 +608,28 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         tc::tmem_wait_st();
       }
       // V^T tile of this chunk (thread = value column; conflict-free 16-byte stores)
-      wait_or_abort(&bar_tma[buf], (n >> 1) & 1, abort_flag);
-      {
-        const uint16_t* rv = sRawV + buf * (kC * kDV);
+      wait_or_abort(&bar_tma, n & 1, abort_flag);
 #pragma unroll 4
-        for (int s4 = 0; s4 < kC; s4 += 4) {
-          const float4 f4 = make_float4(__uint_as_float((uint32_t)rv[(s4 + 0) * kDV + dv] << 16),
-                                        __uint_as_float((uint32_t)rv[(s4 + 1) * kDV + dv] << 16),
-                                        __uint_as_float((uint32_t)rv[(s4 + 2) * kDV + dv] << 16),
-                                        __uint_as_float((uint32_t)rv[(s4 + 3) * kDV + dv] << 16));
-          *reinterpret_cast<float4*>(sVt + tc::swz_offset(kDV, dv, s4)) = f4;
-        }
+      for (int s4 = 0; s4 < kC; s4 += 4) {
+        const float4 f4 = make_float4(__uint_as_float((uint32_t)sRawV[(s4 + 0) * kDV + dv] << 16),
+                                      __uint_as_float((uint32_t)sRawV[(s4 + 1) * kDV + dv] << 16),
+                                      __uint_as_float((uint32_t)sRawV[(s4 + 2) * kDV + dv] << 16),
+                                      __uint_as_float((uint32_t)sRawV[(s4 + 3) * kDV + dv] << 16));
+        *reinterpret_cast<float4*>(sVt + tc::swz_offset(kDV, dv, s4)) = f4;
       }
+      tc::fence_async_smem();
+      mbar_arrive(&bar_v);  // this TMEM worker is done with the raw v tile
       if (issuer) {
         Walker nx = wk;
         nx.next();
+        wait_or_abort(&bar_v, n & 1, abort_flag);
         if (nx.valid()) {
-          // the other buffer held chunk n-1, whose V^T was built before bar_ready(n-1) completed
           const Chunk c = nx.get();
           ++n_tma_issued;
-          tc::mbar_arrive_expect_tx(&bar_tma[buf ^ 1], kC * kDV * 2);
-          tc::tma_load_4d(sm + kOffRawV + (buf ^ 1) * (kC * kDV * 2), &maps.v, &bar_tma[buf ^ 1], 0, c.h,
-                          c.c0, c.b);
+          tc::mbar_arrive_expect_tx(&bar_tma, kC * kDV * 2);
+          tc::tma_load_4d(sm + kOffRawV, &maps.v, &bar_tma, 0, c.h, c.c0, c.b);
         }
       }
-      tc::fence_async_smem();
       tc::tmem_fence_before();
       mbar_arrive(&bar_ready);
       wait_or_abort(&bar_ready, n & 1, abort_flag);
@@ -621,6 +659,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
               tc::mma_tf32_ss(tb + kColH, tc::smem_desc(vt + off, 16, 1024), tc::smem_desc(wt + off, 16, 1024),
                               tc::idesc_tf32(kDV, kM, 0, 0), 1);
             }
+            tc::mma_commit(&bar_t);  // Qh, Wh, Wh^T are free for the next chunk
           }
           // S -> A (rows t = 16*(warp%4) + lane for lane < 16, at TMEM lanes 32*(warp%4) + lane)
           wait_or_abort(&bar_s, n_s & 1, abort_flag);
@@ -667,6 +706,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             tc::mma_tf32_ss(tb + kColH, tc::smem_desc(vt + off, 16, 1024), tc::smem_desc(wt + off, 16, 1024),
                             tc::idesc_tf32(kDV, kM, 0, 0), 1);
           }
+          tc::mma_commit(&bar_t);
           tc::mma_commit(&bar_o);
         }
       } else {
@@ -686,8 +726,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         }
         tc::tmem_wait_st();
         tc::tmem_fence_before();
-        sync_x();  // X1
-        sync_x();  // X2: the row workers have written A and Wh^T
+        sync_x();  // X1: the row workers have written Qh, A and Wh^T
         if (issuer) {
           tc::tmem_fence_after();
           if (!SUMMARY) {
@@ -713,6 +752,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                               tc::idesc_tf32(kDV, kC, 0, 0), 1);
             }
           }
+          tc::mma_commit(&bar_t);
           tc::mma_commit(&bar_o);
         }
       }
@@ -725,7 +765,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       // no MMA or tile load may still be running when the CTA releases its memory
       tc::mma_commit(&bar_o);
       tc::mbar_wait(&bar_o, n & 1);
-      if (n_tma_issued > n) tc::mbar_wait(&bar_tma[n & 1], (n >> 1) & 1);
+      if (n_tma_issued > n) tc::mbar_wait(&bar_tma, n & 1);
     }
   }
 
@@ -811,56 +851,83 @@ Plan plan_for(const rsm_forward_args& a, int sms) {
   return {nseg, seg_chunks};
 }
 
-size_t ws_bytes(const rsm_forward_args& a, const Plan& pl) {
-  if (pl.nseg <= 1) return 0;
-  const size_t per = (size_t)a.B * a.H * pl.nseg;
-  auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
-  return up(per * kM * kDV * 4) + up(per * kM * 4) + up(per * kM * 4);
+size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// Workspace: routing records, then (segmented runs) the segment states, decays and touch flags.
+struct WsLayout {
+  size_t rec, state, D, touch, total;
+};
+WsLayout ws_layout(const rsm_forward_args& a, const Plan& pl) {
+  WsLayout l;
+  const size_t rows = (size_t)a.B * a.T * a.H;
+  l.rec = 0;
+  size_t off = up256(rows * (size_t)route_record_bytes(a.K));
+  l.state = l.D = l.touch = off;
+  if (pl.nseg > 1) {
+    const size_t per = (size_t)a.B * a.H * pl.nseg;
+    l.state = off;
+    off += up256(per * kM * kDV * 4);
+    l.D = off;
+    off += up256(per * kM * 4);
+    l.touch = off;
+    off += up256(per * kM * 4);
+  }
+  l.total = off;
+  return l;
 }
 
 }  // namespace
 
 bool prefill_tc_supported(const rsm_forward_args& a) {
-  return a.qkv_dtype == RSM_BF16 && a.M == kM && a.Dv == kDV && a.K <= kKMax;
+  return a.qkv_dtype == RSM_BF16 && a.M == kM && a.Dv == kDV && a.K <= kKMax && route_records_supported(a.M, a.K);
 }
 
 size_t prefill_tc_workspace_bytes(const rsm_forward_args& a) {
   if (!prefill_tc_supported(a)) return 0;
-  return ws_bytes(a, plan_for(a, sm_count()));
+  return ws_layout(a, plan_for(a, sm_count())).total;
+}
+
+int prefill_tc_launches(const rsm_forward_args& a) {
+  if (!prefill_tc_supported(a) || a.T == 0) return 0;
+  return plan_for(a, sm_count()).nseg > 1 ? 4 : 2;
 }
 
 cudaError_t launch_prefill_tc(const rsm_forward_args& a, cudaStream_t stream) {
   const int sms = sm_count();
   const Plan pl = plan_for(a, sms);
+  const WsLayout wl = ws_layout(a, pl);
+  char* ws = static_cast<char*>(a.workspace);
+  unsigned char* rec = reinterpret_cast<unsigned char*>(ws + wl.rec);
+  const int64_t rows = (int64_t)a.B * a.T * a.H;
+  cudaError_t e = launch_route_records(a.logits, a.f, rows, a.M, a.K, a.decay == RSM_DECAY_SLOT,
+                                       (a.flags & RSM_FLAG_VALIDATE) != 0, rec, a.idx_out, a.score_out, stream);
+  if (e != cudaSuccess) return e;
   Maps maps;
   if (!make_map(&maps.v, a.v, a.B, a.T, a.H, kDV)) return cudaErrorInvalidValue;
   Params p;
   p.B = a.B; p.T = a.T; p.H = a.H; p.K = a.K;
-  p.decay_slot = a.decay == RSM_DECAY_SLOT;
   p.q = static_cast<const __nv_bfloat16*>(a.q);
   p.k = static_cast<const __nv_bfloat16*>(a.k);
-  p.logits = a.logits; p.f = a.f; p.H0 = a.H0;
-  p.o = a.o; p.HT = a.HT; p.idx_out = a.idx_out; p.score_out = a.score_out;
-  p.validate = (a.flags & RSM_FLAG_VALIDATE) != 0;
+  p.rec = rec;
+  p.rec_bytes = route_record_bytes(a.K);
+  p.H0 = a.H0;
+  p.o = a.o; p.HT = a.HT;
   p.nseg = pl.nseg; p.seg_chunks = pl.seg_chunks;
   p.ws_state = nullptr; p.ws_D = nullptr; p.ws_touch = nullptr;
   if (pl.nseg > 1) {
-    const size_t per = (size_t)a.B * a.H * pl.nseg;
-    auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
-    char* w = static_cast<char*>(a.workspace);
-    p.ws_state = reinterpret_cast<float*>(w);
-    p.ws_D = reinterpret_cast<float*>(w + up(per * kM * kDV * 4));
-    p.ws_touch = reinterpret_cast<int*>(w + up(per * kM * kDV * 4) + up(per * kM * 4));
+    p.ws_state = reinterpret_cast<float*>(ws + wl.state);
+    p.ws_D = reinterpret_cast<float*>(ws + wl.D);
+    p.ws_touch = reinterpret_cast<int*>(ws + wl.touch);
   }
-  cudaError_t e0 = cudaFuncSetAttribute(prefill_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-  if (e0 == cudaSuccess)
-    e0 = cudaFuncSetAttribute(prefill_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-  if (e0 != cudaSuccess) return e0;
+  e = cudaFuncSetAttribute(prefill_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(prefill_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (e != cudaSuccess) return e;
   const int64_t pairs = (int64_t)a.B * a.H;
   if (pl.nseg > 1) {
     const int items = (int)(pairs * (pl.nseg - 1));
     prefill_tc_kernel<true><<<std::min(items, sms), kThreads, kSmemBytes, stream>>>(maps, p);
-    cudaError_t e = cudaGetLastError();
+    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     dim3 g((kM * kDV + 255) / 256, (unsigned)pairs);
     segment_scan_kernel<<<g, 256, 0, stream>>>(p);
