@@ -1,16 +1,25 @@
 // decode.cu -- one generation step per (b,h) (rsm_decode_step).
 //
-// Persistent CTAs (three per SM) walk the (b,h) items. Each item's fp32 state H [M, Dv] streams
-// through shared memory in blocks of rows fetched by bulk asynchronous copies into two buffers:
-// while one block is processed, the next block -- of this item or of the next item -- is already
-// in flight, so the copies never wait for the arithmetic. Warp 0 runs the TopK routing of an item
-// and prepares the decay and write weight of each selected slot while that item's first block is
-// still arriving. Every thread applies the sparse update to the rows it covers, writes back only
-// the selected rows, and accumulates o = sum_i q_i H'[i,:] over all M rows.
-// Bytes per (b,h): M*Dv*4 read + K*Dv*4 written + the token's inputs.
+// The step streams the whole fp32 state once: for every (b,h) it reads the M x Dv state, writes
+// back only the K selected rows and produces o = sum_i q_i H'[i,:] (Raven README "Model Structure":
+// the fused recurrent form used for generation). Bytes per (b,h): M*Dv*4 read + K*Dv*4 written +
+// the token's inputs, so the kernel is bound by HBM bandwidth and is organised to keep the copy
+// engine busy without pause:
 //
-// Thread layout: CG = Dv/4 column groups of float4 by RG = floor(256/CG) row groups; thread
-// (rg, cg) covers rows rg, rg+RG, ... of column group cg (a warp reads whole 512-byte rows).
+//   one persistent CTA per SM owns a contiguous range of (b,h) items (ranges differ by at most one
+//   item) and splits the work among three warp roles that meet at mbarriers in shared memory:
+//     producer  (1 thread)   streams the state of its items, block by block (32 KB of rows per
+//                            block), through a ring of kStages buffers with cp.async.bulk;
+//     routers   (kRouters warps) run ahead of the consumers: TopK of the item's logits, then the
+//                            decay a = e^{s f} and write weight w = k (1 - a) of every slot (a = 1,
+//                            w = 0 off the selection), q and v, into a ring of routing slots;
+//     consumers (8 warps)    apply the update to the selected rows of each block, store those rows,
+//                            accumulate the read over all rows, and reduce o at the item's end.
+//   Selected slots carry their decay with the sign bit set (-a), so one load tells a consumer both
+//   whether to write the row and by how much to decay it.
+//
+// Every wait is bounded; on expiry the CTA records RSM_ERR_TIMEOUT, stops, and the producer waits
+// (bounded) for its copies still in flight before the CTA exits.
 #include "common.cuh"
 #include "kernels.h"
 #include "tc.cuh"
@@ -19,9 +28,33 @@ namespace rsm {
 
 namespace {
 
-constexpr int kDecodeThreads = 256;
-constexpr int kBlockBytes = 32 * 1024;  // state rows per bulk copy (one of two buffers)
-constexpr int kCtasPerSm = 3;
+constexpr int kConsumerWarps = 8;
+constexpr int kConsumers = kConsumerWarps * 32;
+constexpr int kRouters = 4;                       // routing warps
+constexpr int kProducerWarp = kConsumerWarps;     // warp 8
+constexpr int kRouterWarp0 = kConsumerWarps + 1;  // warps 9..12
+constexpr int kThreads = (kConsumerWarps + 1 + kRouters) * 32;
+constexpr int kStages = 6;
+constexpr int kStageBytes = 32 * 1024;  // 16 KB blocks measured slower: per-block consumer overhead
+constexpr int kRouteSlotsMax = 8;
+constexpr int kSmemMax = 232448;       // dynamic shared memory per CTA on sm_100
+constexpr int kRedBytes = 2 * 8 * 32 * 16;
+
+// Bytes of one routing slot: a[M], w[M], q[M] (fp32) and v[Dv] (fp32).
+__host__ __device__ constexpr int route_slot_bytes(int M, int Dv) { return (3 * M + Dv) * 4; }
+
+// Routing slots that fit beside the state ring (2 to kRouteSlotsMax).
+__host__ __device__ constexpr int route_slots(int M, int Dv) {
+  return (kSmemMax - kStages * kStageBytes - kRedBytes) / route_slot_bytes(M, Dv) < kRouteSlotsMax
+             ? (kSmemMax - kStages * kStageBytes - kRedBytes) / route_slot_bytes(M, Dv)
+             : kRouteSlotsMax;
+}
+
+struct Smem {
+  unsigned char* stage;  // [kStages][kStageBytes]
+  unsigned char* route;  // [nslots][route_slot_bytes]
+  float4* red;           // [2][kConsumers]
+};
 
 RSM_DEV void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile(
@@ -30,78 +63,116 @@ RSM_DEV void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar
       "l"(src), "r"(bytes), "r"(tc::smem_u32(bar))
       : "memory");
 }
+RSM_DEV void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(tc::smem_u32(bar)) : "memory");
+}
+// Barrier among the consumer warps that also ORs a flag over them (all of them get the result).
+RSM_DEV bool bar_consumers_or(bool flag) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.or.pred p, 1, %2, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)flag), "n"(kConsumers)
+      : "memory");
+  return r != 0;
+}
+
+static_assert(kRedBytes == 2 * kConsumers * 16, "reduction buffer");
+static_assert(route_slots(256, 256) >= kRouters, "routing ring too small for the largest shape");
 
 template <int M, typename TIn>
-__global__ void __launch_bounds__(kDecodeThreads) decode_kernel(rsm_decode_args a) {
+__global__ void __launch_bounds__(kThreads, 1) decode_kernel(rsm_decode_args a) {
   constexpr int E = M / 32;
   const int Dv = a.Dv, K = a.K;
-  const int CG = Dv >> 2;
-  const int RG = kDecodeThreads / CG;
-  const int rows_blk = min(M, kBlockBytes / (Dv * 4));  // rows per block
+  const int rows_blk = min(M, kStageBytes / (Dv * 4));  // state rows per block
   const int nblk = (M + rows_blk - 1) / rows_blk;        // blocks per item
-  const int tid = threadIdx.x;
-  const int cg = tid % CG, rg = tid / CG;
-  const bool active = rg < RG;  // threads past CG*RG only help with the small loads
+  const int slot_bytes = route_slot_bytes(M, Dv);
+  const int nslots = route_slots(M, Dv);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  // this CTA's items: a contiguous range, sizes differing by at most one across CTAs
   const int64_t items = (int64_t)a.B * a.H;
+  const int64_t it0 = items * blockIdx.x / gridDim.x;
+  const int64_t it1 = items * (blockIdx.x + 1) / gridDim.x;
+  const int nitems = (int)(it1 - it0);
 
   extern __shared__ __align__(128) unsigned char dsm[];
-  auto buf = [&](uint32_t j) { return reinterpret_cast<float*>(dsm + (j & 1) * kBlockBytes); };
-  __shared__ float s_a[M], s_w[M], s_q[M];
-  __shared__ unsigned char s_sel[M];
-  __shared__ __align__(16) float s_v[256];
-  __shared__ __align__(16) float s_red[kDecodeThreads * 4];
-  __shared__ __align__(8) uint64_t bar[2];
+  Smem s;
+  s.stage = dsm;
+  s.route = dsm + kStages * kStageBytes;
+  s.red = reinterpret_cast<float4*>(s.route + nslots * slot_bytes);
+  __shared__ __align__(8) uint64_t full[kStages], empty[kStages], rfull[kRouteSlotsMax], rempty[kRouteSlotsMax];
   __shared__ int s_abort;
 
   if (tid == 0) {
-    tc::mbar_init(&bar[0], 1);
-    tc::mbar_init(&bar[1], 1);
+    for (int i = 0; i < kStages; ++i) {
+      tc::mbar_init(&full[i], 1);
+      tc::mbar_init(&empty[i], kConsumerWarps);
+    }
+    for (int i = 0; i < kRouteSlotsMax; ++i) {
+      tc::mbar_init(&rfull[i], 1);
+      tc::mbar_init(&rempty[i], 1);
+    }
     tc::fence_mbar_init();
     s_abort = 0;
   }
   __syncthreads();
-
-  // The CTA's blocks form one stream: (item, block) in order. Block j goes to buffer j & 1.
-  auto issue = [&](int64_t item, int blk, uint32_t j) {
-    const int r0 = blk * rows_blk;
-    const int rows = min(rows_blk, M - r0);
-    const uint32_t bytes = (uint32_t)(rows * Dv * 4);
-    tc::mbar_arrive_expect_tx(&bar[j & 1], bytes);
-    bulk_load(buf(j), a.state + (item * M + r0) * (int64_t)Dv, bytes, &bar[j & 1]);
+  volatile int* abort_flag = &s_abort;
+  auto fail = [&]() {
+    *abort_flag = 1;
+    raise_status(RSM_ERR_TIMEOUT);
   };
-  uint32_t j_issue = 0, j_use = 0;  // blocks issued / consumed by this CTA
-  int64_t nx_item = blockIdx.x;
-  int nx_blk = 0;
-  auto issue_next = [&]() {
-    if (nx_item < items) {
-      issue(nx_item, nx_blk, j_issue++);
-      if (++nx_blk == nblk) {
-        nx_blk = 0;
-        nx_item += gridDim.x;
+
+  if (warp == kProducerWarp) {
+    // ------------------------------------------------------------------------------ producer
+    if (lane == 0) {
+      const int total = nitems * nblk;
+      int n = 0;
+      for (; n < total && !*abort_flag; ++n) {
+        const int st = n % kStages;
+        if (n >= kStages && !tc::mbar_wait(&empty[st], ((n / kStages) - 1) & 1)) {
+          fail();
+          break;
+        }
+        const int64_t item = it0 + n / nblk;
+        const int r0 = (n % nblk) * rows_blk;
+        const uint32_t bytes = (uint32_t)(min(rows_blk, M - r0) * Dv * 4);
+        tc::mbar_arrive_expect_tx(&full[st], bytes);
+        bulk_load(s.stage + st * kStageBytes, a.state + (item * M + r0) * (int64_t)Dv, bytes, &full[st]);
       }
+      // copies still in flight must land before the CTA's shared memory is released
+      for (int m = max(0, n - kStages); m < n; ++m) tc::mbar_wait(&full[m % kStages], (m / kStages) & 1);
     }
-  };
-  if (tid == 0) {
-    issue_next();
-    issue_next();
-  }
-
-  for (int64_t pair = blockIdx.x; pair < items; pair += gridDim.x) {
-    float* state = a.state + pair * (int64_t)M * Dv;
-    // 1. small inputs and the routing of this item (its first block is in flight)
-    const TIn* q = reinterpret_cast<const TIn*>(a.q) + pair * M;
-    const TIn* k = reinterpret_cast<const TIn*>(a.k) + pair * M;
-    const TIn* v = reinterpret_cast<const TIn*>(a.v) + pair * Dv;
-    for (int i = tid; i < M; i += blockDim.x) s_q[i] = In<TIn>::ld(q + i);
-    for (int d = tid; d < Dv; d += blockDim.x) s_v[d] = In<TIn>::ld(v + d);
-    if (tid < 32) {
-      const int lane = tid;
-      float x[E];
+  } else if (warp >= kRouterWarp0) {
+    // ------------------------------------------------------------------------------ routers
+    const int r = warp - kRouterWarp0;
+    for (int m = r; m < nitems && !*abort_flag; m += kRouters) {
+      const int slot = m % nslots;
+      if (m >= nslots && !tc::mbar_wait(&rempty[slot], ((m / nslots) - 1) & 1)) {
+        fail();
+        break;
+      }
+      const int64_t pair = it0 + m;
+      float* sa = reinterpret_cast<float*>(s.route + slot * slot_bytes);
+      float* sw = sa + M;
+      float* sq = sw + M;
+      float* sv = sq + M;
+      const TIn* q = reinterpret_cast<const TIn*>(a.q) + pair * M;
+      const TIn* k = reinterpret_cast<const TIn*>(a.k) + pair * M;
+      const TIn* v = reinterpret_cast<const TIn*>(a.v) + pair * Dv;
+      float x[E], fv[E], kv[E];
       load_row_logits<M>(a.logits + pair * M, lane, x);
-      float fv[E];
 #pragma unroll
-      for (int e = 0; e < E; ++e)
-        fv[e] = (a.decay == RSM_DECAY_SLOT) ? a.f[pair * M + lane * E + e] : a.f[pair];
+      for (int e = 0; e < E; ++e) {
+        const int i = lane * E + e;
+        fv[e] = (a.decay == RSM_DECAY_SLOT) ? a.f[pair * M + i] : a.f[pair];
+        kv[e] = In<TIn>::ld(k + i);
+        sq[i] = In<TIn>::ld(q + i);
+      }
+      for (int d = lane; d < Dv; d += 32) sv[d] = In<TIn>::ld(v + d);
       if (a.flags & RSM_FLAG_VALIDATE) {
         bool bad = false;
 #pragma unroll
@@ -110,80 +181,94 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(rsm_decode_args 
       }
       int32_t* io = a.idx_out ? a.idx_out + pair * K : nullptr;
       float* so = a.score_out ? a.score_out + pair * K : nullptr;
-      const uint32_t sel = warp_topk<M>(x, K, lane, [&](int r, int slot, int e) {
-        if (io) io[r] = slot;
-        if (so) so[r] = sigmoid_f32(x[e]);
+      const uint32_t sel = warp_topk<M>(x, K, lane, [&](int rank, int slot_i, int e) {
+        if (io) io[rank] = slot_i;
+        if (so) so[rank] = sigmoid_f32(x[e]);
       });
 #pragma unroll
       for (int e = 0; e < E; ++e) {
         const int i = lane * E + e;
         if (sel & (1u << e)) {
           const float lam = sigmoid_f32(x[e]) * fv[e];  // log of the decay, <= 0
-          s_sel[i] = 1;
-          s_a[i] = expf(lam);
-          s_w[i] = In<TIn>::ld(k + i) * (-expm1f(lam));  // k_i * (1 - a_i)
+          sa[i] = -expf(lam);                           // sign bit: selected
+          sw[i] = kv[e] * (-expm1f(lam));               // k_i (1 - a_i)
         } else {
-          s_sel[i] = 0;
-          s_a[i] = 1.f;
-          s_w[i] = 0.f;
+          sa[i] = 1.f;
+          sw[i] = 0.f;
         }
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&rfull[slot]);
     }
-    __syncthreads();
-
-    // 2. blocks of rows: sparse update of the selected rows, read over all rows
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    const float4 vv = active ? reinterpret_cast<const float4*>(s_v)[cg] : make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int blk = 0; blk < nblk; ++blk) {
-      const uint32_t j = j_use++;
-      if (!tc::mbar_wait(&bar[j & 1], (j >> 1) & 1)) {
-        if (tid == 0) {
-          s_abort = 1;
-          raise_status(RSM_ERR_TIMEOUT);
-        }
+  } else {
+    // ------------------------------------------------------------------------------ consumers
+    const int CG = Dv >> 2;          // float4 column groups
+    const int RG = kConsumers / CG;  // row groups
+    const int cg = tid % CG, rg = tid / CG;
+    const bool active = rg < RG;
+    int n = 0;
+    for (int m = 0; m < nitems; ++m) {
+      // A thread that sees a failure stops waiting and computing but still reaches the item's
+      // barrier, which ORs the failure over all consumers, so that they leave together.
+      bool ab = false;
+      const int slot = m % nslots;
+      if (!tc::mbar_wait(&rfull[slot], (m / nslots) & 1)) {
+        fail();
+        ab = true;
       }
-      const float* sb = buf(j);
-      const int r0 = blk * rows_blk;
-      const int rows = min(rows_blk, M - r0);
-      if (active) {
-        for (int rr = rg; rr < rows; rr += RG) {
-          const int r = r0 + rr;
-          float4 hv = reinterpret_cast<const float4*>(sb + rr * Dv)[cg];
-          if (s_sel[r]) {
-            const float ar = s_a[r], wr = s_w[r];
-            hv.x = fmaf(ar, hv.x, wr * vv.x);
-            hv.y = fmaf(ar, hv.y, wr * vv.y);
-            hv.z = fmaf(ar, hv.z, wr * vv.z);
-            hv.w = fmaf(ar, hv.w, wr * vv.w);
-            reinterpret_cast<float4*>(state + (int64_t)r * Dv)[cg] = hv;
+      const float* sa = reinterpret_cast<const float*>(s.route + slot * slot_bytes);
+      const float* sw = sa + M;
+      const float* sq = sw + M;
+      const float4 vv = active ? reinterpret_cast<const float4*>(sq + M)[cg] : make_float4(0.f, 0.f, 0.f, 0.f);
+      float* state = a.state + (it0 + m) * (int64_t)M * Dv;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int blk = 0; blk < nblk; ++blk, ++n) {
+        const int st = n % kStages;
+        ab = ab || *abort_flag;
+        if (!ab && !tc::mbar_wait(&full[st], (n / kStages) & 1)) {
+          fail();
+          ab = true;
+        }
+        const float* sb = reinterpret_cast<const float*>(s.stage + st * kStageBytes);
+        const int r0 = blk * rows_blk;
+        const int rows = min(rows_blk, M - r0);
+        if (active && !ab) {
+#pragma unroll 4
+          for (int rr = rg; rr < rows; rr += RG) {
+            const int row = r0 + rr;
+            float4 hv = reinterpret_cast<const float4*>(sb + rr * Dv)[cg];
+            const float as = sa[row];
+            if (__float_as_uint(as) & 0x80000000u) {
+              const float ar = -as, wr = sw[row];
+              hv.x = fmaf(ar, hv.x, wr * vv.x);
+              hv.y = fmaf(ar, hv.y, wr * vv.y);
+              hv.z = fmaf(ar, hv.z, wr * vv.z);
+              hv.w = fmaf(ar, hv.w, wr * vv.w);
+              reinterpret_cast<float4*>(state + (int64_t)row * Dv)[cg] = hv;
+            }
+            const float qr = sq[row];
+            acc.x = fmaf(qr, hv.x, acc.x);
+            acc.y = fmaf(qr, hv.y, acc.y);
+            acc.z = fmaf(qr, hv.z, acc.z);
+            acc.w = fmaf(qr, hv.w, acc.w);
           }
-          const float qr = s_q[r];
-          acc.x = fmaf(qr, hv.x, acc.x);
-          acc.y = fmaf(qr, hv.y, acc.y);
-          acc.z = fmaf(qr, hv.z, acc.z);
-          acc.w = fmaf(qr, hv.w, acc.w);
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[st]);  // this warp is done with the buffer
       }
-      __syncthreads();             // the buffer is consumed ...
-      if (tid == 0) issue_next();  // ... and refilled with the stream's next block
-    }
-    if (active) reinterpret_cast<float4*>(s_red)[rg * CG + cg] = acc;
-    __syncthreads();
-
-    // 3. reduce over the row groups
-    for (int d = tid; d < Dv; d += blockDim.x) {
-      float s = 0.f;
-      for (int g = 0; g < RG; ++g) s += s_red[g * Dv + d];
-      a.o[pair * Dv + d] = s;
-    }
-    __syncthreads();  // small shared arrays are reused by the next item
-    if (s_abort) break;
-  }
-  // a copy still in flight (only after an abort) must land before the CTA leaves
-  if (tid == 0) {
-    while (j_use < j_issue) {
-      const uint32_t j = j_use++;
-      tc::mbar_wait(&bar[j & 1], (j >> 1) & 1);
+      // o = sum over the row groups (double-buffered partials: one barrier per item)
+      float4* red = s.red + (m & 1) * kConsumers;
+      if (active) red[rg * CG + cg] = acc;
+      if (bar_consumers_or(ab || *abort_flag)) break;
+      for (int c = tid; c < CG; c += kConsumers) {
+        float4 o4 = red[c];
+        for (int g = 1; g < RG; ++g) {
+          const float4 p = red[g * CG + c];
+          o4.x += p.x; o4.y += p.y; o4.z += p.z; o4.w += p.w;
+        }
+        reinterpret_cast<float4*>(a.o + (it0 + m) * (int64_t)Dv)[c] = o4;
+      }
+      if (tid == 0) mbar_arrive(&rempty[slot]);  // every consumer is past the routing slot
     }
   }
 }
@@ -195,22 +280,20 @@ int sm_count() {
   return n;
 }
 
+template <int M, typename TIn>
+cudaError_t launch_t(const rsm_decode_args& a, cudaStream_t stream) {
+  const int smem = kStages * kStageBytes + route_slots(M, a.Dv) * route_slot_bytes(M, a.Dv) + kRedBytes;
+  cudaError_t e = cudaFuncSetAttribute(decode_kernel<M, TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  const int64_t items = (int64_t)a.B * a.H;
+  const unsigned grid = (unsigned)std::min<int64_t>(items, (int64_t)sm_count());
+  decode_kernel<M, TIn><<<grid, kThreads, smem, stream>>>(a);
+  return cudaGetLastError();
+}
+
 template <int M>
 cudaError_t launch_m(const rsm_decode_args& a, cudaStream_t stream) {
-  const int smem = 2 * kBlockBytes;
-  const int64_t items = (int64_t)a.B * a.H;
-  const unsigned grid = (unsigned)std::min<int64_t>(items, (int64_t)sm_count() * kCtasPerSm);
-  cudaError_t e;
-  if (a.qkv_dtype == RSM_BF16) {
-    e = cudaFuncSetAttribute(decode_kernel<M, __nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    decode_kernel<M, __nv_bfloat16><<<grid, kDecodeThreads, smem, stream>>>(a);
-  } else {
-    e = cudaFuncSetAttribute(decode_kernel<M, float>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    decode_kernel<M, float><<<grid, kDecodeThreads, smem, stream>>>(a);
-  }
-  return cudaGetLastError();
+  return a.qkv_dtype == RSM_BF16 ? launch_t<M, __nv_bfloat16>(a, stream) : launch_t<M, float>(a, stream);
 }
 
 }  // namespace
