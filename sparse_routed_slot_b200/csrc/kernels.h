@@ -11,14 +11,15 @@ namespace rsm {
 cudaError_t launch_route(const float* logits, int64_t rows, int M, int K, int32_t* idx_out,
                          float* score_out, int validate, cudaStream_t stream);
 
-// Thread-per-row TopK for M = 128, K <= 32 (route_rec.cu): routing records for the tensor prefill
-// (`rec`, route_record_bytes(K) bytes per row) and/or ranked indices and scores; null outputs are
-// skipped. `f` is read only when `rec` is written (or `validate` is set).
+// Thread-per-row TopK for M = 128, K <= 32 (route_rec.cu) over rows given as [B, T, H] (rsm_route:
+// B = H = 1, T = rows). Writes routing records for the tensor prefill (`rec`, route_record_bytes(K)
+// bytes per row, rows in [B, H, T] order; needs f and k) and/or ranked indices and scores in the
+// input row order; null outputs are skipped.
 bool route_records_supported(int M, int K);
 int route_record_bytes(int K);
-cudaError_t launch_route_records(const float* logits, const float* f, int64_t rows, int M, int K, int decay_slot,
-                                 int validate, unsigned char* rec, int32_t* idx_out, float* score_out,
-                                 cudaStream_t stream);
+cudaError_t launch_route_records(const float* logits, const float* f, const void* k, int64_t B, int64_t T,
+                                 int64_t H, int M, int K, int decay_slot, int validate, unsigned char* rec,
+                                 int32_t* idx_out, float* score_out, cudaStream_t stream);
 
 cudaError_t launch_decode(const rsm_decode_args& a, cudaStream_t stream);
 

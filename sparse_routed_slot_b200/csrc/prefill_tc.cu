@@ -17,21 +17,37 @@
 // the state is decayed.
 //
 // The routing is not done here: a thread-per-row kernel (route_rec.cu) has already turned the
-// logits into one record per row (selection mask, selected slots, lam of each), read here.
+// logits into one record per row (selected slots, lam = log of each decay, w = k (1 - a)), stored
+// time-contiguous per (b,h) stream; the chunk's 64 records are read here.
 //
 // Operands are fp32 tiles rounded to nearest tf32 (kind::tf32), accumulated in fp32. The fp32
 // state lives in TMEM as H^T (lane = value column, column = slot); the carry accumulates into it
-// and a tf32-rounded copy feeds the next chunk's read as the A operand straight from TMEM.
-// TMEM columns: [0,128) H^T, [128,256) rounded H^T, [256,320) O^T, [320,384) S (64-lane layout).
+// and a tf32-rounded copy feeds the next chunk's read as the A operand straight from TMEM (the
+// tensor core would truncate fp32, a bias proportional to each output).
+// TMEM columns: [0,128) H^T, [128,256) rounded H^T, [256,320) and [320,384) O^T of even and odd
+// chunks, [384,448) S (64-lane layout); [384,512) U^T, the carry of an exact-path chunk, shares
+// S's columns (an exact chunk has no S, and the next S waits until the epilogue has used U).
 //
-// Warp roles (one persistent CTA per SM, 12 warps):
-//   warps 0-7  row workers, 8 rows of each chunk per warp: the decays of the selected entries of
-//              their rows (one lane per entry), the per-slot product over their rows, then, once
-//              the previous chunk's MMAs have read the operand tiles, their rows of Qh, Wh, Wh^T.
-//              q, k and the records of the next chunk are loaded while this one is processed.
-//   warps 8-11 TMEM workers (one per TMEM lane quarter): outputs of chunk n-1, the decay of the
-//              state and its rounded copy, the V^T tile of chunk n, the S -> A masking. Thread 256
-//              also issues the v tile loads and the MMAs.
+// Warp roles (one persistent CTA per SM, 13 warps):
+//   warps 0-7  row workers; warp w owns tokens 8w..8w+7 of the chunk, lane l slots 4l..4l+3.
+//              A warp scatters the decays of its rows' selected entries into its rows of a dense
+//              per-chunk table (a = 1 elsewhere, the sign bit marks a selected entry), multiplies
+//              along its rows, and exchanges the per-warp products for the in-chunk prefix at its
+//              first row. It then walks its rows: the running product G gives Qh = q G and, at
+//              the selected entries, G itself, from which each entry's owner forms Wh = w / G in
+//              the Wh and Wh^T tiles. q and the records of the next chunk are loaded while this one
+//              is processed.
+//   warp 8     MMA issuer (one thread): v tile loads (two chunks ahead) and the tcgen05.mma of
+//              every chunk, as soon as their operands are ready.
+//   warps 9-12 epilogue (one per TMEM lane quarter): S -> A masking, the decay of the state after
+//              the carry (and the state in and out at item boundaries), the V^T tile of the next
+//              chunk, the output of the chunk from TMEM.
+// Per chunk the issuer runs S = Qh Wh^T (as soon as the row tiles are ready), then, once the
+// state is decayed and the V^T tile is there, O^T = H^T Qh^T and the carry H^T += V^T Wh, and
+// finally O^T += V^T A^T when the epilogue has masked S into A. An exact-path chunk carries into
+// U^T = V^T Wh_end (end-referenced weights) and the epilogue forms H = D H + U.
+// Every mbarrier is waited on by a role that the barrier's next phase depends on, so no waiter
+// can fall two phases behind (which a parity wait cannot tell from zero).
 //
 // Long sequences with few (b,h) streams are split into segments processed in parallel: a summary
 // pass runs the state recurrence of each segment but the last from a zero state and stores
@@ -55,29 +71,28 @@ constexpr int kDV = 128;       // value columns
 constexpr int kKMax = 32;      // largest TopK on this path
 constexpr int kRWarps = 8;     // row workers
 constexpr int kRowsPerWarp = kC / kRWarps;
-constexpr int kThreads = 384;
 constexpr int kRThreads = kRWarps * 32;
-constexpr int kIssuer = kRThreads;       // first thread of the TMEM workers
+constexpr int kIssuerWarp = kRWarps;          // warp 8
+constexpr int kEpiThreads = 4 * 32;
+constexpr int kThreads = (kRWarps + 1 + 4) * 32;
 constexpr float kDMin = 1.80485139e-35f;  // e^-80: fast-path bound on the in-chunk decay
-constexpr int kRecMax = 176;              // routing record bytes for K = 32
 
-constexpr int kColH = 0, kColHr = 128, kColO = 256, kColS = 320, kTmemCols = 512;
+constexpr int kColH = 0, kColHr = 128, kColO = 256, kColS = 384, kColU = 384, kTmemCols = 512;
 
 // Dynamic shared memory (offsets from a 1024-byte aligned base). Operand tiles are K-major in the
 // swizzled format of tc.cuh; Wh^T and V^T are stored transposed because they are contracted over
 // tokens (a tf32 operand cannot be MN-major in this swizzle).
-constexpr int kOffQ = 0;                      // Qh   [64 t][128 slot]   (A of S, B of the read)
-constexpr int kOffW = kOffQ + 32768;          // Wh   [64 s][128 slot]   (B of S); exact path: dense g
-constexpr int kOffWt = kOffW + 32768;         // Wh^T [128 slot][64 s]   (B of the carry)
-constexpr int kOffVt = kOffWt + 32768;        // V^T  [128 dv][64 s]     (A of carry and A.V)
-constexpr int kOffA = kOffVt + 32768;         // A    [64 t][64 s]       (B of A.V)
-constexpr int kOffRawV = kOffA + 16384;       // v tile from TMA, [64][128] bf16
-constexpr int kOffCmp = kOffRawV + 16384;     // per selected entry (a, 1/a, 1-a, lam), [64][KP] float4
-constexpr int kOffRec = kOffCmp + kC * kKMax * 16;                   // records, [8 warps][8 rows][RB]
-constexpr int kOffTot = kOffRec + kRWarps * kRowsPerWarp * kRecMax;  // per-warp slot totals, [2][8][128]
+constexpr int kOffQ = 0;                   // Qh   [64 t][128 slot]   (A of S, B of the read)
+constexpr int kOffW = kOffQ + 32768;       // Wh   [64 s][128 slot]   (B of S); exact path: dense g
+constexpr int kOffWt = kOffW + 32768;      // Wh^T [128 slot][64 s]   (B of the carry)
+constexpr int kOffVt = kOffWt + 32768;     // V^T  [128 dv][64 s]     (A of carry and A.V)
+constexpr int kOffA = kOffVt + 32768;      // A    [64 t][64 s]       (B of A.V)
+constexpr int kOffRawV = kOffA + 16384;    // v tiles from TMA, [2][64][128] bf16
+constexpr int kOffTab = kOffRawV + 32768;  // decay table [64 t][128 slot] fp32 (exact path: lam)
+constexpr int kOffTot = kOffTab + 32768;   // per-warp slot products (sums), [2][8][128]
 constexpr int kOffSmall = kOffTot + 2 * kRWarps * kM * 4;
-// D[2][M], touched[2][M], mask OR [2][8][4], fast[2]
-constexpr int kSmallBytes = (2 * kM + 2 * kM + 2 * kRWarps * 4 + 2) * 4 + 8;
+// D[2][M], fast[2]
+constexpr int kSmallBytes = 2 * kM * 4 + 16;
 constexpr int kSmemBytes = kOffSmall + kSmallBytes + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
@@ -88,8 +103,7 @@ struct Maps {
 struct Params {
   int B, T, H, K;
   const __nv_bfloat16* q;
-  const __nv_bfloat16* k;
-  const unsigned char* rec;  // routing records, rec_bytes per row, rows in [B, T, H] order
+  const unsigned char* rec;  // routing records, rec_bytes per row, rows in [B, H, T] order
   int rec_bytes;
   const float* H0;
   float* o;
@@ -97,7 +111,6 @@ struct Params {
   int nseg, seg_chunks;
   float* ws_state;  // [pairs][nseg][M][Dv]: slot 0 = start state, slot j+1 = summary of segment j
   float* ws_D;      // [pairs][nseg][M]
-  int* ws_touch;    // [pairs][nseg][M]
 };
 
 RSM_DEV float4 bf16x4_to_f32(uint2 r) {
@@ -108,6 +121,15 @@ RSM_DEV float fget(const float4& v, int e) { return e == 0 ? v.x : e == 1 ? v.y 
 RSM_DEV float bf16_at(const __nv_bfloat16* p) {
   return __uint_as_float((uint32_t)(*reinterpret_cast<const uint16_t*>(p)) << 16);
 }
+// v[j] *= d[j] for 32 consecutive slots (d in shared memory, 16-byte aligned).
+RSM_DEV void scale_by(float (&v)[32], const float* d) {
+#pragma unroll
+  for (int j = 0; j < 32; j += 4) {
+    const float4 d4 = *reinterpret_cast<const float4*>(d + j);
+    v[j] *= d4.x; v[j + 1] *= d4.y; v[j + 2] *= d4.z; v[j + 3] *= d4.w;
+  }
+}
+RSM_DEV bool sign_set(float x) { return (__float_as_uint(x) >> 31) != 0u; }
 
 // Bounded mbarrier wait; on expiry records a timeout and raises the CTA abort flag.
 RSM_DEV void wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
@@ -177,40 +199,67 @@ struct Walker {
   }
 };
 
-// A row worker's inputs for one chunk: q and k of its 8 rows (4 slots per lane) and the pieces of
-// its 8 routing records (16 bytes per piece, up to 3 pieces per lane).
+// A row worker's inputs for one chunk: q of its 8 rows (4 slots per lane) and up to 8 entries of
+// its rows' records (groups of 4 consecutive entries: slots, lam, w).
+template <int KP>
 struct RowInputs {
-  uint2 q[kRowsPerWarp], k[kRowsPerWarp];
-  uint4 rec[3];
+  static constexpr int kGroups = KP / 16;  // groups of 4 entries per lane
+  uint2 q[kRowsPerWarp];
+  uint32_t es[kGroups];
+  float4 el[kGroups], ew[kGroups];
 };
 
-template <bool SUMMARY>
-RSM_DEV void load_rows(const Params& p, const Chunk& c, int w, int lane, int n16, RowInputs& in) {
+// Entry group g of lane `lane` in a warp's 8 records of KP entries each: row r, first entry j0.
+RSM_DEV void entry_pos(int lane, int g, int KP, int& r, int& j0) {
+  const int f = (lane + 32 * g) * 4;
+  r = f / KP;
+  j0 = f - r * KP;
+}
+
+template <bool SUMMARY, int KP>
+RSM_DEV void load_rows(const Params& p, const Chunk& c, int w, int lane, RowInputs<KP>& in) {
 #pragma unroll
   for (int r = 0; r < kRowsPerWarp; ++r) {
     const int t = w * kRowsPerWarp + r;
-    in.k[r] = make_uint2(0u, 0u);
     in.q[r] = make_uint2(0u, 0u);
-    if (t < c.nrows) {
+    if (!SUMMARY && t < c.nrows) {
       const int64_t row = ((int64_t)c.b * p.T + c.c0 + t) * p.H + c.h;
-      in.k[r] = reinterpret_cast<const uint2*>(p.k + row * kM)[lane];
-      if (!SUMMARY) in.q[r] = reinterpret_cast<const uint2*>(p.q + row * kM)[lane];
+      in.q[r] = reinterpret_cast<const uint2*>(p.q + row * kM)[lane];
     }
   }
+  const unsigned char* rb = p.rec + ((int64_t)c.pair * p.T + c.c0 + w * kRowsPerWarp) * p.rec_bytes;
 #pragma unroll
-  for (int u = 0; u < 3; ++u) {
-    const int idx = lane + 32 * u;
-    const int r = idx / n16, part = idx - r * n16;
-    const int t = w * kRowsPerWarp + r;
-    in.rec[u] = make_uint4(0u, 0u, 0u, 0u);
-    if (r < kRowsPerWarp && t < c.nrows) {
-      const int64_t row = ((int64_t)c.b * p.T + c.c0 + t) * p.H + c.h;
-      in.rec[u] = *reinterpret_cast<const uint4*>(p.rec + row * p.rec_bytes + part * 16);
+  for (int g = 0; g < RowInputs<KP>::kGroups; ++g) {
+    int r, j0;
+    entry_pos(lane, g, KP, r, j0);
+    in.es[g] = 0u;
+    in.el[g] = make_float4(0.f, 0.f, 0.f, 0.f);
+    in.ew[g] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (r < kRowsPerWarp && w * kRowsPerWarp + r < c.nrows) {
+      const unsigned char* e = rb + r * p.rec_bytes;
+      in.es[g] = *reinterpret_cast<const uint32_t*>(e + j0);
+      in.el[g] = *reinterpret_cast<const float4*>(e + KP + 4 * j0);
+      in.ew[g] = *reinterpret_cast<const float4*>(e + 5 * KP + 4 * j0);
     }
   }
 }
 
-template <bool SUMMARY>
+// Calls fn(r, slot, lam, w) for every valid entry of the lane's groups (row r of the warp).
+template <int KP, class Fn>
+RSM_DEV void for_entries(const RowInputs<KP>& in, int lane, int K, int nrows_w, Fn fn) {
+#pragma unroll
+  for (int g = 0; g < RowInputs<KP>::kGroups; ++g) {
+    int r, j0;
+    entry_pos(lane, g, KP, r, j0);
+    if (r >= kRowsPerWarp || r >= nrows_w) continue;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (j0 + e < K) fn(r, (int)((in.es[g] >> (8 * e)) & 255u), fget(in.el[g], e), fget(in.ew[g], e));
+    }
+  }
+}
+
+template <bool SUMMARY, int KP>
 __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_constant__ Maps maps,
                                                                   const Params p) {
   extern __shared__ unsigned char smem_raw[];
@@ -220,121 +269,98 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
   unsigned char* sWt = sm + kOffWt;
   unsigned char* sVt = sm + kOffVt;
   unsigned char* sA = sm + kOffA;
-  const uint16_t* sRawV = reinterpret_cast<const uint16_t*>(sm + kOffRawV);
-  float4* sCmp = reinterpret_cast<float4*>(sm + kOffCmp);
-  unsigned char* sRec = sm + kOffRec;
+  unsigned char* sRawV = sm + kOffRawV;
+  float* sTab = reinterpret_cast<float*>(sm + kOffTab);
   float* sTot = reinterpret_cast<float*>(sm + kOffTot);
-  float* sDc = reinterpret_cast<float*>(sm + kOffSmall);         // [2][M]
-  int* sTouch = reinterpret_cast<int*>(sDc + 2 * kM);             // [2][M]
-  uint32_t* sOr = reinterpret_cast<uint32_t*>(sTouch + 2 * kM);  // [2][8][4]
-  int* sFast = reinterpret_cast<int*>(sOr + 2 * kRWarps * 4);    // [2]
+  float* sDc = reinterpret_cast<float*>(sm + kOffSmall);    // [2][M]
+  int* sFast = reinterpret_cast<int*>(sDc + 2 * kM);         // [2]
 
-  __shared__ __align__(8) uint64_t bar_tma, bar_v, bar_ready, bar_s, bar_a, bar_t, bar_o, bar_x;
+  // mbarriers (phase k of a barrier = its k-th completion; every role counts the same way)
+  __shared__ __align__(8) uint64_t bar_rdy,  // row tiles of chunk n written         (row threads)
+      bar_tma[2],                             // raw v tile of chunk n landed          (TMA, buffer n&1)
+      bar_vt,                                 // V^T of chunk n written                (epilogue)
+      bar_s,                                  // main pass: S of chunk n done          (MMA commit)
+      bar_a,                                  // main pass: A of chunk n written       (epilogue)
+      bar_t,                                  // read and carry of chunk n done        (MMA commit)
+      bar_o,                                  // every MMA of chunk n done             (MMA commit)
+      bar_h,                                  // state ready for chunk n               (epilogue)
+      bar_of[2],                              // O buffer n&1 stored after chunk n     (epilogue)
+      bar_fin;                                // issuer only: every MMA issued is done (MMA commit)
   __shared__ uint32_t s_tbase;
   __shared__ int s_abort;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const bool row_worker = warp < kRWarps;
   const int T = p.T, H = p.H, K = p.K;
   const int pairs = p.B * H;
   const int segs_here = SUMMARY ? p.nseg - 1 : p.nseg;
   const int items = pairs * segs_here;
-  const int KP = K <= 16 ? 16 : 32;  // entries per row in sCmp
 
-  if (warp == kRWarps) tc::tmem_alloc(&s_tbase, kTmemCols);
+  if (warp == kIssuerWarp) tc::tmem_alloc(&s_tbase, kTmemCols);
   if (tid == 0) {
-    tc::mbar_init(&bar_tma, 1);
-    tc::mbar_init(&bar_v, kThreads - kRThreads);
-    tc::mbar_init(&bar_ready, kThreads);
+    tc::mbar_init(&bar_rdy, kRThreads);
+    tc::mbar_init(&bar_tma[0], 1);
+    tc::mbar_init(&bar_tma[1], 1);
+    tc::mbar_init(&bar_vt, kEpiThreads);
     tc::mbar_init(&bar_s, 1);
-    tc::mbar_init(&bar_a, kThreads - kRThreads);
+    tc::mbar_init(&bar_a, kEpiThreads);
     tc::mbar_init(&bar_t, 1);
     tc::mbar_init(&bar_o, 1);
-    tc::mbar_init(&bar_x, kThreads);
+    tc::mbar_init(&bar_h, kEpiThreads);
+    tc::mbar_init(&bar_of[0], kEpiThreads);
+    tc::mbar_init(&bar_of[1], kEpiThreads);
+    tc::mbar_init(&bar_fin, 1);
     tc::fence_mbar_init();
     s_abort = 0;
   }
-  if (tid == kIssuer) tc::tma_prefetch_desc(&maps.v);
+  if (warp == kIssuerWarp && lane == 0) tc::tma_prefetch_desc(&maps.v);
   tc::tmem_fence_before();
   __syncthreads();
   tc::tmem_fence_after();
   const uint32_t tb = s_tbase;
   volatile int* abort_flag = &s_abort;
-  uint32_t n_x = 0;  // completed phases of bar_x (exact-path synchronisation), kept by every thread
-  auto sync_x = [&]() {
-    mbar_arrive(&bar_x);
-    wait_or_abort(&bar_x, n_x & 1, abort_flag);
-    ++n_x;
-  };
 
   Walker wk;
   wk.start(items, pairs, H, T, p.seg_chunks);
 
-  if (row_worker) {
+  if (warp < kRWarps) {
     // =========================================================================== row workers
     const int w = warp;
-    const int RB = p.rec_bytes, n16 = RB / 16;
-    const int slot_off = 16, lam_off = 16 + ((K + 15) & ~15);
-    unsigned char* myRec = sRec + w * (kRowsPerWarp * kRecMax);  // this warp's 8 records, stride RB
-    const int mw = lane >> 3;                  // mask word holding the lane's 4 slots
-    const int sh = (lane & 7) * 4;             // bit offset of the lane's slots in that word
-    const uint32_t below = (1u << sh) - 1u;    // the word's bits of lower slots
-    const int ej = lane % KP, er = lane / KP;  // entry-parallel mapping: entry ej of row r0 + er
-    const int rpp = 32 / KP;                   // rows per entry pass
-    float Dseg[4] = {1.f, 1.f, 1.f, 1.f};      // summary pass, warp 0: product of the chunk decays
-    int tseg[4] = {0, 0, 0, 0};
+    const int RB = p.rec_bytes;
+    float* tab = sTab + w * kRowsPerWarp * kM;  // this warp's rows of the decay table
+    float Dseg[4] = {1.f, 1.f, 1.f, 1.f};       // summary pass, warp 0: product of the chunk decays
 
-    RowInputs cur;
-    if (wk.valid()) load_rows<SUMMARY>(p, wk.get(), w, lane, n16, cur);
+    RowInputs<KP> cur;
+    if (wk.valid()) load_rows<SUMMARY, KP>(p, wk.get(), w, lane, cur);
     for (uint32_t n = 0; wk.valid(); ++n, wk.next()) {
       const Chunk ck = wk.get();
       const int buf = n & 1;
-      // ---- records into shared memory; the next chunk's inputs start loading
-#pragma unroll
-      for (int u = 0; u < 3; ++u) {
-        const int idx = lane + 32 * u;
-        const int r = idx / n16, part = idx - r * n16;
-        if (r < kRowsPerWarp) *reinterpret_cast<uint4*>(myRec + r * RB + part * 16) = cur.rec[u];
-      }
-      RowInputs nxt;
+      const int nrows_w = ck.nrows - w * kRowsPerWarp;  // rows of this warp inside the chunk
+      RowInputs<KP> nxt;
       {
         Walker nx = wk;
         nx.next();
-        if (nx.valid()) load_rows<SUMMARY>(p, nx.get(), w, lane, n16, nxt);
+        if (nx.valid()) load_rows<SUMMARY, KP>(p, nx.get(), w, lane, nxt);
       }
-      __syncwarp();
-      // ---- decay of every selected entry of the warp's rows (one lane per entry)
-      for (int r0 = 0; r0 < kRowsPerWarp; r0 += rpp) {
-        const int r = r0 + er;
-        const int t = w * kRowsPerWarp + r;
-        if (ej < K && t < ck.nrows) {
-          const float lam = *reinterpret_cast<const float*>(myRec + r * RB + lam_off + 4 * ej);
-          sCmp[t * KP + ej] = make_float4(expf(lam), expf(-lam), -expm1f(lam), lam);
-        }
-      }
-      float* tot = sTot + (buf * kRWarps + w) * kM;
-      reinterpret_cast<float4*>(tot)[lane] = make_float4(1.f, 1.f, 1.f, 1.f);
-      if (lane < 4) {
-        uint32_t om = 0u;
+      // ---- this warp's rows of the decay table: 1 everywhere, -a at the selected entries
 #pragma unroll
-        for (int r = 0; r < kRowsPerWarp; ++r) om |= reinterpret_cast<const uint32_t*>(myRec + r * RB)[lane];
-        sOr[(buf * kRWarps + w) * 4 + lane] = om;
-      }
+      for (int i = 0; i < kRowsPerWarp; ++i)
+        reinterpret_cast<float4*>(tab)[lane + 32 * i] = make_float4(1.f, 1.f, 1.f, 1.f);
       __syncwarp();
-      // per-slot product of the decays over the warp's rows, rows in order
+      for_entries(cur, lane, K, nrows_w, [&](int r, int slot, float lam, float) {
+        tab[r * kM + slot] = -expf(lam);
+      });
+      __syncwarp();
+      // ---- product of the decays over the warp's rows, per slot
+      float P[4] = {1.f, 1.f, 1.f, 1.f};
 #pragma unroll
       for (int r = 0; r < kRowsPerWarp; ++r) {
-        const int t = w * kRowsPerWarp + r;
-        if (lane < K && t < ck.nrows) {
-          const int slot = myRec[r * RB + slot_off + lane];
-          tot[slot] *= sCmp[t * KP + lane].x;
-        }
-        __syncwarp();
+        const float4 a4 = reinterpret_cast<const float4*>(tab + r * kM)[lane];
+        P[0] *= fabsf(a4.x); P[1] *= fabsf(a4.y); P[2] *= fabsf(a4.z); P[3] *= fabsf(a4.w);
       }
+      reinterpret_cast<float4*>(sTot + (buf * kRWarps + w) * kM)[lane] = make_float4(P[0], P[1], P[2], P[3]);
       if (bar_rows_or(*abort_flag != 0)) break;  // every row worker takes the same decision
-      // ---- in-chunk products at the warp's first row (off) and over the chunk (gend)
+      // ---- in-chunk products before the warp's first row (off) and over the chunk (gend)
       float off[4] = {1.f, 1.f, 1.f, 1.f}, gend[4] = {1.f, 1.f, 1.f, 1.f};
-      uint32_t orw = 0u;
 #pragma unroll
       for (int w2 = 0; w2 < kRWarps; ++w2) {
         const float4 t4 = reinterpret_cast<const float4*>(sTot + (buf * kRWarps + w2) * kM)[lane];
@@ -344,109 +370,85 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
           if (w2 < w) off[e] *= tv[e];
           gend[e] *= tv[e];
         }
-        orw |= sOr[(buf * kRWarps + w2) * 4 + mw];
       }
       bool ok = true;
 #pragma unroll
       for (int e = 0; e < 4; ++e) ok &= gend[e] >= kDMin;
       const bool fast = __all_sync(kFull, ok);
-      // ---- the previous chunk's MMAs have read the operand tiles (and the TMEM workers have
-      // finished the chunk before it, whose decay buffer this chunk reuses)
+      // ---- the previous chunk's read and carry have consumed the operand tiles (and the epilogue
+      // has decayed the state of the chunk before it, whose decay buffer this chunk reuses)
       if (n > 0) wait_or_abort(&bar_t, (n - 1) & 1, abort_flag);
       if (w == 0) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int slot = lane * 4 + e;
-          const int touched = (orw >> (sh + e)) & 1u;
           sDc[buf * kM + slot] = gend[e];
-          sTouch[buf * kM + slot] = touched;
           if (SUMMARY) {
-            if (ck.first) {
-              Dseg[e] = 1.f;
-              tseg[e] = 0;
-            }
+            if (ck.first) Dseg[e] = 1.f;
             Dseg[e] *= gend[e];
-            tseg[e] |= touched;
-            if (ck.last) {
-              const int64_t base = ((int64_t)ck.pair * p.nseg + ck.seg + 1) * kM;
-              p.ws_D[base + slot] = Dseg[e];
-              p.ws_touch[base + slot] = tseg[e];
-            }
+            if (ck.last) p.ws_D[((int64_t)ck.pair * p.nseg + ck.seg + 1) * kM + slot] = Dseg[e];
           }
         }
         if (lane == 0) sFast[buf] = fast;
       }
       if (fast) {
-        // ---- this warp's rows of Qh, Wh and Wh^T
-        float G[4], Gi[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          G[e] = off[e];
-          Gi[e] = 1.f / off[e];
-        }
-        float stash[4][4];
+        // ---- walk the warp's rows: Qh = q G, and G at the selected entries (0 elsewhere)
+        float G[4] = {off[0], off[1], off[2], off[3]};
 #pragma unroll
         for (int r = 0; r < kRowsPerWarp; ++r) {
           const int t = w * kRowsPerWarp + r;
-          const uint4 mk = *reinterpret_cast<const uint4*>(myRec + r * RB);
-          const uint32_t wd = mw == 0 ? mk.x : mw == 1 ? mk.y : mw == 2 ? mk.z : mk.w;
-          int base = __popc(wd & below) + (mw > 0 ? __popc(mk.x) : 0) + (mw > 1 ? __popc(mk.y) : 0) +
-                     (mw > 2 ? __popc(mk.z) : 0);
+          const float4 a4 = reinterpret_cast<const float4*>(tab + r * kM)[lane];
+          const float av[4] = {a4.x, a4.y, a4.z, a4.w};
           const float4 q4 = bf16x4_to_f32(cur.q[r]);
-          const float4 k4 = bf16x4_to_f32(cur.k[r]);
-          float qh[4], wh[4];
+          float qh[4], gw[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            float wt = 0.f;
-            if ((wd >> (sh + e)) & 1u) {
-              const float4 c = sCmp[t * KP + base];
-              ++base;
-              G[e] *= c.x;
-              Gi[e] *= c.y;
-              wt = fget(k4, e) * c.z * Gi[e];  // k (1 - a) / G_t
-            }
-            qh[e] = SUMMARY ? 0.f : tc::to_tf32(fget(q4, e) * G[e]);
-            wh[e] = tc::to_tf32(wt);
-            stash[r & 3][e] = wh[e];
+            G[e] *= fabsf(av[e]);
+            qh[e] = tc::to_tf32(fget(q4, e) * G[e]);
+            gw[e] = (SUMMARY || sign_set(av[e])) ? G[e] : 0.f;
           }
-          if (!SUMMARY) {
+          if (!SUMMARY)
             *reinterpret_cast<float4*>(sQ + tc::swz_offset(kC, t, lane * 4)) = make_float4(qh[0], qh[1], qh[2], qh[3]);
-            *reinterpret_cast<float4*>(sW + tc::swz_offset(kC, t, lane * 4)) = make_float4(wh[0], wh[1], wh[2], wh[3]);
-          }
-          if ((r & 3) == 3) {
-            // four consecutive tokens of each of the lane's slots; the slot order is rotated by
-            // lane pair so that 8 neighbouring lanes hit 8 different 16-byte bank groups
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const int e = (j + (lane >> 1)) & 3;
-              float4 v4;
-              v4.x = e == 0 ? stash[0][0] : e == 1 ? stash[0][1] : e == 2 ? stash[0][2] : stash[0][3];
-              v4.y = e == 0 ? stash[1][0] : e == 1 ? stash[1][1] : e == 2 ? stash[1][2] : stash[1][3];
-              v4.z = e == 0 ? stash[2][0] : e == 1 ? stash[2][1] : e == 2 ? stash[2][2] : stash[2][3];
-              v4.w = e == 0 ? stash[3][0] : e == 1 ? stash[3][1] : e == 2 ? stash[3][2] : stash[3][3];
-              *reinterpret_cast<float4*>(sWt + tc::swz_offset(kM, lane * 4 + e, t - 3)) = v4;
-            }
-          }
+          *reinterpret_cast<float4*>(sW + tc::swz_offset(kC, t, lane * 4)) = make_float4(gw[0], gw[1], gw[2], gw[3]);
         }
-        tc::fence_async_smem();
-        mbar_arrive(&bar_ready);
-      } else {
-        // ---- exact path (rare), with the TMEM workers: dense g (log domain, in the Wh region),
-        // the Qh tile, the end-referenced Wh^T and A from pairwise sums, exponents <= 0
-        mbar_arrive(&bar_ready);
-        sync_x();  // X0: every row worker is past the product totals; the TMEM workers decay H
-        float* totL = sTot + (buf * kRWarps + w) * kM;  // now: per-warp sums of lam
-        reinterpret_cast<float4*>(totL)[lane] = make_float4(0.f, 0.f, 0.f, 0.f);
+        // this warp's token columns of Wh^T start at zero
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int slot = lane * 4 + e;
+          *reinterpret_cast<float4*>(sWt + tc::swz_offset(kM, slot, w * kRowsPerWarp)) = make_float4(0.f, 0.f, 0.f, 0.f);
+          *reinterpret_cast<float4*>(sWt + tc::swz_offset(kM, slot, w * kRowsPerWarp + 4)) =
+              make_float4(0.f, 0.f, 0.f, 0.f);
+        }
         __syncwarp();
+        // ---- each entry's owner: Wh = w / G_t (finite: G_t >= gend >= e^-80)
+        for_entries(cur, lane, K, nrows_w, [&](int r, int slot, float, float wv) {
+          const int t = w * kRowsPerWarp + r;
+          float* gp = reinterpret_cast<float*>(sW + tc::swz_offset(kC, t, slot));
+          const float wh = tc::to_tf32(__fdividef(wv, *gp));
+          if (!SUMMARY) *gp = wh;
+          *reinterpret_cast<float*>(sWt + tc::swz_offset(kM, slot, t)) = wh;
+        });
+        tc::fence_async_smem();
+        mbar_arrive(&bar_rdy);
+      } else {
+        // ---- exact path (rare): log-domain table and dense g (in the Wh region), the Qh tile,
+        // the end-referenced Wh^T and A from pairwise sums, exponents <= 0. The issuer runs the
+        // read, the carry into U and A.V; the epilogue then forms H = D H + U.
+        if (n > 0) wait_or_abort(&bar_o, (n - 1) & 1, abort_flag);  // A.V of the chunk before is done with A
+        bar_rows();  // every row worker is past the product totals
+#pragma unroll
+        for (int i = 0; i < kRowsPerWarp; ++i)
+          reinterpret_cast<float4*>(tab)[lane + 32 * i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        __syncwarp();
+        for_entries(cur, lane, K, nrows_w, [&](int r, int slot, float lam, float) { tab[r * kM + slot] = lam; });
+        __syncwarp();
+        float S[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int r = 0; r < kRowsPerWarp; ++r) {
-          const int t = w * kRowsPerWarp + r;
-          if (lane < K && t < ck.nrows) {
-            const int slot = myRec[r * RB + slot_off + lane];
-            totL[slot] += sCmp[t * KP + lane].w;
-          }
-          __syncwarp();
+          const float4 l4 = reinterpret_cast<const float4*>(tab + r * kM)[lane];
+          S[0] += l4.x; S[1] += l4.y; S[2] += l4.z; S[3] += l4.w;
         }
+        reinterpret_cast<float4*>(sTot + (buf * kRWarps + w) * kM)[lane] = make_float4(S[0], S[1], S[2], S[3]);
         bar_rows();
         float g[4] = {0.f, 0.f, 0.f, 0.f};
         for (int w2 = 0; w2 < w; ++w2) {
@@ -457,213 +459,201 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
 #pragma unroll
         for (int r = 0; r < kRowsPerWarp; ++r) {
           const int t = w * kRowsPerWarp + r;
-          const uint4 mk = *reinterpret_cast<const uint4*>(myRec + r * RB);
-          const uint32_t wd = mw == 0 ? mk.x : mw == 1 ? mk.y : mw == 2 ? mk.z : mk.w;
-          int base = __popc(wd & below) + (mw > 0 ? __popc(mk.x) : 0) + (mw > 1 ? __popc(mk.y) : 0) +
-                     (mw > 2 ? __popc(mk.z) : 0);
-          const float4 q4 = bf16x4_to_f32(cur.q[r]);
-          float qh[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            if ((wd >> (sh + e)) & 1u) {
-              g[e] += sCmp[t * KP + base].w;
-              ++base;
-            }
-            qh[e] = SUMMARY ? 0.f : tc::to_tf32(fget(q4, e) * expf(g[e]));
-          }
+          const float4 l4 = reinterpret_cast<const float4*>(tab + r * kM)[lane];
+          g[0] += l4.x; g[1] += l4.y; g[2] += l4.z; g[3] += l4.w;
           reinterpret_cast<float4*>(dg + t * kM)[lane] = make_float4(g[0], g[1], g[2], g[3]);
-          if (!SUMMARY)
-            *reinterpret_cast<float4*>(sQ + tc::swz_offset(kC, t, lane * 4)) = make_float4(qh[0], qh[1], qh[2], qh[3]);
-        }
-        // write weight of every selected entry, w = k (1 - a), into its (unused) 1/a field
-        for (int r0 = 0; r0 < kRowsPerWarp; r0 += rpp) {
-          const int r = r0 + er;
-          const int t = w * kRowsPerWarp + r;
-          if (ej < K && t < ck.nrows) {
-            const int slot = myRec[r * RB + slot_off + ej];
-            const int64_t row = ((int64_t)ck.b * T + ck.c0 + t) * H + ck.h;
-            sCmp[t * KP + ej].y = bf16_at(p.k + row * kM + slot) * sCmp[t * KP + ej].z;
+          if (!SUMMARY) {
+            const float4 q4 = bf16x4_to_f32(cur.q[r]);
+            *reinterpret_cast<float4*>(sQ + tc::swz_offset(kC, t, lane * 4)) =
+                make_float4(tc::to_tf32(q4.x * expf(g[0])), tc::to_tf32(q4.y * expf(g[1])),
+                            tc::to_tf32(q4.z * expf(g[2])), tc::to_tf32(q4.w * expf(g[3])));
           }
         }
-        for (int e = tid; e < kC * kM / 4; e += kRThreads)
-          reinterpret_cast<float4*>(sWt)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
-        bar_rows();
-        const int nrows = ck.nrows;
-        for (int e = tid; e < nrows * KP; e += kRThreads) {
-          const int t = e / KP, j = e % KP;
-          if (j >= K) continue;
-          const unsigned char* rt = sRec + (t / kRowsPerWarp) * (kRowsPerWarp * kRecMax) + (t % kRowsPerWarp) * RB;
-          const int i = rt[slot_off + j];
-          const float gend_i = dg[(kC - 1) * kM + i];
-          *reinterpret_cast<float*>(sWt + tc::swz_offset(kM, i, t)) =
-              tc::to_tf32(sCmp[t * KP + j].y * expf(gend_i - dg[t * kM + i]));
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int slot = lane * 4 + e;
+          *reinterpret_cast<float4*>(sWt + tc::swz_offset(kM, slot, w * kRowsPerWarp)) = make_float4(0.f, 0.f, 0.f, 0.f);
+          *reinterpret_cast<float4*>(sWt + tc::swz_offset(kM, slot, w * kRowsPerWarp + 4)) =
+              make_float4(0.f, 0.f, 0.f, 0.f);
         }
+        bar_rows();  // dense g complete (row 63 holds the chunk totals)
+        for_entries(cur, lane, K, nrows_w, [&](int r, int slot, float, float wv) {
+          const int t = w * kRowsPerWarp + r;
+          *reinterpret_cast<float*>(sWt + tc::swz_offset(kM, slot, t)) =
+              tc::to_tf32(wv * expf(dg[(kC - 1) * kM + slot] - dg[t * kM + slot]));
+        });
         if (!SUMMARY) {
+          const int nrows = ck.nrows;
+          const unsigned char* rb = p.rec + ((int64_t)ck.pair * T + ck.c0) * RB;
           for (int e = tid; e < kC * kC; e += kRThreads) {
             const int t = e / kC, s = e % kC;
             float acc = 0.f;
             if (s <= t && t < nrows) {
-              const unsigned char* rs = sRec + (s / kRowsPerWarp) * (kRowsPerWarp * kRecMax) + (s % kRowsPerWarp) * RB;
               const int64_t rowt = ((int64_t)ck.b * T + ck.c0 + t) * H + ck.h;
+              const unsigned char* rs = rb + s * RB;
               for (int j = 0; j < K; ++j) {
-                const int i = rs[slot_off + j];
-                const float qti = bf16_at(p.q + rowt * kM + i);
-                acc = fmaf(qti * sCmp[s * KP + j].y, expf(dg[t * kM + i] - dg[s * kM + i]), acc);
+                const int i = rs[j];
+                const float wj = reinterpret_cast<const float*>(rs + 5 * KP)[j];
+                acc = fmaf(bf16_at(p.q + rowt * kM + i) * wj, expf(dg[t * kM + i] - dg[s * kM + i]), acc);
               }
             }
             *reinterpret_cast<float*>(sA + tc::swz_offset(kC, t, s)) = tc::to_tf32(acc);
           }
         }
         tc::fence_async_smem();
-        sync_x();  // X1
+        mbar_arrive(&bar_rdy);
       }
       cur = nxt;
     }
-  } else {
-    // =========================================================================== TMEM workers
-    const int dv = tid - kRThreads;                 // TMEM lane = value column
-    const uint32_t sub_lane = (uint32_t)((warp & 3) * 32);
-    const bool issuer = tid == kIssuer;
-    uint32_t n_s = 0, n_tma_issued = 0;
-    Chunk prev;
-    prev.nrows = 0;
-    bool have_prev = false, fast_prev = true;
-
-    // outputs of chunk `prev`, then the decay of the state (or, at the item's end, the state out)
-    auto finish_prev = [&](uint32_t n_prev) {
-      wait_or_abort(&bar_o, n_prev & 1, abort_flag);
-      tc::tmem_fence_after();
-      if (!SUMMARY) {
-        float* orow = p.o + (((int64_t)prev.b * T + prev.c0) * H + prev.h) * kDV + dv;
-        const int64_t ostride = (int64_t)H * kDV;
+  } else if (warp == kIssuerWarp) {
+    // =========================================================================== MMA issuer
+    if (lane == 0) {
+      uint32_t n = 0, n_tma = 0;
+      auto load_v = [&](const Walker& at, uint32_t j) {  // v tile of the walker's chunk, as chunk j
+        if (!at.valid()) return;
+        const Chunk c = at.get();
+        tc::mbar_arrive_expect_tx(&bar_tma[j & 1], kC * kDV * 2);
+        tc::tma_load_4d(sRawV + (j & 1) * (kC * kDV * 2), &maps.v, &bar_tma[j & 1], 0, c.h, c.c0, c.b);
+        ++n_tma;
+      };
+      {
+        Walker nx = wk;
+        load_v(nx, 0);
+        nx.next();
+        load_v(nx, 1);
+      }
+      const uint32_t q = tc::smem_u32(sQ), wsm = tc::smem_u32(sW), wt = tc::smem_u32(sWt),
+                     vt = tc::smem_u32(sVt), a = tc::smem_u32(sA);
+      auto mma_read = [&](uint32_t ob) {  // O^T = H^T Qh^T (state read from TMEM)
 #pragma unroll 1
-        for (int c = 0; c < kC; c += 32) {
-          float ov[32];
-          tc::tmem_ld32(tc::tmem_addr(tb, sub_lane, kColO + c), ov);
-          tc::tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (c + j < prev.nrows) orow[(int64_t)(c + j) * ostride] = ov[j];
+        for (int j = 0; j < kM / 8; ++j) {
+          const uint32_t off = (j >> 2) * (kC * 128) + (j & 3) * 32;
+          tc::mma_tf32_ts(tb + kColO + ob, tb + kColHr + 8 * j, tc::smem_desc(q + off, 16, 1024),
+                          tc::idesc_tf32(kDV, kC, 0, 0), j > 0);
         }
+      };
+      auto mma_carry = [&](uint32_t col, bool acc) {  // H^T += V^T Wh, or U^T = V^T Wh
+#pragma unroll 1
+        for (int j = 0; j < kC / 8; ++j) {
+          const uint32_t off = (j >> 2) * (kM * 128) + (j & 3) * 32;
+          tc::mma_tf32_ss(tb + col, tc::smem_desc(vt + off, 16, 1024), tc::smem_desc(wt + off, 16, 1024),
+                          tc::idesc_tf32(kDV, kM, 0, 0), (acc || j > 0) ? 1u : 0u);
+        }
+      };
+      auto mma_av = [&](uint32_t ob) {  // O^T += V^T A^T
+#pragma unroll 1
+        for (int j = 0; j < kC / 8; ++j) {
+          const uint32_t offa = (j >> 2) * (kC * 128) + (j & 3) * 32;
+          const uint32_t offv = (j >> 2) * (kDV * 128) + (j & 3) * 32;
+          tc::mma_tf32_ss(tb + kColO + ob, tc::smem_desc(vt + offv, 16, 1024), tc::smem_desc(a + offa, 16, 1024),
+                          tc::idesc_tf32(kDV, kC, 0, 0), 1);
+        }
+      };
+      bool prev_exact = false;
+      for (; wk.valid() && !*abort_flag; ++n, wk.next()) {
+        const uint32_t ob = (n & 1) * kC;  // O buffer of this chunk
+        wait_or_abort(&bar_rdy, n & 1, abort_flag);
+        const bool fast = sFast[n & 1] != 0;
+        tc::tmem_fence_after();
+        if (!SUMMARY) {
+          if (fast && prev_exact) {  // S overwrites the columns of the previous chunk's U
+            wait_or_abort(&bar_h, n & 1, abort_flag);
+            tc::tmem_fence_after();
+          }
+          if (fast) {
+#pragma unroll 1
+            for (int j = 0; j < kM / 8; ++j) {  // S = Qh Wh^T
+              const uint32_t off = (j >> 2) * (kC * 128) + (j & 3) * 32;
+              tc::mma_tf32_ss(tb + kColS, tc::smem_desc(q + off, 16, 1024), tc::smem_desc(wsm + off, 16, 1024),
+                              tc::idesc_tf32(64, kC, 0, 0), j > 0);
+            }
+          }
+          tc::mma_commit(&bar_s);  // every main-pass chunk: tells the epilogue the chunk is ready
+        }
+        wait_or_abort(&bar_h, n & 1, abort_flag);  // state ready
+        if (!SUMMARY && n >= 2) wait_or_abort(&bar_of[n & 1], ((n - 2) >> 1) & 1, abort_flag);  // O buffer free
+        wait_or_abort(&bar_vt, n & 1, abort_flag);  // V^T written
+        tc::tmem_fence_after();
+        {
+          // the raw v buffer of this chunk is free again: load the chunk two ahead into it
+          Walker nx = wk;
+          nx.next();
+          nx.next();
+          load_v(nx, n + 2);
+        }
+        if (!SUMMARY) mma_read(ob);
+        mma_carry(fast ? kColH : kColU, fast);
+        tc::mma_commit(&bar_t);
+        if (!SUMMARY) {
+          wait_or_abort(&bar_a, n & 1, abort_flag);
+          tc::tmem_fence_after();
+          mma_av(ob);
+        }
+        tc::mma_commit(&bar_o);
+        prev_exact = !fast;
       }
-      const float* Dp = sDc + (n_prev & 1) * kM;
-      const int* Tp = sTouch + (n_prev & 1) * kM;
-      float* dst = nullptr;
-      if (prev.last) {
-        if (SUMMARY) dst = p.ws_state + ((int64_t)prev.pair * p.nseg + prev.seg + 1) * kM * kDV;
-        else if (prev.seg == p.nseg - 1 && p.HT) dst = p.HT + (int64_t)prev.pair * kM * kDV;
-      }
+      // no MMA or tile load may still be running when the CTA releases its memory (a barrier of
+      // its own: another phase of bar_o could overtake the epilogue's last wait on it)
+      tc::mma_commit(&bar_fin);
+      tc::mbar_wait(&bar_fin, 0);
+      for (uint32_t j = n; j < n_tma; ++j) tc::mbar_wait(&bar_tma[j & 1], (j >> 1) & 1);
+    }
+    __syncwarp();  // the whole warp reaches the CTA barrier and the TMEM release together
+  } else {
+    // =========================================================================== epilogue
+    const uint32_t sub_lane = (uint32_t)((warp & 3) * 32);
+    const int dv = (int)sub_lane + lane;  // TMEM lane = value column
+
+    // the state of chunk ck's item into TMEM (H0, a segment start state, or zeros)
+    auto load_state = [&](const Chunk& ck) {
+      const float* Hs = nullptr;
+      if (!SUMMARY)
+        Hs = p.nseg > 1 ? p.ws_state + ((int64_t)ck.pair * p.nseg + ck.seg) * kM * kDV
+                        : (p.H0 ? p.H0 + (int64_t)ck.pair * kM * kDV : nullptr);
 #pragma unroll 1
       for (int c = 0; c < kM; c += 32) {
-        float hv[32];
-        tc::tmem_ld32(tc::tmem_addr(tb, sub_lane, kColH + c), hv);
-        tc::tmem_wait_ld();
-        if (fast_prev) {
+        float v[32];
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (Tp[c + j]) hv[j] *= Dp[c + j];
-        }
-        if (prev.last) {
-          if (dst) {
+        for (int j = 0; j < 32; ++j) v[j] = Hs ? Hs[(c + j) * kDV + dv] : 0.f;
+        tc::tmem_st32(tc::tmem_addr(tb, sub_lane, kColH + c), v);
 #pragma unroll
-            for (int j = 0; j < 32; ++j) dst[(c + j) * kDV + dv] = hv[j];
-          }
-        } else {
-          if (fast_prev) tc::tmem_st32(tc::tmem_addr(tb, sub_lane, kColH + c), hv);
-#pragma unroll
-          for (int j = 0; j < 32; ++j) hv[j] = tc::to_tf32(hv[j]);
-          tc::tmem_st32(tc::tmem_addr(tb, sub_lane, kColHr + c), hv);
-        }
+        for (int j = 0; j < 32; ++j) v[j] = tc::to_tf32(v[j]);
+        tc::tmem_st32(tc::tmem_addr(tb, sub_lane, kColHr + c), v);
       }
       tc::tmem_wait_st();
     };
-
-    if (issuer && wk.valid()) {
-      const Chunk c = wk.get();
-      ++n_tma_issued;
-      tc::mbar_arrive_expect_tx(&bar_tma, kC * kDV * 2);
-      tc::tma_load_4d(sm + kOffRawV, &maps.v, &bar_tma, 0, c.h, c.c0, c.b);
+    // V^T tile of chunk j (thread = value column; conflict-free 16-byte stores)
+    auto make_vt = [&](uint32_t j) {
+      wait_or_abort(&bar_tma[j & 1], (j >> 1) & 1, abort_flag);
+      const uint16_t* raw = reinterpret_cast<const uint16_t*>(sRawV + (j & 1) * (kC * kDV * 2));
+#pragma unroll 4
+      for (int s4 = 0; s4 < kC; s4 += 4) {
+        const float4 f4 = make_float4(__uint_as_float((uint32_t)raw[(s4 + 0) * kDV + dv] << 16),
+                                      __uint_as_float((uint32_t)raw[(s4 + 1) * kDV + dv] << 16),
+                                      __uint_as_float((uint32_t)raw[(s4 + 2) * kDV + dv] << 16),
+                                      __uint_as_float((uint32_t)raw[(s4 + 3) * kDV + dv] << 16));
+        *reinterpret_cast<float4*>(sVt + tc::swz_offset(kDV, dv, s4)) = f4;
+      }
+      tc::fence_async_smem();
+      mbar_arrive(&bar_vt);
+    };
+    if (wk.valid()) {
+      load_state(wk.get());
+      tc::tmem_fence_before();
+      mbar_arrive(&bar_h);  // phase 0: the first chunk's state
+      make_vt(0);
     }
     uint32_t n = 0;
     for (; wk.valid() && !*abort_flag; ++n, wk.next()) {
       const Chunk ck = wk.get();
-      const int buf = n & 1;
-      if (have_prev) finish_prev(n - 1);
-      if (ck.first) {
-        // start state of the item into TMEM (fp32 and its tf32-rounded copy)
-        const float* Hs = nullptr;
-        if (!SUMMARY)
-          Hs = p.nseg > 1 ? p.ws_state + ((int64_t)ck.pair * p.nseg + ck.seg) * kM * kDV
-                          : (p.H0 ? p.H0 + (int64_t)ck.pair * kM * kDV : nullptr);
-#pragma unroll 1
-        for (int c = 0; c < kM; c += 32) {
-          float v[32];
-#pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = Hs ? Hs[(c + j) * kDV + dv] : 0.f;
-          tc::tmem_st32(tc::tmem_addr(tb, sub_lane, kColH + c), v);
-#pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = tc::to_tf32(v[j]);
-          tc::tmem_st32(tc::tmem_addr(tb, sub_lane, kColHr + c), v);
-        }
-        tc::tmem_wait_st();
-      }
-      // V^T tile of this chunk (thread = value column; conflict-free 16-byte stores)
-      wait_or_abort(&bar_tma, n & 1, abort_flag);
-#pragma unroll 4
-      for (int s4 = 0; s4 < kC; s4 += 4) {
-        const float4 f4 = make_float4(__uint_as_float((uint32_t)sRawV[(s4 + 0) * kDV + dv] << 16),
-                                      __uint_as_float((uint32_t)sRawV[(s4 + 1) * kDV + dv] << 16),
-                                      __uint_as_float((uint32_t)sRawV[(s4 + 2) * kDV + dv] << 16),
-                                      __uint_as_float((uint32_t)sRawV[(s4 + 3) * kDV + dv] << 16));
-        *reinterpret_cast<float4*>(sVt + tc::swz_offset(kDV, dv, s4)) = f4;
-      }
-      tc::fence_async_smem();
-      mbar_arrive(&bar_v);  // this TMEM worker is done with the raw v tile
-      if (issuer) {
-        Walker nx = wk;
-        nx.next();
-        wait_or_abort(&bar_v, n & 1, abort_flag);
-        if (nx.valid()) {
-          const Chunk c = nx.get();
-          ++n_tma_issued;
-          tc::mbar_arrive_expect_tx(&bar_tma, kC * kDV * 2);
-          tc::tma_load_4d(sm + kOffRawV, &maps.v, &bar_tma, 0, c.h, c.c0, c.b);
-        }
-      }
-      tc::tmem_fence_before();
-      mbar_arrive(&bar_ready);
-      wait_or_abort(&bar_ready, n & 1, abort_flag);
-      const bool fast = sFast[buf] != 0;
-      const uint32_t q = tc::smem_u32(sQ), w = tc::smem_u32(sW), wt = tc::smem_u32(sWt),
-                     vt = tc::smem_u32(sVt), a = tc::smem_u32(sA);
-      if (fast) {
-        if (!SUMMARY) {
-          if (issuer) {
-            tc::tmem_fence_after();
-#pragma unroll 1
-            for (int j = 0; j < kM / 8; ++j) {  // S = Qh Wh^T
-              const uint32_t off = (j >> 2) * (kC * 128) + (j & 3) * 32;
-              tc::mma_tf32_ss(tb + kColS, tc::smem_desc(q + off, 16, 1024), tc::smem_desc(w + off, 16, 1024),
-                              tc::idesc_tf32(64, kC, 0, 0), j > 0);
-            }
-            tc::mma_commit(&bar_s);
-#pragma unroll 1
-            for (int j = 0; j < kM / 8; ++j) {  // O^T = Hr^T Qh^T (state read from TMEM)
-              const uint32_t off = (j >> 2) * (kC * 128) + (j & 3) * 32;
-              tc::mma_tf32_ts(tb + kColO, tb + kColHr + 8 * j, tc::smem_desc(q + off, 16, 1024),
-                              tc::idesc_tf32(kDV, kC, 0, 0), j > 0);
-            }
-#pragma unroll 1
-            for (int j = 0; j < kC / 8; ++j) {  // H^T += V^T Wh (carry)
-              const uint32_t off = (j >> 2) * (kM * 128) + (j & 3) * 32;
-              tc::mma_tf32_ss(tb + kColH, tc::smem_desc(vt + off, 16, 1024), tc::smem_desc(wt + off, 16, 1024),
-                              tc::idesc_tf32(kDV, kM, 0, 0), 1);
-            }
-            tc::mma_commit(&bar_t);  // Qh, Wh, Wh^T are free for the next chunk
-          }
+      const float* Dn = sDc + (n & 1) * kM;
+      bool fast;
+      if (!SUMMARY) {
+        wait_or_abort(&bar_s, n & 1, abort_flag);
+        tc::tmem_fence_after();
+        fast = sFast[n & 1] != 0;
+        if (fast) {
           // S -> A (rows t = 16*(warp%4) + lane for lane < 16, at TMEM lanes 32*(warp%4) + lane)
-          wait_or_abort(&bar_s, n_s & 1, abort_flag);
-          tc::tmem_fence_after();
           const int t = (warp & 3) * 16 + lane;
 #pragma unroll 1
           for (int c = 0; c < kC; c += 32) {
@@ -683,101 +673,90 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             }
           }
           tc::fence_async_smem();
-          tc::tmem_fence_before();
-          mbar_arrive(&bar_a);
-          if (issuer) {
-            wait_or_abort(&bar_a, n_s & 1, abort_flag);
-            tc::tmem_fence_after();
-#pragma unroll 1
-            for (int j = 0; j < kC / 8; ++j) {  // O^T += V^T A^T
-              const uint32_t offa = (j >> 2) * (kC * 128) + (j & 3) * 32;
-              const uint32_t offv = (j >> 2) * (kDV * 128) + (j & 3) * 32;
-              tc::mma_tf32_ss(tb + kColO, tc::smem_desc(vt + offv, 16, 1024), tc::smem_desc(a + offa, 16, 1024),
-                              tc::idesc_tf32(kDV, kC, 0, 0), 1);
-            }
-            tc::mma_commit(&bar_o);
-          }
-          ++n_s;
-        } else if (issuer) {
-          tc::tmem_fence_after();
-#pragma unroll 1
-          for (int j = 0; j < kC / 8; ++j) {  // H^T += V^T Wh (carry)
-            const uint32_t off = (j >> 2) * (kM * 128) + (j & 3) * 32;
-            tc::mma_tf32_ss(tb + kColH, tc::smem_desc(vt + off, 16, 1024), tc::smem_desc(wt + off, 16, 1024),
-                            tc::idesc_tf32(kDV, kM, 0, 0), 1);
-          }
-          tc::mma_commit(&bar_t);
-          tc::mma_commit(&bar_o);
         }
-      } else {
-        // ---- exact path: decay the state by this chunk first (end-referenced carry weights)
-        sync_x();  // X0
-        const float* Dc = sDc + buf * kM;
-        const int* Tc = sTouch + buf * kM;
+        tc::tmem_fence_before();
+        mbar_arrive(&bar_a);  // every main-pass chunk (an exact chunk's A comes from the row workers)
+      }
+      // ---- after the carry: the state of the chunk end (fast: H = D H; exact: H = D H + U), the
+      // item's state out at its end, the next item's state in at its start
+      wait_or_abort(&bar_t, n & 1, abort_flag);
+      tc::tmem_fence_after();
+      if (SUMMARY) fast = sFast[n & 1] != 0;
+      Walker nx = wk;
+      nx.next();
+      float* dst = nullptr;
+      if (ck.last) {
+        if (SUMMARY) dst = p.ws_state + ((int64_t)ck.pair * p.nseg + ck.seg + 1) * kM * kDV;
+        else if (ck.seg == p.nseg - 1 && p.HT) dst = p.HT + (int64_t)ck.pair * kM * kDV;
+      }
 #pragma unroll 1
-        for (int c = 0; c < kM; c += 32) {
-          float hv[32];
-          tc::tmem_ld32(tc::tmem_addr(tb, sub_lane, kColH + c), hv);
+      for (int c = 0; c < kM; c += 32) {
+        float hv[32];
+        tc::tmem_ld32(tc::tmem_addr(tb, sub_lane, kColH + c), hv);
+        if (!fast) {
+          float uv[32];
+          tc::tmem_ld32(tc::tmem_addr(tb, sub_lane, kColU + c), uv);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; j += 4) {
+            const float4 d4 = *reinterpret_cast<const float4*>(Dn + c + j);
+            hv[j] = fmaf(d4.x, hv[j], uv[j]);
+            hv[j + 1] = fmaf(d4.y, hv[j + 1], uv[j + 1]);
+            hv[j + 2] = fmaf(d4.z, hv[j + 2], uv[j + 2]);
+            hv[j + 3] = fmaf(d4.w, hv[j + 3], uv[j + 3]);
+          }
+        } else {
+          tc::tmem_wait_ld();
+          scale_by(hv, Dn + c);  // slots not selected in the chunk: D = 1 exactly
+        }
+        if (ck.last) {
+          if (dst) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) dst[(c + j) * kDV + dv] = hv[j];
+          }
+        } else {
+          tc::tmem_st32(tc::tmem_addr(tb, sub_lane, kColH + c), hv);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) hv[j] = tc::to_tf32(hv[j]);
+          tc::tmem_st32(tc::tmem_addr(tb, sub_lane, kColHr + c), hv);
+        }
+      }
+      tc::tmem_wait_st();
+      if (ck.last && nx.valid()) load_state(nx.get());
+      tc::tmem_fence_before();
+      mbar_arrive(&bar_h);  // phase n+1: the state of the next chunk
+      // ---- every MMA of this chunk is done: the next V^T, then this chunk's output
+      wait_or_abort(&bar_o, n & 1, abort_flag);
+      tc::tmem_fence_after();
+      if (nx.valid()) make_vt(n + 1);
+      if (!SUMMARY) {
+        float* orow = p.o + (((int64_t)ck.b * T + ck.c0) * H + ck.h) * kDV + dv;
+        const int64_t ostride = (int64_t)H * kDV;
+#pragma unroll 1
+        for (int c = 0; c < kC; c += 32) {
+          float ov[32];
+          tc::tmem_ld32(tc::tmem_addr(tb, sub_lane, kColO + (n & 1) * kC + c), ov);
           tc::tmem_wait_ld();
 #pragma unroll
           for (int j = 0; j < 32; ++j)
-            if (Tc[c + j]) hv[j] *= Dc[c + j];
-          tc::tmem_st32(tc::tmem_addr(tb, sub_lane, kColH + c), hv);
+            if (c + j < ck.nrows) orow[(int64_t)(c + j) * ostride] = ov[j];
         }
-        tc::tmem_wait_st();
         tc::tmem_fence_before();
-        sync_x();  // X1: the row workers have written Qh, A and Wh^T
-        if (issuer) {
-          tc::tmem_fence_after();
-          if (!SUMMARY) {
-#pragma unroll 1
-            for (int j = 0; j < kM / 8; ++j) {
-              const uint32_t off = (j >> 2) * (kC * 128) + (j & 3) * 32;
-              tc::mma_tf32_ts(tb + kColO, tb + kColHr + 8 * j, tc::smem_desc(q + off, 16, 1024),
-                              tc::idesc_tf32(kDV, kC, 0, 0), j > 0);
-            }
-          }
-#pragma unroll 1
-          for (int j = 0; j < kC / 8; ++j) {
-            const uint32_t off = (j >> 2) * (kM * 128) + (j & 3) * 32;
-            tc::mma_tf32_ss(tb + kColH, tc::smem_desc(vt + off, 16, 1024), tc::smem_desc(wt + off, 16, 1024),
-                            tc::idesc_tf32(kDV, kM, 0, 0), 1);
-          }
-          if (!SUMMARY) {
-#pragma unroll 1
-            for (int j = 0; j < kC / 8; ++j) {
-              const uint32_t offa = (j >> 2) * (kC * 128) + (j & 3) * 32;
-              const uint32_t offv = (j >> 2) * (kDV * 128) + (j & 3) * 32;
-              tc::mma_tf32_ss(tb + kColO, tc::smem_desc(vt + offv, 16, 1024), tc::smem_desc(a + offa, 16, 1024),
-                              tc::idesc_tf32(kDV, kC, 0, 0), 1);
-            }
-          }
-          tc::mma_commit(&bar_t);
-          tc::mma_commit(&bar_o);
-        }
+        mbar_arrive(&bar_of[n & 1]);
       }
-      prev = ck;
-      have_prev = true;
-      fast_prev = fast;
-    }
-    if (have_prev && !*abort_flag) finish_prev(n - 1);
-    if (issuer) {
-      // no MMA or tile load may still be running when the CTA releases its memory
-      tc::mma_commit(&bar_o);
-      tc::mbar_wait(&bar_o, n & 1);
-      if (n_tma_issued > n) tc::mbar_wait(&bar_tma, n & 1);
     }
   }
 
   tc::tmem_fence_before();
   __syncthreads();
   tc::tmem_fence_after();
-  if (warp == kRWarps) tc::tmem_dealloc(tb, kTmemCols);
+  if (warp == kIssuerWarp) tc::tmem_dealloc(tb, kTmemCols);
 }
 
 // Combines the segment summaries of each (b,h) into start states:
-// state[0] = H0 (or 0); state[j] = D_{j-1} * state[j-1] + U_{j-1} on the slots touched in
-// segment j-1 (the summary of segment j-1 is stored in slot j and is replaced in place).
+// state[0] = H0 (or 0); state[j] = D_{j-1} * state[j-1] + U_{j-1} (the summary of segment j-1 is
+// stored in slot j and is replaced in place). A slot with D = 1 and U = 0 (not selected in the
+// segment) keeps its bits.
 __global__ void __launch_bounds__(256) segment_scan_kernel(const Params p) {
   const int pair = blockIdx.y;
   const int e = blockIdx.x * blockDim.x + threadIdx.x;  // element (slot, column)
@@ -785,11 +764,11 @@ __global__ void __launch_bounds__(256) segment_scan_kernel(const Params p) {
   const int i = e / kDV;
   float* st = p.ws_state + (int64_t)pair * p.nseg * kM * kDV;
   const float* D = p.ws_D + (int64_t)pair * p.nseg * kM;
-  const int* touch = p.ws_touch + (int64_t)pair * p.nseg * kM;
   float hcur = p.H0 ? p.H0[(int64_t)pair * kM * kDV + e] : 0.f;
   st[e] = hcur;
   for (int j = 1; j < p.nseg; ++j) {
-    if (touch[j * kM + i]) hcur = fmaf(D[j * kM + i], hcur, st[(int64_t)j * kM * kDV + e]);
+    const float d = D[j * kM + i], u = st[(int64_t)j * kM * kDV + e];
+    if (d != 1.f || u != 0.f) hcur = fmaf(d, hcur, u);
     st[(int64_t)j * kM * kDV + e] = hcur;
   }
 }
@@ -853,27 +832,49 @@ Plan plan_for(const rsm_forward_args& a, int sms) {
 
 size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-// Workspace: routing records, then (segmented runs) the segment states, decays and touch flags.
+// Workspace: routing records, then (segmented runs) the segment states and decays.
 struct WsLayout {
-  size_t rec, state, D, touch, total;
+  size_t rec, state, D, total;
 };
 WsLayout ws_layout(const rsm_forward_args& a, const Plan& pl) {
   WsLayout l;
   const size_t rows = (size_t)a.B * a.T * a.H;
   l.rec = 0;
   size_t off = up256(rows * (size_t)route_record_bytes(a.K));
-  l.state = l.D = l.touch = off;
+  l.state = l.D = off;
   if (pl.nseg > 1) {
     const size_t per = (size_t)a.B * a.H * pl.nseg;
     l.state = off;
     off += up256(per * kM * kDV * 4);
     l.D = off;
     off += up256(per * kM * 4);
-    l.touch = off;
-    off += up256(per * kM * 4);
   }
   l.total = off;
   return l;
+}
+
+// Summary pass + segment scan (segmented runs only), then the main pass.
+template <int KP>
+cudaError_t launch_passes(const Maps& maps, const Params& p, const Plan& pl, int64_t pairs, int sms,
+                          cudaStream_t stream) {
+  cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel<false, KP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kSmemBytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(prefill_tc_kernel<true, KP>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (e != cudaSuccess) return e;
+  if (pl.nseg > 1) {
+    const int items = (int)(pairs * (pl.nseg - 1));
+    prefill_tc_kernel<true, KP><<<std::min(items, sms), kThreads, kSmemBytes, stream>>>(maps, p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    dim3 g((kM * kDV + 255) / 256, (unsigned)pairs);
+    segment_scan_kernel<<<g, 256, 0, stream>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  const int64_t items = pairs * pl.nseg;
+  prefill_tc_kernel<false, KP><<<(unsigned)std::min<int64_t>(items, sms), kThreads, kSmemBytes, stream>>>(maps, p);
+  return cudaGetLastError();
 }
 
 }  // namespace
@@ -898,8 +899,7 @@ cudaError_t launch_prefill_tc(const rsm_forward_args& a, cudaStream_t stream) {
   const WsLayout wl = ws_layout(a, pl);
   char* ws = static_cast<char*>(a.workspace);
   unsigned char* rec = reinterpret_cast<unsigned char*>(ws + wl.rec);
-  const int64_t rows = (int64_t)a.B * a.T * a.H;
-  cudaError_t e = launch_route_records(a.logits, a.f, rows, a.M, a.K, a.decay == RSM_DECAY_SLOT,
+  cudaError_t e = launch_route_records(a.logits, a.f, a.k, a.B, a.T, a.H, a.M, a.K, a.decay == RSM_DECAY_SLOT,
                                        (a.flags & RSM_FLAG_VALIDATE) != 0, rec, a.idx_out, a.score_out, stream);
   if (e != cudaSuccess) return e;
   Maps maps;
@@ -907,36 +907,18 @@ cudaError_t launch_prefill_tc(const rsm_forward_args& a, cudaStream_t stream) {
   Params p;
   p.B = a.B; p.T = a.T; p.H = a.H; p.K = a.K;
   p.q = static_cast<const __nv_bfloat16*>(a.q);
-  p.k = static_cast<const __nv_bfloat16*>(a.k);
   p.rec = rec;
   p.rec_bytes = route_record_bytes(a.K);
   p.H0 = a.H0;
   p.o = a.o; p.HT = a.HT;
   p.nseg = pl.nseg; p.seg_chunks = pl.seg_chunks;
-  p.ws_state = nullptr; p.ws_D = nullptr; p.ws_touch = nullptr;
+  p.ws_state = nullptr; p.ws_D = nullptr;
   if (pl.nseg > 1) {
     p.ws_state = reinterpret_cast<float*>(ws + wl.state);
     p.ws_D = reinterpret_cast<float*>(ws + wl.D);
-    p.ws_touch = reinterpret_cast<int*>(ws + wl.touch);
   }
-  e = cudaFuncSetAttribute(prefill_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(prefill_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-  if (e != cudaSuccess) return e;
   const int64_t pairs = (int64_t)a.B * a.H;
-  if (pl.nseg > 1) {
-    const int items = (int)(pairs * (pl.nseg - 1));
-    prefill_tc_kernel<true><<<std::min(items, sms), kThreads, kSmemBytes, stream>>>(maps, p);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    dim3 g((kM * kDV + 255) / 256, (unsigned)pairs);
-    segment_scan_kernel<<<g, 256, 0, stream>>>(p);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-  }
-  const int64_t items = pairs * pl.nseg;
-  prefill_tc_kernel<false><<<(unsigned)std::min<int64_t>(items, sms), kThreads, kSmemBytes, stream>>>(maps, p);
-  return cudaGetLastError();
+  return a.K <= 16 ? launch_passes<16>(maps, p, pl, pairs, sms, stream) : launch_passes<32>(maps, p, pl, pairs, sms, stream);
 }
 
 }  // namespace rsm
