@@ -127,12 +127,7 @@ rsm_status rsm_route(const float* logits, int64_t rows, int M, int K, int32_t* i
   RSM_REQUIRE_PTR(logits, "logits");
   RSM_REQUIRE_PTR(idx_out, "idx_out");
   RSM_OPTIONAL_PTR(score_out, "score_out");
-  // M = 128 with K <= 32: the thread-per-row selection kernel; other sizes: one warp per row
-  cudaError_t e = rsm::route_records_supported(M, K)
-                      ? rsm::launch_route_records(logits, nullptr, nullptr, 1, rows, 1, M, K, 0, 0, nullptr, idx_out,
-                                                  score_out, static_cast<cudaStream_t>(stream))
-                      : rsm::launch_route(logits, rows, M, K, idx_out, score_out, 0,
-                                          static_cast<cudaStream_t>(stream));
+  cudaError_t e = rsm::launch_route(logits, rows, M, K, idx_out, score_out, 0, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? RSM_OK : cuda_fail(e, "rsm_route launch");
 }
 

@@ -11,10 +11,9 @@ namespace rsm {
 cudaError_t launch_route(const float* logits, int64_t rows, int M, int K, int32_t* idx_out,
                          float* score_out, int validate, cudaStream_t stream);
 
-// Thread-per-row TopK for M = 128, K <= 32 (route_rec.cu) over rows given as [B, T, H] (rsm_route:
-// B = H = 1, T = rows). Writes routing records for the tensor prefill (`rec`, route_record_bytes(K)
-// bytes per row, rows in [B, H, T] order; needs f and k) and/or ranked indices and scores in the
-// input row order; null outputs are skipped.
+// Routing records for the tensor prefill (route_rec.cu, M = 128, K <= 32) over rows given as
+// [B, T, H]: route_record_bytes(K) bytes per row, rows in [B, H, T] order; also the ranked
+// indices and scores in the input row order when idx_out / score_out are not null.
 bool route_records_supported(int M, int K);
 int route_record_bytes(int K);
 cudaError_t launch_route_records(const float* logits, const float* f, const void* k, int64_t B, int64_t T,

@@ -163,8 +163,9 @@ struct Chunk {
 };
 
 // The CTA walks its items (item = blockIdx.x + j*gridDim.x) and each item's chunks in order.
+// The item's coordinates are computed once per item (integer division is not cheap here).
 struct Walker {
-  int items, pairs, H, T, seg_chunks, item, c0, t0, t1;
+  int items, pairs, H, T, seg_chunks, item, c0, t0, t1, pair, seg, b, h;
   __device__ void start(int items_, int pairs_, int H_, int T_, int seg_chunks_) {
     items = items_; pairs = pairs_; H = H_; T = T_; seg_chunks = seg_chunks_;
     item = blockIdx.x;
@@ -172,7 +173,10 @@ struct Walker {
   }
   __device__ void set_item() {
     if (item >= items) return;
-    const int seg = item / pairs;
+    seg = item / pairs;
+    pair = item - seg * pairs;
+    b = pair / H;
+    h = pair - b * H;
     t0 = seg * seg_chunks * kC;
     t1 = min(T, t0 + seg_chunks * kC);
     c0 = t0;
@@ -180,10 +184,10 @@ struct Walker {
   __device__ bool valid() const { return item < items; }
   __device__ Chunk get() const {
     Chunk c;
-    c.pair = item % pairs;
-    c.seg = item / pairs;
-    c.b = c.pair / H;
-    c.h = c.pair % H;
+    c.pair = pair;
+    c.seg = seg;
+    c.b = b;
+    c.h = h;
     c.c0 = c0;
     c.nrows = min(kC, t1 - c0);
     c.first = c0 == t0;

@@ -1,8 +1,8 @@
-// route_rec.cu -- TopK routing, one THREAD per row (M = 128 slots, K <= 32).
+// route_rec.cu -- routing records for the tensor-core prefill (M = 128 slots, K <= 32).
 //
-// Used by rsm_route (indices and scores in rank order) and by the tensor-core prefill, which
-// reads compact routing records instead of the logits (Raven README "How Raven Works":
-// route_scores = TopK(sigmoid(r_proj(x))); "Model Structure": a = exp(score * f)):
+// The chunk kernels of the tensor-core prefill read compact routing records instead of the
+// logits (Raven README "How Raven Works": route_scores = TopK(sigmoid(r_proj(x))); "Model
+// Structure": a = exp(score * f)):
 //
 //   record (route_record_bytes(K) = 9 * KP bytes, KP = 16 for K <= 16 else 32; rows in
 //   [B, H, T] order, so the records of one (b,h) stream are contiguous along time):
@@ -12,28 +12,36 @@
 //   Entries are in rank order (logit descending, slot ascending) except that logits agreeing in
 //   their upper 25 key bits may be listed in slot order; the set is always exact.
 //
-// Selection (router scores are monotone in the logits, so TopK of the scores = TopK of the
-// logits; -0 ties +0): each logit becomes a packed 32-bit key, its order-preserving bit pattern
-// with the low 7 bits replaced by (127 - slot), which makes every key distinct and breaks ties to
-// the lower slot. The top N (N = 16 or 32 >= K) keys come from a bitonic network in registers: the
-// row is read in groups of N logits straight from global memory (the next group is in flight while
-// the current one is sorted), each group is sorted and merged into the running top N (the larger
-// half of two sorted runs is bitonic; one half-cleaner cascade sorts it). Dropping the low 7 bits
-// can only misorder logits whose upper 25 key bits agree; if the K-th and (K+1)-th keys share them,
-// or ranked outputs are requested and two of the first K share them, the row is finished by an
-// exact selection over the full keys instead.
+// Two threads per row. A warp takes 16 consecutive rows and copies them into shared memory with
+// asynchronous 16-byte copies (one 512-byte row per warp instruction), into one of two buffers per
+// warp, so the next 16 rows arrive while the current ones are ranked. Each thread of the pair
+// ranks half of the row's slots; the two sorted halves are merged through shuffles. Selection (router scores are monotone in the
+// logits, so TopK of the scores = TopK of the logits; -0 ties +0): each logit becomes a packed
+// 32-bit key, its order-preserving bit pattern with the low 7 bits replaced by (127 - slot), which
+// makes every key distinct and breaks ties to the lower slot. The top N (N = 16 or 32 >= K) keys
+// come from a bitonic network in registers: each group of N is sorted and merged into the running
+// top N (the larger half of two sorted runs is bitonic; one half-cleaner cascade sorts it).
+// Dropping the low 7 bits can only misorder logits whose upper 25 key bits agree; if the K-th and
+// (K+1)-th keys share them, or ranked outputs are requested and two of the first K share them,
+// the whole warp ranks that row exactly with the tournament of common.cuh instead.
 #include <algorithm>
 
 #include "common.cuh"
 #include "kernels.h"
+#include "tc.cuh"
 
 namespace rsm {
 
 namespace {
 
 constexpr int kRM = 128;              // slots on this path
-constexpr int kThreads = 128;
-constexpr uint32_t kCoarse = ~0x7Fu;  // key bits above the slot field
+constexpr int kRowFloats = kRM + 4;    // staged row stride (16-byte pad: conflict-free float4 reads)
+constexpr int kWarps = 4;              // warps per CTA
+constexpr int kThreads = kWarps * 32;
+constexpr int kRowsPerTask = 16;       // rows per warp task (two threads per row)
+constexpr int kBufBytes = kRowsPerTask * kRowFloats * 4;  // one warp's staged rows
+constexpr int kSmem = kWarps * 2 * kBufBytes;
+constexpr uint32_t kCoarse = ~0x7Fu;   // key bits above the slot field
 
 RSM_DEV uint32_t packed_key(float x, int slot) { return (order_key(x) & kCoarse) | (uint32_t)(127 - slot); }
 
@@ -76,25 +84,12 @@ RSM_DEV void merge_top(uint32_t (&top)[N], const uint32_t (&g)[N], uint32_t& dro
   }
 }
 
-RSM_DEV bool has_bit(const uint32_t (&m)[4], int slot) {
-  const int w = slot >> 5;
-  const uint32_t word = w == 0 ? m[0] : w == 1 ? m[1] : w == 2 ? m[2] : m[3];
-  return (word >> (slot & 31)) & 1u;
+RSM_DEV void cp_async16(void* smem, const void* gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(tc::smem_u32(smem)), "l"(gmem) : "memory");
 }
-RSM_DEV void set_bit(uint32_t (&m)[4], int slot) {
-  const uint32_t bit = 1u << (slot & 31);
-  const int w = slot >> 5;
-  m[0] |= w == 0 ? bit : 0u;
-  m[1] |= w == 1 ? bit : 0u;
-  m[2] |= w == 2 ? bit : 0u;
-  m[3] |= w == 3 ? bit : 0u;
-}
-
-template <int N>
-RSM_DEV void load_group(const float* row, int g, float4 (&v)[N / 4]) {
-#pragma unroll
-  for (int i = 0; i < N / 4; ++i) v[i] = __ldg(reinterpret_cast<const float4*>(row + g * N) + i);
-}
+RSM_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+RSM_DEV void cp_async_wait_prev() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+RSM_DEV void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 struct Rows {
   const float* logits;
@@ -107,9 +102,8 @@ struct Rows {
   float* score_out;
 };
 
-// The lam and w of one selected slot of input row `ir`.
-RSM_DEV void entry_values(const Rows& R, int64_t ir, int slot, float fh, float& s, float& lam, float& w) {
-  const float x = __ldg(R.logits + ir * kRM + slot);
+// The score, lam and w of one selected slot of input row `ir` (x = its logit).
+RSM_DEV void entry_values(const Rows& R, int64_t ir, int slot, float x, float fh, float& s, float& lam, float& w) {
   s = sigmoid_f32(x);
   const float fv = R.decay_slot ? __ldg(R.f + ir * kRM + slot) : fh;
   lam = s * fv;
@@ -120,56 +114,100 @@ RSM_DEV void entry_values(const Rows& R, int64_t ir, int slot, float fh, float& 
 template <int N, bool VALIDATE>
 __global__ void __launch_bounds__(kThreads) route_rec_kernel(const Rows R) {
   constexpr int KP = N;  // record entries
+  extern __shared__ __align__(128) unsigned char smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rl = lane >> 1, half = lane & 1;  // row of the task, half of the row (slots 64*half..)
   const int K = R.K;
   const int64_t rows = R.B * R.H * R.T;
-  for (int64_t p = (int64_t)blockIdx.x * kThreads + threadIdx.x; p < rows; p += (int64_t)gridDim.x * kThreads) {
-    // p enumerates rows in [B, H, T] order; ir is the row's index in the [B, T, H] input layout
-    const int64_t bh = p / R.T, t = p - bh * R.T;
-    const int64_t b = bh / R.H, h = bh - b * R.H;
-    const int64_t ir = (b * R.T + t) * R.H + h;
-    const float* xr = R.logits + ir * kRM;
-    const float fh = (R.f && !R.decay_slot) ? __ldg(R.f + ir) : 0.f;
+  const int64_t tasks = (rows + kRowsPerTask - 1) / kRowsPerTask;
+  const int64_t stride = (int64_t)gridDim.x * kWarps;
+  unsigned char* wbuf = smem + warp * 2 * kBufBytes;
+  // input row index (in the [B, T, H] layout) of row p = 16*task + r of the [B, H, T] order:
+  // one division per warp and task (lane 0), then a walk along the stream
+  auto input_row = [&](int64_t task, int r) {
+    int64_t b = 0, h = 0, t = 0;
+    if (lane == 0) {
+      const int64_t p0 = task * kRowsPerTask;
+      const int64_t bh = p0 / R.T;
+      t = p0 - bh * R.T;
+      b = bh / R.H;
+      h = bh - b * R.H;
+    }
+    b = __shfl_sync(kFull, b, 0);
+    h = __shfl_sync(kFull, h, 0);
+    t = __shfl_sync(kFull, t, 0) + r;
+    while (t >= R.T) {  // past the end of the stream: the next (b,h)
+      t -= R.T;
+      if (++h == R.H) {
+        h = 0;
+        ++b;
+      }
+    }
+    return (b * R.T + t) * R.H + h;
+  };
+  // the warp copies the 16 rows of task `task` into buffer j&1 (16 bytes per lane per row)
+  auto stage = [&](int64_t task, uint32_t j) {
+    if (task < tasks) {
+      const int64_t ir0 = input_row(task, lane & 15);  // lane r (r < 16) knows row r's index
+      for (int r = 0; r < kRowsPerTask; ++r) {
+        const int64_t irr = __shfl_sync(kFull, ir0, r);
+        if (task * kRowsPerTask + r < rows)
+          cp_async16(wbuf + (j & 1) * kBufBytes + (r * kRowFloats + lane * 4) * 4, R.logits + irr * kRM + lane * 4);
+      }
+    }
+    cp_async_commit();
+  };
+  const int64_t task0 = (int64_t)blockIdx.x * kWarps + warp;
+  stage(task0, 0);
+  uint32_t j = 0;
+  for (int64_t task = task0; task < tasks; task += stride, ++j) {
+    stage(task + stride, j + 1);  // the next rows arrive while these are ranked
+    cp_async_wait_prev();
+    __syncwarp();
+    const int64_t p = task * kRowsPerTask + rl;
+    const int64_t ir = input_row(task, rl);
+    const bool live = p < rows;  // both lanes of a pair agree
+    const float* xr = reinterpret_cast<const float*>(wbuf + (j & 1) * kBufBytes) + rl * kRowFloats;
+    const float fh = (R.decay_slot || !live) ? 0.f : __ldg(R.f + ir);
 
-    // ---- top N packed keys
+    // ---- top N packed keys of this thread's half of the row, then of the whole row
     uint32_t top[N], g[N], dropped = 0u;
     bool bad = false;
-    float4 cur[N / 4], nxt[N / 4];
     auto keys = [&](int grp, uint32_t (&dst)[N]) {
 #pragma unroll
       for (int i = 0; i < N / 4; ++i) {
-        const int s0 = grp * N + 4 * i;
-        dst[4 * i] = packed_key(cur[i].x, s0);
-        dst[4 * i + 1] = packed_key(cur[i].y, s0 + 1);
-        dst[4 * i + 2] = packed_key(cur[i].z, s0 + 2);
-        dst[4 * i + 3] = packed_key(cur[i].w, s0 + 3);
-        if (VALIDATE)
-          bad |= !finite_f32(cur[i].x) || !finite_f32(cur[i].y) || !finite_f32(cur[i].z) || !finite_f32(cur[i].w);
+        const int s0 = half * (kRM / 2) + grp * N + 4 * i;
+        const float4 v = *reinterpret_cast<const float4*>(xr + s0);
+        dst[4 * i] = packed_key(v.x, s0);
+        dst[4 * i + 1] = packed_key(v.y, s0 + 1);
+        dst[4 * i + 2] = packed_key(v.z, s0 + 2);
+        dst[4 * i + 3] = packed_key(v.w, s0 + 3);
+        if (VALIDATE) bad |= !finite_f32(v.x) || !finite_f32(v.y) || !finite_f32(v.z) || !finite_f32(v.w);
       }
     };
-    load_group<N>(xr, 0, cur);
-    load_group<N>(xr, 1, nxt);
     keys(0, top);
     sort_desc<N>(top);
 #pragma unroll 1
-    for (int grp = 1; grp < kRM / N; ++grp) {
-#pragma unroll
-      for (int i = 0; i < N / 4; ++i) cur[i] = nxt[i];
-      if (grp + 1 < kRM / N) load_group<N>(xr, grp + 1, nxt);
+    for (int grp = 1; grp < kRM / 2 / N; ++grp) {
       keys(grp, g);
       sort_desc<N>(g);
       merge_top<N>(top, g, dropped);
     }
-    if (VALIDATE && R.f) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) g[i] = __shfl_xor_sync(kFull, top[i], 1);  // the partner's half
+    merge_top<N>(top, g, dropped);  // both lanes now hold the row's top N
+    dropped = max(dropped, __shfl_xor_sync(kFull, dropped, 1));
+    if (VALIDATE && live) {
       if (R.decay_slot) {
-        for (int s = 0; s < kRM; ++s) {
+        for (int s = half * (kRM / 2); s < (half + 1) * (kRM / 2); ++s) {
           const float fv = __ldg(R.f + ir * kRM + s);
           bad |= !finite_f32(fv) || fv > 0.f;
         }
       } else {
         bad |= !finite_f32(fh) || fh > 0.f;
       }
+      if (bad) raise_status(RSM_ERR_NONFINITE);
     }
-    if (VALIDATE && bad) raise_status(RSM_ERR_NONFINITE);
 
     // ---- is the coarse order enough? (the K-th and (K+1)-th keys; neighbours among the first K)
     uint32_t kth = 0xffffffffu, next = dropped;
@@ -182,92 +220,97 @@ __global__ void __launch_bounds__(kThreads) route_rec_kernel(const Rows R) {
     }
     const bool ranked = R.idx_out || R.score_out;
     const bool exact = ((next ^ kth) & kCoarse) == 0u || (ranked && near_tie);
-    const bool rec = R.rec != nullptr;
-    unsigned char* rp = rec ? R.rec + p * (int64_t)(9 * KP) : nullptr;
+    unsigned char* rp = R.rec + p * (int64_t)(9 * KP);
     int32_t* io = R.idx_out ? R.idx_out + ir * K : nullptr;
     float* so = R.score_out ? R.score_out + ir * K : nullptr;
 
-    if (!exact) {
-      // ---- entries in rank order from the sorted keys
-      uint32_t sw[KP / 4];
-      float lam[KP], wv[KP];
+    if (live && !exact) {
+      // ---- entries in rank order from the sorted keys; each lane of the pair computes half
+      constexpr int KH = KP / 2;
+      uint32_t sw[KH / 4];
+      float lam[KH], wv[KH];
 #pragma unroll
-      for (int i = 0; i < KP / 4; ++i) sw[i] = 0u;
+      for (int i = 0; i < KH / 4; ++i) sw[i] = 0u;
 #pragma unroll
-      for (int r = 0; r < KP; ++r) {
-        lam[r] = 0.f;
-        wv[r] = 0.f;
+      for (int q = 0; q < KH; ++q) {
+        const int r = half * KH + q;
+        uint32_t key = 0u;
+#pragma unroll
+        for (int rr = 0; rr < N; ++rr) key = rr == r ? top[rr] : key;
+        lam[q] = 0.f;
+        wv[q] = 0.f;
         if (r < K) {
-          const int slot = 127 - (int)(top[r] & 0x7Fu);
-          sw[r / 4] |= (uint32_t)slot << (8 * (r % 4));
-          float s;
-          if (rec) {
-            entry_values(R, ir, slot, fh, s, lam[r], wv[r]);
-          } else {
-            s = sigmoid_f32(__ldg(xr + slot));
-          }
+          const int slot = 127 - (int)(key & 0x7Fu);
+          sw[q / 4] |= (uint32_t)slot << (8 * (q % 4));
+          float sc;
+          entry_values(R, ir, slot, xr[slot], fh, sc, lam[q], wv[q]);
           if (io) io[r] = slot;
-          if (so) so[r] = s;
+          if (so) so[r] = sc;
         }
       }
-      if (rec) {
 #pragma unroll
-        for (int i = 0; i < KP / 16; ++i)
-          reinterpret_cast<uint4*>(rp)[i] = make_uint4(sw[4 * i], sw[4 * i + 1], sw[4 * i + 2], sw[4 * i + 3]);
-#pragma unroll
-        for (int i = 0; i < KP / 4; ++i) {
-          reinterpret_cast<float4*>(rp + KP)[i] = make_float4(lam[4 * i], lam[4 * i + 1], lam[4 * i + 2], lam[4 * i + 3]);
-          reinterpret_cast<float4*>(rp + 5 * KP)[i] = make_float4(wv[4 * i], wv[4 * i + 1], wv[4 * i + 2], wv[4 * i + 3]);
-        }
+      for (int i = 0; i < KH / 16; ++i)
+        reinterpret_cast<uint4*>(rp + half * KH)[i] = make_uint4(sw[4 * i], sw[4 * i + 1], sw[4 * i + 2], sw[4 * i + 3]);
+      if (KH % 16 != 0) {  // KH = 8: two words of slots
+        reinterpret_cast<uint2*>(rp + half * KH)[0] = make_uint2(sw[0], sw[1]);
       }
-    } else {
-      // ---- rare: exact selection on the full keys, one rank at a time (logit desc, slot asc)
-      uint32_t chosen[4] = {0u, 0u, 0u, 0u};
-      for (int j = 0; j < KP; ++j) {
-        if (j >= K) {
-          if (rec) {
-            rp[j] = 0;
-            reinterpret_cast<float*>(rp + KP)[j] = 0.f;
-            reinterpret_cast<float*>(rp + 5 * KP)[j] = 0.f;
-          }
-          continue;
-        }
-        int best = -1;
-        uint32_t bk = 0u;
-        for (int s = 0; s < kRM; ++s) {
-          if (has_bit(chosen, s)) continue;
-          const uint32_t kx = order_key(__ldg(xr + s));
-          if (best < 0 || kx > bk) {
-            best = s;
-            bk = kx;
-          }
-        }
-        set_bit(chosen, best);
-        float s, lam = 0.f, wv = 0.f;
-        if (rec) entry_values(R, ir, best, fh, s, lam, wv);
-        else s = sigmoid_f32(__ldg(xr + best));
-        if (rec) {
-          rp[j] = (unsigned char)best;
-          reinterpret_cast<float*>(rp + KP)[j] = lam;
-          reinterpret_cast<float*>(rp + 5 * KP)[j] = wv;
-        }
-        if (io) io[j] = best;
-        if (so) so[j] = s;
+#pragma unroll
+      for (int i = 0; i < KH / 4; ++i) {
+        reinterpret_cast<float4*>(rp + KP + 4 * half * KH)[i] =
+            make_float4(lam[4 * i], lam[4 * i + 1], lam[4 * i + 2], lam[4 * i + 3]);
+        reinterpret_cast<float4*>(rp + 5 * KP + 4 * half * KH)[i] =
+            make_float4(wv[4 * i], wv[4 * i + 1], wv[4 * i + 2], wv[4 * i + 3]);
       }
     }
+    // ---- rare rows (a near-tie at the cut, or ranked output with near-ties among the first K):
+    // the whole warp ranks each of them exactly with the tournament (logit desc, slot asc)
+    uint32_t pending = __ballot_sync(kFull, live && exact && half == 0);
+    while (pending) {
+      const int src = __ffs(pending) - 1;
+      pending &= pending - 1u;
+      const int r = src >> 1;
+      const float* xw = reinterpret_cast<const float*>(wbuf + (j & 1) * kBufBytes) + r * kRowFloats;
+      float x4[kRM / 32];
+#pragma unroll
+      for (int e = 0; e < kRM / 32; ++e) x4[e] = xw[lane * (kRM / 32) + e];
+      const int64_t irw = __shfl_sync(kFull, ir, src);
+      const int64_t pw = __shfl_sync(kFull, p, src);
+      const float fhw = __shfl_sync(kFull, fh, src);
+      unsigned char* rpw = R.rec + pw * (int64_t)(9 * KP);
+      int32_t* iow = R.idx_out ? R.idx_out + irw * K : nullptr;
+      float* sow = R.score_out ? R.score_out + irw * K : nullptr;
+      warp_topk<kRM>(x4, K, lane, [&](int rk, int slot, int e) {
+        float sc, lm, wvv;
+        entry_values(R, irw, slot, x4[e], fhw, sc, lm, wvv);
+        rpw[rk] = (unsigned char)slot;
+        reinterpret_cast<float*>(rpw + KP)[rk] = lm;
+        reinterpret_cast<float*>(rpw + 5 * KP)[rk] = wvv;
+        if (iow) iow[rk] = slot;
+        if (sow) sow[rk] = sc;
+      });
+      if (lane < KP - K) {  // padding entries
+        rpw[K + lane] = 0;
+        reinterpret_cast<float*>(rpw + KP)[K + lane] = 0.f;
+        reinterpret_cast<float*>(rpw + 5 * KP)[K + lane] = 0.f;
+      }
+    }
+    __syncwarp();  // every lane is done with the buffer before it is refilled
   }
+  cp_async_wait_all();
 }
 
 template <int N, bool V>
 cudaError_t launch_n(const Rows& R, cudaStream_t stream) {
+  cudaError_t e = cudaFuncSetAttribute(route_rec_kernel<N, V>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+  if (e != cudaSuccess) return e;
   int dev = 0, sms = 148, per_sm = 1;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, route_rec_kernel<N, V>, kThreads, 0);
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, route_rec_kernel<N, V>, kThreads, kSmem);
   const int64_t rows = R.B * R.H * R.T;
-  const int64_t need = (rows + kThreads - 1) / kThreads;
-  const int64_t grid = std::min<int64_t>(need, (int64_t)sms * std::max(per_sm, 1) * 4);
-  route_rec_kernel<N, V><<<(unsigned)grid, kThreads, 0, stream>>>(R);
+  const int64_t tasks = (rows + kRowsPerTask - 1) / kRowsPerTask;
+  const int64_t grid = std::min<int64_t>((tasks + kWarps - 1) / kWarps, (int64_t)sms * std::max(per_sm, 1));
+  route_rec_kernel<N, V><<<(unsigned)grid, kThreads, kSmem, stream>>>(R);
   return cudaGetLastError();
 }
 
@@ -280,9 +323,8 @@ bool route_records_supported(int M, int K) { return M == kRM && K >= 1 && K <= 3
 cudaError_t launch_route_records(const float* logits, const float* f, const void* k, int64_t B, int64_t T,
                                  int64_t H, int M, int K, int decay_slot, int validate, unsigned char* rec,
                                  int32_t* idx_out, float* score_out, cudaStream_t stream) {
-  if (!route_records_supported(M, K)) return cudaErrorInvalidValue;
+  if (!route_records_supported(M, K) || !rec || !f || !k) return cudaErrorInvalidValue;
   if (B * T * H == 0) return cudaSuccess;
-  if (rec && (!f || !k)) return cudaErrorInvalidValue;
   Rows R;
   R.logits = logits;
   R.f = f;
