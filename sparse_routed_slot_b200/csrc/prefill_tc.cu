@@ -39,9 +39,10 @@
 //              is processed.
 //   warp 8     MMA issuer (one thread): v tile loads (two chunks ahead) and the tcgen05.mma of
 //              every chunk, as soon as their operands are ready.
+//              Once a chunk's tiles are handed over, they also convert its v tile into V^T.
 //   warps 9-12 epilogue (one per TMEM lane quarter): S -> A masking, the decay of the state after
-//              the carry (and the state in and out at item boundaries), the V^T tile of the next
-//              chunk, the output of the chunk from TMEM.
+//              the carry (and the state in and out at item boundaries), the output of the chunk
+//              from TMEM.
 // Per chunk the issuer runs S = Qh Wh^T (as soon as the row tiles are ready), then, once the
 // state is decayed and the V^T tile is there, O^T = H^T Qh^T and the carry H^T += V^T Wh, and
 // finally O^T += V^T A^T when the epilogue has masked S into A. An exact-path chunk carries into
@@ -282,7 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
   // mbarriers (phase k of a barrier = its k-th completion; every role counts the same way)
   __shared__ __align__(8) uint64_t bar_rdy,  // row tiles of chunk n written         (row threads)
       bar_tma[2],                             // raw v tile of chunk n landed          (TMA, buffer n&1)
-      bar_vt,                                 // V^T of chunk n written                (epilogue)
+      bar_vt,                                 // V^T of chunk n written                (row threads)
       bar_s,                                  // main pass: S of chunk n done          (MMA commit)
       bar_a,                                  // main pass: A of chunk n written       (epilogue)
       bar_t,                                  // read and carry of chunk n done        (MMA commit)
@@ -304,7 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     tc::mbar_init(&bar_rdy, kRThreads);
     tc::mbar_init(&bar_tma[0], 1);
     tc::mbar_init(&bar_tma[1], 1);
-    tc::mbar_init(&bar_vt, kEpiThreads);
+    tc::mbar_init(&bar_vt, kRThreads);
     tc::mbar_init(&bar_s, 1);
     tc::mbar_init(&bar_a, kEpiThreads);
     tc::mbar_init(&bar_t, 1);
@@ -507,6 +508,23 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         tc::fence_async_smem();
         mbar_arrive(&bar_rdy);
       }
+      // ---- V^T of this chunk: its v tile has landed and the chunk before has finished A.V
+      if (n > 0) wait_or_abort(&bar_o, (n - 1) & 1, abort_flag);
+      wait_or_abort(&bar_tma[n & 1], (n >> 1) & 1, abort_flag);
+      {
+        const uint16_t* raw = reinterpret_cast<const uint16_t*>(sRawV + (n & 1) * (kC * kDV * 2));
+        const int dv = tid & (kDV - 1), s_beg = (tid >> 7) * (kC / 2);
+#pragma unroll 4
+        for (int s4 = s_beg; s4 < s_beg + kC / 2; s4 += 4) {
+          const float4 f4 = make_float4(__uint_as_float((uint32_t)raw[(s4 + 0) * kDV + dv] << 16),
+                                        __uint_as_float((uint32_t)raw[(s4 + 1) * kDV + dv] << 16),
+                                        __uint_as_float((uint32_t)raw[(s4 + 2) * kDV + dv] << 16),
+                                        __uint_as_float((uint32_t)raw[(s4 + 3) * kDV + dv] << 16));
+          *reinterpret_cast<float4*>(sVt + tc::swz_offset(kDV, dv, s4)) = f4;
+        }
+        tc::fence_async_smem();
+        mbar_arrive(&bar_vt);
+      }
       cur = nxt;
     }
   } else if (warp == kIssuerWarp) {
@@ -626,26 +644,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       }
       tc::tmem_wait_st();
     };
-    // V^T tile of chunk j (thread = value column; conflict-free 16-byte stores)
-    auto make_vt = [&](uint32_t j) {
-      wait_or_abort(&bar_tma[j & 1], (j >> 1) & 1, abort_flag);
-      const uint16_t* raw = reinterpret_cast<const uint16_t*>(sRawV + (j & 1) * (kC * kDV * 2));
-#pragma unroll 4
-      for (int s4 = 0; s4 < kC; s4 += 4) {
-        const float4 f4 = make_float4(__uint_as_float((uint32_t)raw[(s4 + 0) * kDV + dv] << 16),
-                                      __uint_as_float((uint32_t)raw[(s4 + 1) * kDV + dv] << 16),
-                                      __uint_as_float((uint32_t)raw[(s4 + 2) * kDV + dv] << 16),
-                                      __uint_as_float((uint32_t)raw[(s4 + 3) * kDV + dv] << 16));
-        *reinterpret_cast<float4*>(sVt + tc::swz_offset(kDV, dv, s4)) = f4;
-      }
-      tc::fence_async_smem();
-      mbar_arrive(&bar_vt);
-    };
     if (wk.valid()) {
       load_state(wk.get());
       tc::tmem_fence_before();
       mbar_arrive(&bar_h);  // phase 0: the first chunk's state
-      make_vt(0);
     }
     uint32_t n = 0;
     for (; wk.valid() && !*abort_flag; ++n, wk.next()) {
@@ -694,59 +696,63 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         else if (ck.seg == p.nseg - 1 && p.HT) dst = p.HT + (int64_t)ck.pair * kM * kDV;
       }
 #pragma unroll 1
-      for (int c = 0; c < kM; c += 32) {
-        float hv[32];
-        tc::tmem_ld32(tc::tmem_addr(tb, sub_lane, kColH + c), hv);
-        if (!fast) {
-          float uv[32];
-          tc::tmem_ld32(tc::tmem_addr(tb, sub_lane, kColU + c), uv);
-          tc::tmem_wait_ld();
+      for (int c = 0; c < kM; c += 64) {
+        float hv[2][32];
+        tc::tmem_ld32(tc::tmem_addr(tb, sub_lane, kColH + c), hv[0]);
+        tc::tmem_ld32(tc::tmem_addr(tb, sub_lane, kColH + c + 32), hv[1]);
+        tc::tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 32; j += 4) {
-            const float4 d4 = *reinterpret_cast<const float4*>(Dn + c + j);
-            hv[j] = fmaf(d4.x, hv[j], uv[j]);
-            hv[j + 1] = fmaf(d4.y, hv[j + 1], uv[j + 1]);
-            hv[j + 2] = fmaf(d4.z, hv[j + 2], uv[j + 2]);
-            hv[j + 3] = fmaf(d4.w, hv[j + 3], uv[j + 3]);
+        for (int g = 0; g < 2; ++g) {
+          const int cg = c + 32 * g;
+          if (!fast) {
+            float uv[32];
+            tc::tmem_ld32(tc::tmem_addr(tb, sub_lane, kColU + cg), uv);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+              const float4 d4 = *reinterpret_cast<const float4*>(Dn + cg + j);
+              hv[g][j] = fmaf(d4.x, hv[g][j], uv[j]);
+              hv[g][j + 1] = fmaf(d4.y, hv[g][j + 1], uv[j + 1]);
+              hv[g][j + 2] = fmaf(d4.z, hv[g][j + 2], uv[j + 2]);
+              hv[g][j + 3] = fmaf(d4.w, hv[g][j + 3], uv[j + 3]);
+            }
+          } else {
+            scale_by(hv[g], Dn + cg);  // slots not selected in the chunk: D = 1 exactly
           }
-        } else {
-          tc::tmem_wait_ld();
-          scale_by(hv, Dn + c);  // slots not selected in the chunk: D = 1 exactly
-        }
-        if (ck.last) {
-          if (dst) {
+          if (ck.last) {
+            if (dst) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) dst[(c + j) * kDV + dv] = hv[j];
+              for (int j = 0; j < 32; ++j) dst[(cg + j) * kDV + dv] = hv[g][j];
+            }
+          } else {
+            tc::tmem_st32(tc::tmem_addr(tb, sub_lane, kColH + cg), hv[g]);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) hv[g][j] = tc::to_tf32(hv[g][j]);
+            tc::tmem_st32(tc::tmem_addr(tb, sub_lane, kColHr + cg), hv[g]);
           }
-        } else {
-          tc::tmem_st32(tc::tmem_addr(tb, sub_lane, kColH + c), hv);
-#pragma unroll
-          for (int j = 0; j < 32; ++j) hv[j] = tc::to_tf32(hv[j]);
-          tc::tmem_st32(tc::tmem_addr(tb, sub_lane, kColHr + c), hv);
         }
       }
       tc::tmem_wait_st();
       if (ck.last && nx.valid()) load_state(nx.get());
       tc::tmem_fence_before();
       mbar_arrive(&bar_h);  // phase n+1: the state of the next chunk
-      // ---- every MMA of this chunk is done: the next V^T, then this chunk's output
-      wait_or_abort(&bar_o, n & 1, abort_flag);
-      tc::tmem_fence_after();
-      if (nx.valid()) make_vt(n + 1);
+      // ---- every MMA of this chunk is done: its output
       if (!SUMMARY) {
+        wait_or_abort(&bar_o, n & 1, abort_flag);
+        tc::tmem_fence_after();
         float* orow = p.o + (((int64_t)ck.b * T + ck.c0) * H + ck.h) * kDV + dv;
         const int64_t ostride = (int64_t)H * kDV;
-#pragma unroll 1
-        for (int c = 0; c < kC; c += 32) {
-          float ov[32];
-          tc::tmem_ld32(tc::tmem_addr(tb, sub_lane, kColO + (n & 1) * kC + c), ov);
-          tc::tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (c + j < ck.nrows) orow[(int64_t)(c + j) * ostride] = ov[j];
-        }
+        float ov[2][32];
+        tc::tmem_ld32(tc::tmem_addr(tb, sub_lane, kColO + (n & 1) * kC), ov[0]);
+        tc::tmem_ld32(tc::tmem_addr(tb, sub_lane, kColO + (n & 1) * kC + 32), ov[1]);
+        tc::tmem_wait_ld();
+        // the O buffer is free once read; signal before the stores (an arrive after them would
+        // wait for the stores to complete)
         tc::tmem_fence_before();
         mbar_arrive(&bar_of[n & 1]);
+#pragma unroll
+        for (int j = 0; j < kC; ++j)
+          if (j < ck.nrows) orow[(int64_t)j * ostride] = ov[j >> 5][j & 31];
       }
     }
   }
