@@ -18,9 +18,7 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
-import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -68,51 +66,59 @@ def decode_bytes(B, H, M, K, Dv, es=2, per_slot=False) -> tuple[int, int]:
 
 # --------------------------------------------------------------------------- clocks
 
-CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
-
-
 class ClockSampler:
-    """Samples nvidia-smi every 200 ms in the background while the timed region runs."""
+    """Samples the SM clock and the throttle reasons every 10 ms (NVML, in a background thread;
+    nvidia-smi at 200 ms if NVML is missing) while the timed region runs."""
+
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4}
 
     def __init__(self, gpu_index: int):
-        self.path = tempfile.mktemp(prefix="clocks_", suffix=".csv")
-        self.proc = None
+        import threading
+        self.sm, self.smax, self.seen, self.err = [], None, set(), None
+        self._stop = threading.Event()
         try:
-            self.fh = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={CLOCK_FIELDS}", "--format=csv,noheader,nounits",
-                 "-i", str(gpu_index), "-lms", "200"], stdout=self.fh, stderr=subprocess.DEVNULL)
-        except Exception:
-            self.proc = None
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(self._phys_index(gpu_index))
+            self.smax = float(pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM))
+        except Exception as e:  # noqa: BLE001
+            self._nv, self.err = None, f"nvml unavailable: {e}"
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+
+    @staticmethod
+    def _phys_index(i: int) -> int:
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        if vis:
+            try:
+                return int(vis.split(",")[i])
+            except (ValueError, IndexError):
+                return i
+        return i
+
+    def _run(self):
+        while not self._stop.is_set():
+            if self._nv is not None:
+                try:
+                    self.sm.append(float(self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM)))
+                    r = self._nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                    for n, bit in self.REASONS.items():
+                        if r & bit:
+                            self.seen.add(n)
+                except Exception as e:  # noqa: BLE001
+                    self.err = str(e)
+            self._stop.wait(0.01)
 
     def stop(self) -> dict:
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        self.fh.close()
-        sm, smax, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in open(self.path):
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                smax = float(parts[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        os.unlink(self.path)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
-                "samples": len(sm), "reasons": sorted(reasons)}
+        self._stop.set()
+        self._t.join(timeout=2)
+        out = {"sm_mhz": statistics.median(self.sm) if self.sm else None, "sm_max_mhz": self.smax,
+               "samples": len(self.sm), "reasons": sorted(self.seen)}
+        if self.err:
+            out["note"] = self.err
+        return out
 
 
 # --------------------------------------------------------------------------- distributed
@@ -150,39 +156,73 @@ def max_over_ranks(x: float, world: int) -> float:
 
 # --------------------------------------------------------------------------- CPU oracle timing
 
-def oracle_sample(w, seconds_target: float = 12.0) -> dict:
-    """Times the fp64 CPU oracle (as it stands) on a bounded sample of the workload: all heads
-    of sequence 0 over a prefix of the tokens, sized to about `seconds_target` of CPU time."""
-    import numpy as np
-    import torch
+def oracle_sample(w, seconds_target: float = 3.0) -> dict:
+    """Times the fp64 CPU oracle (as it stands) on a bounded sample of the workload: all heads of
+    sequence 0, over a prefix of the tokens or, when the whole sequence is quick, repeated runs of
+    it, for about `seconds_target` seconds of wall time on all host cores."""
     from oracle import oracle
     from sparse_routed_slot_b200.workloads import make_inputs
 
     cores = oracle.default_threads()
 
-    def run(T):
+    def inputs(T):
         x = make_inputs(1, T, w.H, w.M, w.Dv, w.torch_dtype, w.decay, seed=w.seed)
-        c = {n: t.float().numpy() for n, t in x.items()}
+        return {n: t.float().numpy() for n, t in x.items()}
+
+    def run(c, reps=1):
         t0 = time.perf_counter()
-        oracle.forward(c["q"], c["k"], c["v"], c["logits"], c["f"], w.K, want_idx=False, nthreads=cores)
+        for _ in range(reps):
+            oracle.forward(c["q"], c["k"], c["v"], c["logits"], c["f"], w.K, want_idx=False, nthreads=cores)
         return time.perf_counter() - t0
 
     T0 = min(w.T, 256)
-    dt = run(T0)
-    T1 = int(min(w.T, max(T0, T0 * seconds_target / max(dt, 1e-6))))
-    dt1 = run(T1) if T1 != T0 else dt
+    dt0 = run(inputs(T0))
+    T1 = int(min(w.T, max(T0, T0 * seconds_target / max(dt0, 1e-6))))
+    c1 = inputs(T1)
+    dt1 = run(c1)
+    reps = max(1, int(seconds_target / max(dt1, 1e-6))) if T1 == w.T else 1
+    if reps > 1:
+        dt1 = run(c1, reps)
     used = min(cores, w.H)
-    return {"value": T1 / dt1, "unit": "tokens/s", "cores": used, "kind": "oracle",
-            "sample": f"sequence 0, all {w.H} heads, first {T1} of {w.T} tokens, fp64, "
-                      f"{used} threads over heads; {dt1:.1f} s", "seconds": dt1, "tokens": T1}
+    return {"value": reps * T1 / dt1, "unit": "tokens/s", "cores": used, "kind": "oracle",
+            "sample": f"sequence 0, all {w.H} heads, first {T1} of {w.T} tokens x {reps} run(s), fp64, "
+                      f"{used} threads over heads; {dt1:.1f} s", "seconds": dt1, "tokens": T1 * reps}
+
+
+def _sources_digest() -> str:
+    """sha256 of the CUDA sources (used to tell whether stored ncu counters are still current)."""
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "sparse_routed_slot_b200", "csrc", "*"))):
+        h.update(open(f, "rb").read())
+    return h.hexdigest()
+
+
+def stored_traffic(key: str):
+    """DRAM bytes per call measured by ncu for `key` (profiles/traffic.json), or None when the file
+    is missing or was recorded for other kernel sources."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        d = json.load(open(p))
+    except (OSError, ValueError):
+        return None
+    if d.get("sources_sha256") != _sources_digest():
+        return None
+    return d.get("bytes", {}).get(key)
 
 
 # --------------------------------------------------------------------------- our arm
 
+KERNEL_NAMES = {4: ["route records", "segment summary", "segment scan", "chunk scan"],
+                2: ["route records", "chunk scan"], 1: ["chunk scan (CUDA cores)"]}
+
+
 def run_ours(args, world, rank, local):
+    import ctypes
     import torch
     import sparse_routed_slot_b200 as rsm
-    from sparse_routed_slot_b200 import api
+    from sparse_routed_slot_b200 import _lib, api
     from sparse_routed_slot_b200.workloads import WORKLOADS, make_inputs
 
     w = WORKLOADS[args.workload]
@@ -196,7 +236,9 @@ def run_ours(args, world, rank, local):
                           args.path, False)
     ws_bytes = api.workspace_bytes(a)
     path_used = api.selected_path(a)
+    launches = api.kernel_launches(a)
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+    L = _lib.load()
 
     def step():
         rsm.forward(x["q"], x["k"], x["v"], x["logits"], x["f"], w.K, out=outs, workspace=ws,
@@ -206,21 +248,32 @@ def run_ours(args, world, rank, local):
         step()
     torch.cuda.synchronize()
     barrier(world)
-    clocks = ClockSampler(local)
     stream = torch.cuda.current_stream(dev)
+    # per-kernel events inside every timed call (recorded by the library on this stream)
+    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(launches + 1)] for _ in range(args.steps)]
+    for row in kev:  # torch creates the CUDA event on its first record
+        for e in row:
+            e.record(stream)
+    torch.cuda.synchronize()
+    kev_ptrs = [(ctypes.c_void_p * (launches + 1))(*[e.cuda_event for e in row]) for row in kev]
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    clocks = ClockSampler(local)
     torch.cuda.synchronize()
     barrier(world)
     ev[0].record(stream)
     for i in range(args.steps):
+        _lib.check(L.rsm_forward_set_profile_events(kev_ptrs[i], launches + 1))
         step()
         ev[i + 1].record(stream)
     torch.cuda.synchronize()
+    _lib.check(L.rsm_forward_set_profile_events(None, 0))
     barrier(world)
     clk = clocks.stop()
     per = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
     ms = sum(per) / len(per)
     ms_max = max_over_ranks(ms, world)
+    kms = [sum(row[j].elapsed_time(row[j + 1]) for row in kev) / args.steps for j in range(launches)]
+    names = KERNEL_NAMES.get(launches, [f"kernel {j}" for j in range(launches)])
     tokens = w.B * w.T
     value = tokens * world / (ms_max * 1e-3)
 
@@ -264,24 +317,25 @@ def run_ours(args, world, rank, local):
                    "path": path_used, "parallelism": f"replicas{world}",
                    "l2": f"inputs larger than L2 ({nbytes / 1e6:.0f} MB per step, no flush)"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": achieved / peaks["hbm_gbs"], "traffic": None,
-                     "algorithmic_bytes": nbytes, "kernel": "rsm prefill (single launch per step)",
-                     "peak_source": peaks["source"],
+                     "frac": achieved / peaks["hbm_gbs"],
+                     "traffic": stored_traffic(f"{w.name}/forward"),
+                     "algorithmic_bytes": nbytes,
+                     "kernel": f"rsm_forward, all {launches} launches of the step (" + ", ".join(names) + ")",
+                     "peak_source": peaks["source"] + " (burst copy)",
                      "tensor_tflops": prefill_flops(w) / (ms * 1e-3) / 1e12},
+        "kernels": [{"name": n, "ms": t, "share": t / sum(kms) if sum(kms) > 0 else None}
+                    for n, t in zip(names, kms)],
         "e2e": {"value": tokens * world / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": args.steps * launches_per_forward(path_used),
+        "gpu_launches": args.steps * launches,
         "clocks": clk,
     }
     if not args.no_decode:
         line["decode"] = run_decode(args, world, rank, local, peaks)
+        line["gpu_launches"] += line["decode"]["steps_timed"]
     if rank == 0 and not args.no_cpu:
         line["cpu_baseline"] = oracle_sample(w)
     return line
-
-
-def launches_per_forward(path):
-    return 1
 
 
 def run_decode(args, world, rank, local, peaks) -> dict:
@@ -314,12 +368,14 @@ def run_decode(args, world, rank, local, peaks) -> dict:
     torch.cuda.synchronize()
     barrier(world)
     stream = torch.cuda.current_stream(dev)
+    clocks = ClockSampler(local)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for i in range(nsteps):
         step(i)
     e1.record(stream)
     torch.cuda.synchronize()
+    clk = clocks.stop()
     ms = max_over_ranks(e0.elapsed_time(e1) / nsteps, world)
     sb, tb = decode_bytes(w.B, w.H, w.M, w.K, w.Dv, 2, w.decay == "slot")
     state_gbs = sb / (ms * 1e-3) / 1e9
@@ -327,8 +383,10 @@ def run_decode(args, world, rank, local, peaks) -> dict:
     return {"value": state_gbs * world, "unit": "GB/s (state, all GPUs)", "ms_per_step": ms,
             "steps_timed": nsteps, "total_gbs": total_gbs * world,
             "roofline": {"bound": "hbm", "achieved": total_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": total_gbs / peaks["hbm_gbs"], "traffic": None,
-                         "algorithmic_bytes": tb, "kernel": "rsm decode step"},
+                         "frac": total_gbs / peaks["hbm_gbs"],
+                         "traffic": stored_traffic("decode_256x16/step"),
+                         "algorithmic_bytes": tb, "kernel": "rsm decode step (one launch)"},
+            "clocks": clk, "traffic_note": "single launch per step",
             "config": {"workload": w.name, "B": w.B, "H": w.H, "M": w.M, "K": w.K, "Dv": w.Dv,
                        "prefill_T": w.decode_prefill_T, "graph": False,
                        "l2": f"state {w.B * w.H * w.M * w.Dv * 4 / 1e6:.0f} MB > L2"}}
@@ -364,7 +422,7 @@ def run_reference(args, world, rank) -> dict | None:
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="long_ctx_bf16")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])

@@ -134,6 +134,15 @@ RSM_API int rsm_forward_selected_path(const rsm_forward_args* args);
  * path = 1; 0 when B*H == 0 or T == 0), or -1 for arguments rsm_forward rejects. Host-only. */
 RSM_API int rsm_forward_kernel_launches(const rsm_forward_args* args);
 
+/* Profiling aid (no counterpart on the pages): while set, every rsm_forward call made on the
+ * calling host thread records `events[0]` on its stream before its first kernel and `events[i]`
+ * after its i-th kernel (i = 1 .. rsm_forward_kernel_launches(args)), so that the caller can time
+ * each kernel with cudaEventElapsedTime. `events` are cudaEvent_t handles passed as void*, owned
+ * by the caller; `n_events` must be at least the launches of the calls that follow plus one (a
+ * call that needs more returns RSM_ERR_INVALID_ARG before any launch). NULL / 0 stops recording.
+ * The events are only recorded, never waited on or destroyed, by the library. Host-only. */
+RSM_API rsm_status rsm_forward_set_profile_events(void* const* events, int n_events);
+
 /* ---------------------------------------------------------------------------------------------
  * rsm_forward_noalloc -- rsm_forward for callers that cannot allocate device memory.
  *   The pages have no counterpart to this call; it exists for callers with no way to allocate:

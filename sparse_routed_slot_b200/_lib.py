@@ -20,7 +20,7 @@ RSM_FLAG_VALIDATE = 1
 
 # Every symbol include/rsm.h declares (the CPU tests check the library exports all of them).
 EXPORTED = ("rsm_route", "rsm_forward_workspace_size", "rsm_forward", "rsm_forward_selected_path",
-            "rsm_forward_kernel_launches",
+            "rsm_forward_kernel_launches", "rsm_forward_set_profile_events",
             "rsm_decode_step",
             "rsm_status_string", "rsm_last_error", "rsm_get_device_status", "rsm_version",
             "rsm_forward_noalloc", "rsm_forward_noalloc_max_scratch")
@@ -71,6 +71,8 @@ def load() -> ctypes.CDLL:
         lib.rsm_forward_selected_path.restype = _int
         lib.rsm_forward_kernel_launches.argtypes = [ctypes.POINTER(ForwardArgs)]
         lib.rsm_forward_kernel_launches.restype = _int
+        lib.rsm_forward_set_profile_events.argtypes = [ctypes.POINTER(_vp), _int]
+        lib.rsm_forward_set_profile_events.restype = _int
         lib.rsm_forward_noalloc.argtypes = [ctypes.POINTER(ForwardArgs), _vp]
         lib.rsm_forward_noalloc.restype = _int
         lib.rsm_forward_noalloc_max_scratch.argtypes = []

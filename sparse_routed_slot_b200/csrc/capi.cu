@@ -94,6 +94,15 @@ bool use_tensor_path(const rsm_forward_args& a) {
 }  // namespace
 
 namespace rsm {
+ProfileEvents& profile_events() {
+  static thread_local ProfileEvents pe;
+  return pe;
+}
+cudaError_t profile_mark(cudaStream_t stream) {
+  ProfileEvents& pe = profile_events();
+  if (!pe.events || pe.next >= pe.n) return cudaSuccess;
+  return cudaEventRecord(static_cast<cudaEvent_t>(pe.events[pe.next++]), stream);
+}
 // Records a failure message for rsm_last_error() from other translation units of the library.
 rsm_status report_error(rsm_status s, const char* msg) { return fail(s, "%s", msg); }
 }  // namespace rsm
@@ -173,9 +182,28 @@ rsm_status rsm_forward(const rsm_forward_args* a, void* stream) {
     }
     return RSM_OK;
   }
-  cudaError_t e = tc ? rsm::launch_prefill_tc(*a, static_cast<cudaStream_t>(stream))
-                     : rsm::launch_prefill_simt(*a, static_cast<cudaStream_t>(stream));
+  rsm::ProfileEvents& pe = rsm::profile_events();
+  if (pe.events) {
+    const int need = (tc ? rsm::prefill_tc_launches(*a) : 1) + 1;
+    if (pe.n < need) return fail(RSM_ERR_INVALID_ARG, "%d profiling events needed (set: %d)", need, pe.n);
+    pe.next = 0;
+  }
+  cudaError_t e = rsm::profile_mark(static_cast<cudaStream_t>(stream));
+  if (e == cudaSuccess)
+    e = tc ? rsm::launch_prefill_tc(*a, static_cast<cudaStream_t>(stream))
+           : rsm::launch_prefill_simt(*a, static_cast<cudaStream_t>(stream));
+  if (e == cudaSuccess && !tc) e = rsm::profile_mark(static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? RSM_OK : cuda_fail(e, tc ? "rsm_forward (tensor path)" : "rsm_forward (simt path)");
+}
+
+rsm_status rsm_forward_set_profile_events(void* const* events, int n_events) {
+  g_err[0] = 0;
+  if (events && n_events < 1) return fail(RSM_ERR_INVALID_ARG, "n_events must be >= 1");
+  rsm::ProfileEvents& pe = rsm::profile_events();
+  pe.events = n_events > 0 ? events : nullptr;
+  pe.n = pe.events ? n_events : 0;
+  pe.next = 0;
+  return RSM_OK;
 }
 
 rsm_status rsm_decode_step(const rsm_decode_args* a, void* stream) {

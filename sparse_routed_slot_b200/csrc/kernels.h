@@ -32,6 +32,17 @@ size_t prefill_tc_workspace_bytes(const rsm_forward_args& a);
 int prefill_tc_launches(const rsm_forward_args& a);  // kernel launches of one call
 cudaError_t launch_prefill_tc(const rsm_forward_args& a, cudaStream_t stream);
 
+// Profiling events of the calling host thread (rsm_forward_set_profile_events): when set, launch
+// functions record event i after their i-th kernel (event 0 before the first).
+struct ProfileEvents {
+  void* const* events = nullptr;
+  int n = 0;
+  int next = 0;
+};
+ProfileEvents& profile_events();
+// Records the next profiling event on `stream` (no-op when none are set).
+cudaError_t profile_mark(cudaStream_t stream);
+
 // Sets the message rsm_last_error() returns on this host thread; returns `s`.
 rsm_status report_error(rsm_status s, const char* msg);
 

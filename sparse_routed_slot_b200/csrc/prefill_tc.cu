@@ -876,15 +876,19 @@ cudaError_t launch_passes(const Maps& maps, const Params& p, const Plan& pl, int
     const int items = (int)(pairs * (pl.nseg - 1));
     prefill_tc_kernel<true, KP><<<std::min(items, sms), kThreads, kSmemBytes, stream>>>(maps, p);
     e = cudaGetLastError();
+    if (e == cudaSuccess) e = profile_mark(stream);
     if (e != cudaSuccess) return e;
     dim3 g((kM * kDV + 255) / 256, (unsigned)pairs);
     segment_scan_kernel<<<g, 256, 0, stream>>>(p);
     e = cudaGetLastError();
+    if (e == cudaSuccess) e = profile_mark(stream);
     if (e != cudaSuccess) return e;
   }
   const int64_t items = pairs * pl.nseg;
   prefill_tc_kernel<false, KP><<<(unsigned)std::min<int64_t>(items, sms), kThreads, kSmemBytes, stream>>>(maps, p);
-  return cudaGetLastError();
+  e = cudaGetLastError();
+  if (e == cudaSuccess) e = profile_mark(stream);
+  return e;
 }
 
 }  // namespace
@@ -911,6 +915,7 @@ cudaError_t launch_prefill_tc(const rsm_forward_args& a, cudaStream_t stream) {
   unsigned char* rec = reinterpret_cast<unsigned char*>(ws + wl.rec);
   cudaError_t e = launch_route_records(a.logits, a.f, a.k, a.B, a.T, a.H, a.M, a.K, a.decay == RSM_DECAY_SLOT,
                                        (a.flags & RSM_FLAG_VALIDATE) != 0, rec, a.idx_out, a.score_out, stream);
+  if (e == cudaSuccess) e = profile_mark(stream);
   if (e != cudaSuccess) return e;
   Maps maps;
   if (!make_map(&maps.v, a.v, a.B, a.T, a.H, kDV)) return cudaErrorInvalidValue;
