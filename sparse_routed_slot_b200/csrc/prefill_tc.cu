@@ -42,7 +42,8 @@
 //              Once a chunk's tiles are handed over, they also convert its v tile into V^T.
 //   warps 9-12 epilogue (one per TMEM lane quarter): S -> A masking, the decay of the state after
 //              the carry (and the state in and out at item boundaries), the output of the chunk
-//              from TMEM.
+//              from TMEM, staged in halves through the A tile's memory and written by bulk tensor
+//              stores.
 // Per chunk the issuer runs S = Qh Wh^T (as soon as the row tiles are ready), then, once the
 // state is decayed and the V^T tile is there, O^T = H^T Qh^T and the carry H^T += V^T Wh, and
 // finally O^T += V^T A^T when the epilogue has masked S into A. An exact-path chunk carries into
@@ -75,6 +76,7 @@ constexpr int kRowsPerWarp = kC / kRWarps;
 constexpr int kRThreads = kRWarps * 32;
 constexpr int kIssuerWarp = kRWarps;          // warp 8
 constexpr int kEpiThreads = 4 * 32;
+constexpr int kEpiThread0 = (kRWarps + 1) * 32;  // issues the output tile stores
 constexpr int kThreads = (kRWarps + 1 + 4) * 32;
 constexpr float kDMin = 1.80485139e-35f;  // e^-80: fast-path bound on the in-chunk decay
 
@@ -98,7 +100,8 @@ constexpr int kSmemBytes = kOffSmall + kSmallBytes + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 struct Maps {
-  CUtensorMap v;
+  CUtensorMap v;  // v [B,T,H,Dv] bf16, box: one (b,h), 64 tokens
+  CUtensorMap o;  // o [B,T,H,Dv] fp32, box: one (b,h), 32 tokens (output stores)
 };
 
 struct Params {
@@ -156,6 +159,7 @@ RSM_DEV bool bar_rows_or(bool flag) {
   return r != 0;
 }
 RSM_DEV void bar_rows() { asm volatile("bar.sync 1, %0;" ::"n"(kRThreads) : "memory"); }
+RSM_DEV void bar_epi() { asm volatile("bar.sync 2, %0;" ::"n"(kEpiThreads) : "memory"); }
 
 // Position of one chunk in the CTA's work list.
 struct Chunk {
@@ -164,26 +168,28 @@ struct Chunk {
 };
 
 // The CTA walks its items (item = blockIdx.x + j*gridDim.x) and each item's chunks in order.
-// The item's coordinates are computed once per item (integer division is not cheap here).
+// The item's coordinates are computed once per item (integer division is not cheap here); the
+// sizes come from the kernel parameters, so a walker is only a few registers.
 struct Walker {
-  int items, pairs, H, T, seg_chunks, item, c0, t0, t1, pair, seg, b, h;
-  __device__ void start(int items_, int pairs_, int H_, int T_, int seg_chunks_) {
-    items = items_; pairs = pairs_; H = H_; T = T_; seg_chunks = seg_chunks_;
+  int item, c0, t1, pair, seg, b, h;
+  bool first;
+  __device__ void start(const Params& p, int items) {
     item = blockIdx.x;
-    set_item();
+    set_item(p, items);
   }
-  __device__ void set_item() {
+  __device__ void set_item(const Params& p, int items) {
     if (item >= items) return;
+    const int pairs = p.B * p.H;
     seg = item / pairs;
     pair = item - seg * pairs;
-    b = pair / H;
-    h = pair - b * H;
-    t0 = seg * seg_chunks * kC;
-    t1 = min(T, t0 + seg_chunks * kC);
-    c0 = t0;
+    b = pair / p.H;
+    h = pair - b * p.H;
+    c0 = seg * p.seg_chunks * kC;
+    t1 = min(p.T, c0 + p.seg_chunks * kC);
+    first = true;
   }
-  __device__ bool valid() const { return item < items; }
-  __device__ Chunk get() const {
+  __device__ bool valid(int items) const { return item < items; }
+  __device__ Chunk get(const Params& p) const {
     Chunk c;
     c.pair = pair;
     c.seg = seg;
@@ -191,15 +197,16 @@ struct Walker {
     c.h = h;
     c.c0 = c0;
     c.nrows = min(kC, t1 - c0);
-    c.first = c0 == t0;
+    c.first = first;
     c.last = c0 + kC >= t1;
     return c;
   }
-  __device__ void next() {
+  __device__ void next(const Params& p, int items) {
     c0 += kC;
+    first = false;
     if (c0 >= t1) {
       item += gridDim.x;
-      set_item();
+      set_item(p, items);
     }
   }
 };
@@ -325,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
   volatile int* abort_flag = &s_abort;
 
   Walker wk;
-  wk.start(items, pairs, H, T, p.seg_chunks);
+  wk.start(p, items);
 
   if (warp < kRWarps) {
     // =========================================================================== row workers
@@ -335,17 +342,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     float Dseg[4] = {1.f, 1.f, 1.f, 1.f};       // summary pass, warp 0: product of the chunk decays
 
     RowInputs<KP> cur;
-    if (wk.valid()) load_rows<SUMMARY, KP>(p, wk.get(), w, lane, cur);
-    for (uint32_t n = 0; wk.valid(); ++n, wk.next()) {
-      const Chunk ck = wk.get();
+    if (wk.valid(items)) load_rows<SUMMARY, KP>(p, wk.get(p), w, lane, cur);
+    for (uint32_t n = 0; wk.valid(items); ++n, wk.next(p, items)) {
+      const Chunk ck = wk.get(p);
       const int buf = n & 1;
       const int nrows_w = ck.nrows - w * kRowsPerWarp;  // rows of this warp inside the chunk
-      RowInputs<KP> nxt;
-      {
-        Walker nx = wk;
-        nx.next();
-        if (nx.valid()) load_rows<SUMMARY, KP>(p, nx.get(), w, lane, nxt);
-      }
       // ---- this warp's rows of the decay table: 1 everywhere, -a at the selected entries
 #pragma unroll
       for (int i = 0; i < kRowsPerWarp; ++i)
@@ -439,7 +440,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         // ---- exact path (rare): log-domain table and dense g (in the Wh region), the Qh tile,
         // the end-referenced Wh^T and A from pairwise sums, exponents <= 0. The issuer runs the
         // read, the carry into U and A.V; the epilogue then forms H = D H + U.
-        if (n > 0) wait_or_abort(&bar_o, (n - 1) & 1, abort_flag);  // A.V of the chunk before is done with A
+        // A.V of the chunk before is done with A, and the epilogue has staged that chunk's output
+        // through the A tile's memory
+        if (!SUMMARY && n > 0) wait_or_abort(&bar_of[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag);
         bar_rows();  // every row worker is past the product totals
 #pragma unroll
         for (int i = 0; i < kRowsPerWarp; ++i)
@@ -508,6 +511,14 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         tc::fence_async_smem();
         mbar_arrive(&bar_rdy);
       }
+      // ---- the next chunk's q and records start loading (they land during the V^T conversion
+      // and the next chunk's table)
+      RowInputs<KP> nxt;
+      {
+        Walker nx = wk;
+        nx.next(p, items);
+        if (nx.valid(items)) load_rows<SUMMARY, KP>(p, nx.get(p), w, lane, nxt);
+      }
       // ---- V^T of this chunk: its v tile has landed and the chunk before has finished A.V
       if (n > 0) wait_or_abort(&bar_o, (n - 1) & 1, abort_flag);
       wait_or_abort(&bar_tma[n & 1], (n >> 1) & 1, abort_flag);
@@ -532,8 +543,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     if (lane == 0) {
       uint32_t n = 0, n_tma = 0;
       auto load_v = [&](const Walker& at, uint32_t j) {  // v tile of the walker's chunk, as chunk j
-        if (!at.valid()) return;
-        const Chunk c = at.get();
+        if (!at.valid(items)) return;
+        const Chunk c = at.get(p);
         tc::mbar_arrive_expect_tx(&bar_tma[j & 1], kC * kDV * 2);
         tc::tma_load_4d(sRawV + (j & 1) * (kC * kDV * 2), &maps.v, &bar_tma[j & 1], 0, c.h, c.c0, c.b);
         ++n_tma;
@@ -541,7 +552,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       {
         Walker nx = wk;
         load_v(nx, 0);
-        nx.next();
+        nx.next(p, items);
         load_v(nx, 1);
       }
       const uint32_t q = tc::smem_u32(sQ), wsm = tc::smem_u32(sW), wt = tc::smem_u32(sWt),
@@ -572,7 +583,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         }
       };
       bool prev_exact = false;
-      for (; wk.valid() && !*abort_flag; ++n, wk.next()) {
+      for (; wk.valid(items) && !*abort_flag; ++n, wk.next(p, items)) {
         const uint32_t ob = (n & 1) * kC;  // O buffer of this chunk
         wait_or_abort(&bar_rdy, n & 1, abort_flag);
         const bool fast = sFast[n & 1] != 0;
@@ -599,8 +610,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         {
           // the raw v buffer of this chunk is free again: load the chunk two ahead into it
           Walker nx = wk;
-          nx.next();
-          nx.next();
+          nx.next(p, items);
+          nx.next(p, items);
           load_v(nx, n + 2);
         }
         if (!SUMMARY) mma_read(ob);
@@ -644,14 +655,14 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       }
       tc::tmem_wait_st();
     };
-    if (wk.valid()) {
-      load_state(wk.get());
+    if (wk.valid(items)) {
+      load_state(wk.get(p));
       tc::tmem_fence_before();
       mbar_arrive(&bar_h);  // phase 0: the first chunk's state
     }
     uint32_t n = 0;
-    for (; wk.valid() && !*abort_flag; ++n, wk.next()) {
-      const Chunk ck = wk.get();
+    for (; wk.valid(items) && !*abort_flag; ++n, wk.next(p, items)) {
+      const Chunk ck = wk.get(p);
       const float* Dn = sDc + (n & 1) * kM;
       bool fast;
       if (!SUMMARY) {
@@ -689,72 +700,97 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       tc::tmem_fence_after();
       if (SUMMARY) fast = sFast[n & 1] != 0;
       Walker nx = wk;
-      nx.next();
+      nx.next(p, items);
       float* dst = nullptr;
       if (ck.last) {
         if (SUMMARY) dst = p.ws_state + ((int64_t)ck.pair * p.nseg + ck.seg + 1) * kM * kDV;
         else if (ck.seg == p.nseg - 1 && p.HT) dst = p.HT + (int64_t)ck.pair * kM * kDV;
       }
+      // the chunk-end state of 32 slots (in hv) is written out at the item's end, else back to
+      // TMEM with its tf32-rounded copy
+      auto put_state = [&](float (&hv)[32], int cg) {
+        if (ck.last) {
+          if (dst) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) dst[(cg + j) * kDV + dv] = hv[j];
+          }
+        } else {
+          tc::tmem_st32(tc::tmem_addr(tb, sub_lane, kColH + cg), hv);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) hv[j] = tc::to_tf32(hv[j]);
+          tc::tmem_st32(tc::tmem_addr(tb, sub_lane, kColHr + cg), hv);
+        }
+      };
+      if (fast) {
+        // H = D H, two groups of 32 slots per TMEM wait
 #pragma unroll 1
-      for (int c = 0; c < kM; c += 64) {
-        float hv[2][32];
-        tc::tmem_ld32(tc::tmem_addr(tb, sub_lane, kColH + c), hv[0]);
-        tc::tmem_ld32(tc::tmem_addr(tb, sub_lane, kColH + c + 32), hv[1]);
-        tc::tmem_wait_ld();
+        for (int c = 0; c < kM; c += 64) {
+          float hv[2][32];
+          tc::tmem_ld32(tc::tmem_addr(tb, sub_lane, kColH + c), hv[0]);
+          tc::tmem_ld32(tc::tmem_addr(tb, sub_lane, kColH + c + 32), hv[1]);
+          tc::tmem_wait_ld();
 #pragma unroll
-        for (int g = 0; g < 2; ++g) {
-          const int cg = c + 32 * g;
-          if (!fast) {
-            float uv[32];
-            tc::tmem_ld32(tc::tmem_addr(tb, sub_lane, kColU + cg), uv);
-            tc::tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 32; j += 4) {
-              const float4 d4 = *reinterpret_cast<const float4*>(Dn + cg + j);
-              hv[g][j] = fmaf(d4.x, hv[g][j], uv[j]);
-              hv[g][j + 1] = fmaf(d4.y, hv[g][j + 1], uv[j + 1]);
-              hv[g][j + 2] = fmaf(d4.z, hv[g][j + 2], uv[j + 2]);
-              hv[g][j + 3] = fmaf(d4.w, hv[g][j + 3], uv[j + 3]);
-            }
-          } else {
-            scale_by(hv[g], Dn + cg);  // slots not selected in the chunk: D = 1 exactly
+          for (int g = 0; g < 2; ++g) {
+            scale_by(hv[g], Dn + c + 32 * g);  // slots not selected in the chunk: D = 1 exactly
+            put_state(hv[g], c + 32 * g);
           }
-          if (ck.last) {
-            if (dst) {
+        }
+      } else {
+        // exact chunk: H = D H + U
+#pragma unroll 1
+        for (int c = 0; c < kM; c += 32) {
+          float hv[32], uv[32];
+          tc::tmem_ld32(tc::tmem_addr(tb, sub_lane, kColH + c), hv);
+          tc::tmem_ld32(tc::tmem_addr(tb, sub_lane, kColU + c), uv);
+          tc::tmem_wait_ld();
 #pragma unroll
-              for (int j = 0; j < 32; ++j) dst[(cg + j) * kDV + dv] = hv[g][j];
-            }
-          } else {
-            tc::tmem_st32(tc::tmem_addr(tb, sub_lane, kColH + cg), hv[g]);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) hv[g][j] = tc::to_tf32(hv[g][j]);
-            tc::tmem_st32(tc::tmem_addr(tb, sub_lane, kColHr + cg), hv[g]);
+          for (int j = 0; j < 32; j += 4) {
+            const float4 d4 = *reinterpret_cast<const float4*>(Dn + c + j);
+            hv[j] = fmaf(d4.x, hv[j], uv[j]);
+            hv[j + 1] = fmaf(d4.y, hv[j + 1], uv[j + 1]);
+            hv[j + 2] = fmaf(d4.z, hv[j + 2], uv[j + 2]);
+            hv[j + 3] = fmaf(d4.w, hv[j + 3], uv[j + 3]);
           }
+          put_state(hv, c);
         }
       }
       tc::tmem_wait_st();
-      if (ck.last && nx.valid()) load_state(nx.get());
+      if (ck.last && nx.valid(items)) load_state(nx.get(p));
       tc::tmem_fence_before();
       mbar_arrive(&bar_h);  // phase n+1: the state of the next chunk
       // ---- every MMA of this chunk is done: its output
       if (!SUMMARY) {
         wait_or_abort(&bar_o, n & 1, abort_flag);
         tc::tmem_fence_after();
-        float* orow = p.o + (((int64_t)ck.b * T + ck.c0) * H + ck.h) * kDV + dv;
-        const int64_t ostride = (int64_t)H * kDV;
         float ov[2][32];
         tc::tmem_ld32(tc::tmem_addr(tb, sub_lane, kColO + (n & 1) * kC), ov[0]);
         tc::tmem_ld32(tc::tmem_addr(tb, sub_lane, kColO + (n & 1) * kC + 32), ov[1]);
         tc::tmem_wait_ld();
-        // the O buffer is free once read; signal before the stores (an arrive after them would
-        // wait for the stores to complete)
-        tc::tmem_fence_before();
-        mbar_arrive(&bar_of[n & 1]);
+        // each half (32 tokens x 128 columns) is staged in the A tile's memory, free after A.V,
+        // and written out by one bulk tensor store (tokens past T are clipped by the map)
+        float* stg = reinterpret_cast<float*>(sA);
 #pragma unroll
-        for (int j = 0; j < kC; ++j)
-          if (j < ck.nrows) orow[(int64_t)j * ostride] = ov[j >> 5][j & 31];
+        for (int hf = 0; hf < 2; ++hf) {
+          if (hf == 1) {
+            if (tid == kEpiThread0) tc::bulk_wait_read_all();
+            bar_epi();
+          }
+#pragma unroll
+          for (int j = 0; j < 32; ++j) stg[j * kDV + dv] = ov[hf][j];
+          tc::fence_async_smem();
+          bar_epi();
+          if (tid == kEpiThread0) {
+            tc::tma_store_4d(&maps.o, stg, 0, ck.h, ck.c0 + 32 * hf, ck.b);
+            tc::bulk_commit_group();
+          }
+        }
+        if (tid == kEpiThread0) tc::bulk_wait_read_all();
+        bar_epi();
+        tc::tmem_fence_before();
+        mbar_arrive(&bar_of[n & 1]);  // the O buffer and the staging memory are free
       }
     }
+    if (tid == kEpiThread0) tc::bulk_wait_all();  // output stores complete before the CTA ends
   }
 
   tc::tmem_fence_before();
@@ -803,17 +839,18 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 4-D map over [B, T, H, C] bf16 (C innermost) with a box of one (b, h) and 64 tokens.
-bool make_map(CUtensorMap* m, const void* base, int B, int T, int H, int C) {
+// 4-D map over [B, T, H, C] (C innermost) with a box of one (b, h) and `box_t` tokens.
+bool make_map(CUtensorMap* m, const void* base, int B, int T, int H, int C, bool fp32, int box_t) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
+  const cuuint64_t es = fp32 ? 4 : 2;
   cuuint64_t dims[4] = {(cuuint64_t)C, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
-  cuuint64_t strides[3] = {(cuuint64_t)C * 2, (cuuint64_t)H * C * 2, (cuuint64_t)T * H * C * 2};
-  cuuint32_t box[4] = {(cuuint32_t)C, 1, (cuuint32_t)kC, 1};
+  cuuint64_t strides[3] = {(cuuint64_t)C * es, (cuuint64_t)H * C * es, (cuuint64_t)T * H * C * es};
+  cuuint32_t box[4] = {(cuuint32_t)C, 1, (cuuint32_t)box_t, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return fn(m, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base),
+            dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 int sm_count() {
@@ -918,7 +955,8 @@ cudaError_t launch_prefill_tc(const rsm_forward_args& a, cudaStream_t stream) {
   if (e == cudaSuccess) e = profile_mark(stream);
   if (e != cudaSuccess) return e;
   Maps maps;
-  if (!make_map(&maps.v, a.v, a.B, a.T, a.H, kDV)) return cudaErrorInvalidValue;
+  if (!make_map(&maps.v, a.v, a.B, a.T, a.H, kDV, false, kC)) return cudaErrorInvalidValue;
+  if (!make_map(&maps.o, a.o, a.B, a.T, a.H, kDV, true, kC / 2)) return cudaErrorInvalidValue;
   Params p;
   p.B = a.B; p.T = a.T; p.H = a.H; p.K = a.K;
   p.q = static_cast<const __nv_bfloat16*>(a.q);
