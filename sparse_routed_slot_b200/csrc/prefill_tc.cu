@@ -649,9 +649,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] = Hs ? Hs[(c + j) * kDV + dv] : 0.f;
         tc::tmem_st32(tc::tmem_addr(tb, sub_lane, kColH + c), v);
+        if (!SUMMARY) {  // the summary pass has no read, so no rounded copy
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = tc::to_tf32(v[j]);
-        tc::tmem_st32(tc::tmem_addr(tb, sub_lane, kColHr + c), v);
+          for (int j = 0; j < 32; ++j) v[j] = tc::to_tf32(v[j]);
+          tc::tmem_st32(tc::tmem_addr(tb, sub_lane, kColHr + c), v);
+        }
       }
       tc::tmem_wait_st();
     };
@@ -716,9 +718,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
           }
         } else {
           tc::tmem_st32(tc::tmem_addr(tb, sub_lane, kColH + cg), hv);
+          if (!SUMMARY) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) hv[j] = tc::to_tf32(hv[j]);
-          tc::tmem_st32(tc::tmem_addr(tb, sub_lane, kColHr + cg), hv);
+            for (int j = 0; j < 32; ++j) hv[j] = tc::to_tf32(hv[j]);
+            tc::tmem_st32(tc::tmem_addr(tb, sub_lane, kColHr + cg), hv);
+          }
         }
       };
       if (fast) {

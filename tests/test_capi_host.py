@@ -138,3 +138,24 @@ def test_binding_fails_loudly_without_the_library(tmp_path):
                 ROOT, str(tmp_path / "missing.so"))
     out = subprocess.check_output([sys.executable, "-c", code]).decode()
     assert "raised" in out
+
+
+def test_profile_events_arguments(lib):
+    L = lib.load()
+    fake = (ctypes.c_void_p * 2)(1 << 20, 1 << 21)
+    assert L.rsm_forward_set_profile_events(fake, 0) == 1                  # events without a count
+    assert L.rsm_forward_set_profile_events(None, 0) == 0                  # recording off
+    # too few events for a tensor-path call: rejected on the host, before any launch
+    a = lib.ForwardArgs()
+    a.B, a.T, a.H, a.M, a.K, a.Dv = 1, 64, 2, 128, 16, 128
+    a.qkv_dtype, a.decay = lib.RSM_BF16, lib.RSM_DECAY_HEAD
+    for n in ("q", "k", "v", "logits", "f", "o"):
+        setattr(a, n, 1 << 20)
+    a.workspace = 1 << 24
+    a.workspace_bytes = L.rsm_forward_workspace_size(ctypes.byref(a))
+    assert L.rsm_forward_set_profile_events(fake, 2) == 0
+    try:
+        assert L.rsm_forward(ctypes.byref(a), None) == 1
+        assert "profiling events" in lib.last_error()
+    finally:
+        assert L.rsm_forward_set_profile_events(None, 0) == 0

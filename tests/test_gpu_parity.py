@@ -303,3 +303,35 @@ def test_tensor_path_is_selected_for_supported_shapes(rsm):
     a = api._forward_args(y["q"], y["k"], y["v"], y["logits"], y["f"], 16, None, o, None, None, None,
                           "auto", False)
     assert api.selected_path(a) == "simt"
+
+
+def test_forward_profile_events_split_the_call(rsm):
+    """rsm_forward_set_profile_events: one event before the first kernel and one after each; the
+    per-kernel times add up to the whole call, and results are unchanged."""
+    import ctypes
+    from sparse_routed_slot_b200 import _lib, api
+    B, T, H, M, K, Dv = 1, 3000, 2, 128, 16, 128
+    x = make_inputs(B, T, H, M, Dv, torch.bfloat16, "head", seed=31, device="cuda")
+    ref = rsm.forward(x["q"], x["k"], x["v"], x["logits"], x["f"], K)
+    o = torch.empty_like(ref["o"])
+    HT = torch.empty_like(ref["HT"])
+    a = api._forward_args(x["q"], x["k"], x["v"], x["logits"], x["f"], K, None, o, HT, None, None, "auto", False)
+    n = api.kernel_launches(a)
+    assert n >= 2
+    stream = torch.cuda.current_stream()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(n + 1)]
+    for e in ev:
+        e.record(stream)  # creates the CUDA events
+    torch.cuda.synchronize()
+    L = _lib.load()
+    ptrs = (ctypes.c_void_p * (n + 1))(*[e.cuda_event for e in ev])
+    _lib.check(L.rsm_forward_set_profile_events(ptrs, n + 1))
+    try:
+        rsm.forward(x["q"], x["k"], x["v"], x["logits"], x["f"], K, out={"o": o, "HT": HT})
+    finally:
+        _lib.check(L.rsm_forward_set_profile_events(None, 0))
+    torch.cuda.synchronize()
+    parts = [ev[i].elapsed_time(ev[i + 1]) for i in range(n)]
+    assert all(p > 0 for p in parts)
+    assert abs(sum(parts) - ev[0].elapsed_time(ev[n])) < 1e-3
+    assert torch.equal(o, ref["o"]) and torch.equal(HT, ref["HT"])
