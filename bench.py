@@ -145,13 +145,27 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The maximum of `x` over all ranks (a device tensor under NCCL, a host tensor under gloo)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(units_per_rank: int, ms_per_rank: float, world: int) -> tuple[float, float]:
+    """Whole-job rate of N replicas: the units of all ranks over the slowest rank's time.
+    Returns (rate per second, the max time in ms)."""
+    ms_max = max_over_ranks(ms_per_rank, world)
+    return units_per_rank * world / (ms_max * 1e-3), ms_max
+
+
+def replica_seed(base: int, rank: int) -> int:
+    """Each replica draws its own inputs."""
+    return base + 1000 * rank
 
 
 # --------------------------------------------------------------------------- CPU oracle timing
@@ -228,7 +242,7 @@ def run_ours(args, world, rank, local):
     w = WORKLOADS[args.workload]
     dev = torch.device("cuda", local)
     peaks = load_peaks()
-    x = make_inputs(w.B, w.T, w.H, w.M, w.Dv, w.torch_dtype, w.decay, seed=w.seed + 1000 * rank, device=dev)
+    x = make_inputs(w.B, w.T, w.H, w.M, w.Dv, w.torch_dtype, w.decay, seed=replica_seed(w.seed, rank), device=dev)
     o = torch.empty(w.B, w.T, w.H, w.Dv, dtype=torch.float32, device=dev)
     HT = torch.empty(w.B, w.H, w.M, w.Dv, dtype=torch.float32, device=dev)
     outs = {"o": o, "HT": HT}
@@ -271,11 +285,10 @@ def run_ours(args, world, rank, local):
     clk = clocks.stop()
     per = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
     ms = sum(per) / len(per)
-    ms_max = max_over_ranks(ms, world)
     kms = [sum(row[j].elapsed_time(row[j + 1]) for row in kev) / args.steps for j in range(launches)]
     names = KERNEL_NAMES.get(launches, [f"kernel {j}" for j in range(launches)])
     tokens = w.B * w.T
-    value = tokens * world / (ms_max * 1e-3)
+    value, ms_max = job_throughput(tokens, ms, world)
 
     # end to end through the public call with host buffers: pinned inputs copied in, result out
     host_in = {n: t.cpu().pin_memory() for n, t in x.items()}
