@@ -555,32 +555,37 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         nx.next(p, items);
         load_v(nx, 1);
       }
-      const uint32_t q = tc::smem_u32(sQ), wsm = tc::smem_u32(sW), wt = tc::smem_u32(sWt),
-                     vt = tc::smem_u32(sVt), a = tc::smem_u32(sA);
+      // Descriptors are built once per tile; a K step only advances the start-address field (the
+      // low 14 bits, in 16-byte units), so each MMA costs the issuing thread about one add. The
+      // issuer shares its scheduler with three busy warps: fewer instructions per MMA is what
+      // keeps the tensor core fed.
+      const uint64_t dQ = tc::smem_desc(tc::smem_u32(sQ), 16, 1024), dW = tc::smem_desc(tc::smem_u32(sW), 16, 1024),
+                     dWt = tc::smem_desc(tc::smem_u32(sWt), 16, 1024), dVt = tc::smem_desc(tc::smem_u32(sVt), 16, 1024),
+                     dA = tc::smem_desc(tc::smem_u32(sA), 16, 1024);
+      // start-address advance of K step j in a tile with R rows: column block j/4 (R*128 bytes),
+      // 32 bytes (8 tf32) within the 128-byte row
+      auto kstep = [](int R, int j) -> uint64_t { return (uint64_t)(((j >> 2) * (R * 128) + (j & 3) * 32) >> 4); };
+      constexpr uint32_t kIdS = tc::idesc_tf32(64, kC, 0, 0), kIdO = tc::idesc_tf32(kDV, kC, 0, 0),
+                         kIdC = tc::idesc_tf32(kDV, kM, 0, 0);
+      auto mma_s = [&]() {  // S = Qh Wh^T
+#pragma unroll
+        for (int j = 0; j < kM / 8; ++j)
+          tc::mma_tf32_ss(tb + kColS, dQ + kstep(kC, j), dW + kstep(kC, j), kIdS, j > 0);
+      };
       auto mma_read = [&](uint32_t ob) {  // O^T = H^T Qh^T (state read from TMEM)
-#pragma unroll 1
-        for (int j = 0; j < kM / 8; ++j) {
-          const uint32_t off = (j >> 2) * (kC * 128) + (j & 3) * 32;
-          tc::mma_tf32_ts(tb + kColO + ob, tb + kColHr + 8 * j, tc::smem_desc(q + off, 16, 1024),
-                          tc::idesc_tf32(kDV, kC, 0, 0), j > 0);
-        }
+#pragma unroll
+        for (int j = 0; j < kM / 8; ++j)
+          tc::mma_tf32_ts(tb + kColO + ob, tb + kColHr + 8 * j, dQ + kstep(kC, j), kIdO, j > 0);
       };
       auto mma_carry = [&](uint32_t col, bool acc) {  // H^T += V^T Wh, or U^T = V^T Wh
-#pragma unroll 1
-        for (int j = 0; j < kC / 8; ++j) {
-          const uint32_t off = (j >> 2) * (kM * 128) + (j & 3) * 32;
-          tc::mma_tf32_ss(tb + col, tc::smem_desc(vt + off, 16, 1024), tc::smem_desc(wt + off, 16, 1024),
-                          tc::idesc_tf32(kDV, kM, 0, 0), (acc || j > 0) ? 1u : 0u);
-        }
+#pragma unroll
+        for (int j = 0; j < kC / 8; ++j)
+          tc::mma_tf32_ss(tb + col, dVt + kstep(kM, j), dWt + kstep(kM, j), kIdC, (acc || j > 0) ? 1u : 0u);
       };
       auto mma_av = [&](uint32_t ob) {  // O^T += V^T A^T
-#pragma unroll 1
-        for (int j = 0; j < kC / 8; ++j) {
-          const uint32_t offa = (j >> 2) * (kC * 128) + (j & 3) * 32;
-          const uint32_t offv = (j >> 2) * (kDV * 128) + (j & 3) * 32;
-          tc::mma_tf32_ss(tb + kColO + ob, tc::smem_desc(vt + offv, 16, 1024), tc::smem_desc(a + offa, 16, 1024),
-                          tc::idesc_tf32(kDV, kC, 0, 0), 1);
-        }
+#pragma unroll
+        for (int j = 0; j < kC / 8; ++j)
+          tc::mma_tf32_ss(tb + kColO + ob, dVt + kstep(kDV, j), dA + kstep(kC, j), kIdO, 1);
       };
       bool prev_exact = false;
       for (; wk.valid(items) && !*abort_flag; ++n, wk.next(p, items)) {
@@ -593,14 +598,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             wait_or_abort(&bar_h, n & 1, abort_flag);
             tc::tmem_fence_after();
           }
-          if (fast) {
-#pragma unroll 1
-            for (int j = 0; j < kM / 8; ++j) {  // S = Qh Wh^T
-              const uint32_t off = (j >> 2) * (kC * 128) + (j & 3) * 32;
-              tc::mma_tf32_ss(tb + kColS, tc::smem_desc(q + off, 16, 1024), tc::smem_desc(wsm + off, 16, 1024),
-                              tc::idesc_tf32(64, kC, 0, 0), j > 0);
-            }
-          }
+          if (fast) mma_s();
           tc::mma_commit(&bar_s);  // every main-pass chunk: tells the epilogue the chunk is ready
         }
         wait_or_abort(&bar_h, n & 1, abort_flag);  // state ready
