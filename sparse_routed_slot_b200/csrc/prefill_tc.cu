@@ -52,9 +52,10 @@
 // can fall two phases behind (which a parity wait cannot tell from zero).
 //
 // Long sequences with few (b,h) streams are split into segments processed in parallel: a summary
-// pass runs the state recurrence of each segment but the last from a zero state and stores
-// (prod of chunk decays, end state); a scan combines them into the true start state of every
-// segment; the main pass then runs every segment from its start state.
+// kernel (segment_summary_kernel, below) computes for each segment but the last the product of
+// its decays and the state it reaches from a zero start, as one accumulation of end-referenced
+// weights; a scan combines them into the true start state of every segment; the main pass then
+// runs every segment from its start state.
 #include <cuda.h>
 
 #include <mutex>
@@ -271,7 +272,7 @@ RSM_DEV void for_entries(const RowInputs<KP>& in, int lane, int K, int nrows_w, 
   }
 }
 
-template <bool SUMMARY, int KP>
+template <int KP>
 __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_constant__ Maps maps,
                                                                   const Params p) {
   extern __shared__ unsigned char smem_raw[];
@@ -304,8 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int T = p.T, H = p.H, K = p.K;
   const int pairs = p.B * H;
-  const int segs_here = SUMMARY ? p.nseg - 1 : p.nseg;
-  const int items = pairs * segs_here;
+  const int items = pairs * p.nseg;
 
   if (warp == kIssuerWarp) tc::tmem_alloc(&s_tbase, kTmemCols);
   if (tid == 0) {
@@ -339,10 +339,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     const int w = warp;
     const int RB = p.rec_bytes;
     float* tab = sTab + w * kRowsPerWarp * kM;  // this warp's rows of the decay table
-    float Dseg[4] = {1.f, 1.f, 1.f, 1.f};       // summary pass, warp 0: product of the chunk decays
 
     RowInputs<KP> cur;
-    if (wk.valid(items)) load_rows<SUMMARY, KP>(p, wk.get(p), w, lane, cur);
+    if (wk.valid(items)) load_rows<false, KP>(p, wk.get(p), w, lane, cur);
     for (uint32_t n = 0; wk.valid(items); ++n, wk.next(p, items)) {
       const Chunk ck = wk.get(p);
       const int buf = n & 1;
@@ -389,11 +388,6 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         for (int e = 0; e < 4; ++e) {
           const int slot = lane * 4 + e;
           sDc[buf * kM + slot] = gend[e];
-          if (SUMMARY) {
-            if (ck.first) Dseg[e] = 1.f;
-            Dseg[e] *= gend[e];
-            if (ck.last) p.ws_D[((int64_t)ck.pair * p.nseg + ck.seg + 1) * kM + slot] = Dseg[e];
-          }
         }
         if (lane == 0) sFast[buf] = fast;
       }
@@ -411,10 +405,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
           for (int e = 0; e < 4; ++e) {
             G[e] *= fabsf(av[e]);
             qh[e] = tc::to_tf32(fget(q4, e) * G[e]);
-            gw[e] = (SUMMARY || sign_set(av[e])) ? G[e] : 0.f;
+            gw[e] = sign_set(av[e]) ? G[e] : 0.f;
           }
-          if (!SUMMARY)
-            *reinterpret_cast<float4*>(sQ + tc::swz_offset(kC, t, lane * 4)) = make_float4(qh[0], qh[1], qh[2], qh[3]);
+          *reinterpret_cast<float4*>(sQ + tc::swz_offset(kC, t, lane * 4)) = make_float4(qh[0], qh[1], qh[2], qh[3]);
           *reinterpret_cast<float4*>(sW + tc::swz_offset(kC, t, lane * 4)) = make_float4(gw[0], gw[1], gw[2], gw[3]);
         }
         // this warp's token columns of Wh^T start at zero
@@ -431,7 +424,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
           const int t = w * kRowsPerWarp + r;
           float* gp = reinterpret_cast<float*>(sW + tc::swz_offset(kC, t, slot));
           const float wh = tc::to_tf32(__fdividef(wv, *gp));
-          if (!SUMMARY) *gp = wh;
+          *gp = wh;
           *reinterpret_cast<float*>(sWt + tc::swz_offset(kM, slot, t)) = wh;
         });
         tc::fence_async_smem();
@@ -442,7 +435,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         // read, the carry into U and A.V; the epilogue then forms H = D H + U.
         // A.V of the chunk before is done with A, and the epilogue has staged that chunk's output
         // through the A tile's memory
-        if (!SUMMARY && n > 0) wait_or_abort(&bar_of[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag);
+        if (n > 0) wait_or_abort(&bar_of[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag);
         bar_rows();  // every row worker is past the product totals
 #pragma unroll
         for (int i = 0; i < kRowsPerWarp; ++i)
@@ -470,12 +463,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
           const float4 l4 = reinterpret_cast<const float4*>(tab + r * kM)[lane];
           g[0] += l4.x; g[1] += l4.y; g[2] += l4.z; g[3] += l4.w;
           reinterpret_cast<float4*>(dg + t * kM)[lane] = make_float4(g[0], g[1], g[2], g[3]);
-          if (!SUMMARY) {
-            const float4 q4 = bf16x4_to_f32(cur.q[r]);
-            *reinterpret_cast<float4*>(sQ + tc::swz_offset(kC, t, lane * 4)) =
-                make_float4(tc::to_tf32(q4.x * expf(g[0])), tc::to_tf32(q4.y * expf(g[1])),
-                            tc::to_tf32(q4.z * expf(g[2])), tc::to_tf32(q4.w * expf(g[3])));
-          }
+          const float4 q4 = bf16x4_to_f32(cur.q[r]);
+          *reinterpret_cast<float4*>(sQ + tc::swz_offset(kC, t, lane * 4)) =
+              make_float4(tc::to_tf32(q4.x * expf(g[0])), tc::to_tf32(q4.y * expf(g[1])),
+                          tc::to_tf32(q4.z * expf(g[2])), tc::to_tf32(q4.w * expf(g[3])));
         }
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -490,23 +481,21 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
           *reinterpret_cast<float*>(sWt + tc::swz_offset(kM, slot, t)) =
               tc::to_tf32(wv * expf(dg[(kC - 1) * kM + slot] - dg[t * kM + slot]));
         });
-        if (!SUMMARY) {
-          const int nrows = ck.nrows;
-          const unsigned char* rb = p.rec + ((int64_t)ck.pair * T + ck.c0) * RB;
-          for (int e = tid; e < kC * kC; e += kRThreads) {
-            const int t = e / kC, s = e % kC;
-            float acc = 0.f;
-            if (s <= t && t < nrows) {
-              const int64_t rowt = ((int64_t)ck.b * T + ck.c0 + t) * H + ck.h;
-              const unsigned char* rs = rb + s * RB;
-              for (int j = 0; j < K; ++j) {
-                const int i = rs[j];
-                const float wj = reinterpret_cast<const float*>(rs + 5 * KP)[j];
-                acc = fmaf(bf16_at(p.q + rowt * kM + i) * wj, expf(dg[t * kM + i] - dg[s * kM + i]), acc);
-              }
+        const int nrows = ck.nrows;
+        const unsigned char* rb = p.rec + ((int64_t)ck.pair * T + ck.c0) * RB;
+        for (int e = tid; e < kC * kC; e += kRThreads) {
+          const int t = e / kC, s = e % kC;
+          float acc = 0.f;
+          if (s <= t && t < nrows) {
+            const int64_t rowt = ((int64_t)ck.b * T + ck.c0 + t) * H + ck.h;
+            const unsigned char* rs = rb + s * RB;
+            for (int j = 0; j < K; ++j) {
+              const int i = rs[j];
+              const float wj = reinterpret_cast<const float*>(rs + 5 * KP)[j];
+              acc = fmaf(bf16_at(p.q + rowt * kM + i) * wj, expf(dg[t * kM + i] - dg[s * kM + i]), acc);
             }
-            *reinterpret_cast<float*>(sA + tc::swz_offset(kC, t, s)) = tc::to_tf32(acc);
           }
+          *reinterpret_cast<float*>(sA + tc::swz_offset(kC, t, s)) = tc::to_tf32(acc);
         }
         tc::fence_async_smem();
         mbar_arrive(&bar_rdy);
@@ -517,7 +506,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       {
         Walker nx = wk;
         nx.next(p, items);
-        if (nx.valid(items)) load_rows<SUMMARY, KP>(p, nx.get(p), w, lane, nxt);
+        if (nx.valid(items)) load_rows<false, KP>(p, nx.get(p), w, lane, nxt);
       }
       // ---- V^T of this chunk: its v tile has landed and the chunk before has finished A.V
       if (n > 0) wait_or_abort(&bar_o, (n - 1) & 1, abort_flag);
@@ -593,16 +582,14 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         wait_or_abort(&bar_rdy, n & 1, abort_flag);
         const bool fast = sFast[n & 1] != 0;
         tc::tmem_fence_after();
-        if (!SUMMARY) {
-          if (fast && prev_exact) {  // S overwrites the columns of the previous chunk's U
-            wait_or_abort(&bar_h, n & 1, abort_flag);
-            tc::tmem_fence_after();
-          }
-          if (fast) mma_s();
-          tc::mma_commit(&bar_s);  // every main-pass chunk: tells the epilogue the chunk is ready
+        if (fast && prev_exact) {  // S overwrites the columns of the previous chunk's U
+          wait_or_abort(&bar_h, n & 1, abort_flag);
+          tc::tmem_fence_after();
         }
+        if (fast) mma_s();
+        tc::mma_commit(&bar_s);  // every main-pass chunk: tells the epilogue the chunk is ready
         wait_or_abort(&bar_h, n & 1, abort_flag);  // state ready
-        if (!SUMMARY && n >= 2) wait_or_abort(&bar_of[n & 1], ((n - 2) >> 1) & 1, abort_flag);  // O buffer free
+        if (n >= 2) wait_or_abort(&bar_of[n & 1], ((n - 2) >> 1) & 1, abort_flag);  // O buffer free
         wait_or_abort(&bar_vt, n & 1, abort_flag);  // V^T written
         tc::tmem_fence_after();
         {
@@ -612,14 +599,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
           nx.next(p, items);
           load_v(nx, n + 2);
         }
-        if (!SUMMARY) mma_read(ob);
+        mma_read(ob);
         mma_carry(fast ? kColH : kColU, fast);
         tc::mma_commit(&bar_t);
-        if (!SUMMARY) {
-          wait_or_abort(&bar_a, n & 1, abort_flag);
-          tc::tmem_fence_after();
-          mma_av(ob);
-        }
+        wait_or_abort(&bar_a, n & 1, abort_flag);
+        tc::tmem_fence_after();
+        mma_av(ob);
         tc::mma_commit(&bar_o);
         prev_exact = !fast;
       }
@@ -637,21 +622,17 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
 
     // the state of chunk ck's item into TMEM (H0, a segment start state, or zeros)
     auto load_state = [&](const Chunk& ck) {
-      const float* Hs = nullptr;
-      if (!SUMMARY)
-        Hs = p.nseg > 1 ? p.ws_state + ((int64_t)ck.pair * p.nseg + ck.seg) * kM * kDV
-                        : (p.H0 ? p.H0 + (int64_t)ck.pair * kM * kDV : nullptr);
+      const float* Hs = p.nseg > 1 ? p.ws_state + ((int64_t)ck.pair * p.nseg + ck.seg) * kM * kDV
+                                   : (p.H0 ? p.H0 + (int64_t)ck.pair * kM * kDV : nullptr);
 #pragma unroll 1
       for (int c = 0; c < kM; c += 32) {
         float v[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] = Hs ? Hs[(c + j) * kDV + dv] : 0.f;
         tc::tmem_st32(tc::tmem_addr(tb, sub_lane, kColH + c), v);
-        if (!SUMMARY) {  // the summary pass has no read, so no rounded copy
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = tc::to_tf32(v[j]);
-          tc::tmem_st32(tc::tmem_addr(tb, sub_lane, kColHr + c), v);
-        }
+        for (int j = 0; j < 32; ++j) v[j] = tc::to_tf32(v[j]);
+        tc::tmem_st32(tc::tmem_addr(tb, sub_lane, kColHr + c), v);
       }
       tc::tmem_wait_st();
     };
@@ -664,48 +645,41 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     for (; wk.valid(items) && !*abort_flag; ++n, wk.next(p, items)) {
       const Chunk ck = wk.get(p);
       const float* Dn = sDc + (n & 1) * kM;
-      bool fast;
-      if (!SUMMARY) {
-        wait_or_abort(&bar_s, n & 1, abort_flag);
-        tc::tmem_fence_after();
-        fast = sFast[n & 1] != 0;
-        if (fast) {
-          // S -> A (rows t = 16*(warp%4) + lane for lane < 16, at TMEM lanes 32*(warp%4) + lane)
-          const int t = (warp & 3) * 16 + lane;
+      wait_or_abort(&bar_s, n & 1, abort_flag);
+      tc::tmem_fence_after();
+      const bool fast = sFast[n & 1] != 0;
+      if (fast) {
+        // S -> A (rows t = 16*(warp%4) + lane for lane < 16, at TMEM lanes 32*(warp%4) + lane)
+        const int t = (warp & 3) * 16 + lane;
 #pragma unroll 1
-          for (int c = 0; c < kC; c += 32) {
-            float sv[32];
-            tc::tmem_ld32(tc::tmem_addr(tb, sub_lane, kColS + c), sv);
-            tc::tmem_wait_ld();
-            if (lane < 16) {
+        for (int c = 0; c < kC; c += 32) {
+          float sv[32];
+          tc::tmem_ld32(tc::tmem_addr(tb, sub_lane, kColS + c), sv);
+          tc::tmem_wait_ld();
+          if (lane < 16) {
 #pragma unroll
-              for (int j = 0; j < 32; j += 4) {
-                const int s = c + j;
-                const float4 a4 = make_float4(s <= t ? tc::to_tf32(sv[j]) : 0.f,
-                                              s + 1 <= t ? tc::to_tf32(sv[j + 1]) : 0.f,
-                                              s + 2 <= t ? tc::to_tf32(sv[j + 2]) : 0.f,
-                                              s + 3 <= t ? tc::to_tf32(sv[j + 3]) : 0.f);
-                *reinterpret_cast<float4*>(sA + tc::swz_offset(kC, t, s)) = a4;
-              }
+            for (int j = 0; j < 32; j += 4) {
+              const int s = c + j;
+              const float4 a4 = make_float4(s <= t ? tc::to_tf32(sv[j]) : 0.f,
+                                            s + 1 <= t ? tc::to_tf32(sv[j + 1]) : 0.f,
+                                            s + 2 <= t ? tc::to_tf32(sv[j + 2]) : 0.f,
+                                            s + 3 <= t ? tc::to_tf32(sv[j + 3]) : 0.f);
+              *reinterpret_cast<float4*>(sA + tc::swz_offset(kC, t, s)) = a4;
             }
           }
-          tc::fence_async_smem();
         }
-        tc::tmem_fence_before();
-        mbar_arrive(&bar_a);  // every main-pass chunk (an exact chunk's A comes from the row workers)
+        tc::fence_async_smem();
       }
+      tc::tmem_fence_before();
+      mbar_arrive(&bar_a);  // every main-pass chunk (an exact chunk's A comes from the row workers)
       // ---- after the carry: the state of the chunk end (fast: H = D H; exact: H = D H + U), the
       // item's state out at its end, the next item's state in at its start
       wait_or_abort(&bar_t, n & 1, abort_flag);
       tc::tmem_fence_after();
-      if (SUMMARY) fast = sFast[n & 1] != 0;
       Walker nx = wk;
       nx.next(p, items);
       float* dst = nullptr;
-      if (ck.last) {
-        if (SUMMARY) dst = p.ws_state + ((int64_t)ck.pair * p.nseg + ck.seg + 1) * kM * kDV;
-        else if (ck.seg == p.nseg - 1 && p.HT) dst = p.HT + (int64_t)ck.pair * kM * kDV;
-      }
+      if (ck.last && ck.seg == p.nseg - 1 && p.HT) dst = p.HT + (int64_t)ck.pair * kM * kDV;
       // the chunk-end state of 32 slots (in hv) is written out at the item's end, else back to
       // TMEM with its tf32-rounded copy
       auto put_state = [&](float (&hv)[32], int cg) {
@@ -716,11 +690,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
           }
         } else {
           tc::tmem_st32(tc::tmem_addr(tb, sub_lane, kColH + cg), hv);
-          if (!SUMMARY) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) hv[j] = tc::to_tf32(hv[j]);
-            tc::tmem_st32(tc::tmem_addr(tb, sub_lane, kColHr + cg), hv);
-          }
+          for (int j = 0; j < 32; ++j) hv[j] = tc::to_tf32(hv[j]);
+          tc::tmem_st32(tc::tmem_addr(tb, sub_lane, kColHr + cg), hv);
         }
       };
       if (fast) {
@@ -761,36 +733,34 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       tc::tmem_fence_before();
       mbar_arrive(&bar_h);  // phase n+1: the state of the next chunk
       // ---- every MMA of this chunk is done: its output
-      if (!SUMMARY) {
-        wait_or_abort(&bar_o, n & 1, abort_flag);
-        tc::tmem_fence_after();
-        float ov[2][32];
-        tc::tmem_ld32(tc::tmem_addr(tb, sub_lane, kColO + (n & 1) * kC), ov[0]);
-        tc::tmem_ld32(tc::tmem_addr(tb, sub_lane, kColO + (n & 1) * kC + 32), ov[1]);
-        tc::tmem_wait_ld();
-        // each half (32 tokens x 128 columns) is staged in the A tile's memory, free after A.V,
-        // and written out by one bulk tensor store (tokens past T are clipped by the map)
-        float* stg = reinterpret_cast<float*>(sA);
+      wait_or_abort(&bar_o, n & 1, abort_flag);
+      tc::tmem_fence_after();
+      float ov[2][32];
+      tc::tmem_ld32(tc::tmem_addr(tb, sub_lane, kColO + (n & 1) * kC), ov[0]);
+      tc::tmem_ld32(tc::tmem_addr(tb, sub_lane, kColO + (n & 1) * kC + 32), ov[1]);
+      tc::tmem_wait_ld();
+      // each half (32 tokens x 128 columns) is staged in the A tile's memory, free after A.V,
+      // and written out by one bulk tensor store (tokens past T are clipped by the map)
+      float* stg = reinterpret_cast<float*>(sA);
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          if (hf == 1) {
-            if (tid == kEpiThread0) tc::bulk_wait_read_all();
-            bar_epi();
-          }
-#pragma unroll
-          for (int j = 0; j < 32; ++j) stg[j * kDV + dv] = ov[hf][j];
-          tc::fence_async_smem();
+      for (int hf = 0; hf < 2; ++hf) {
+        if (hf == 1) {
+          if (tid == kEpiThread0) tc::bulk_wait_read_all();
           bar_epi();
-          if (tid == kEpiThread0) {
-            tc::tma_store_4d(&maps.o, stg, 0, ck.h, ck.c0 + 32 * hf, ck.b);
-            tc::bulk_commit_group();
-          }
         }
-        if (tid == kEpiThread0) tc::bulk_wait_read_all();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) stg[j * kDV + dv] = ov[hf][j];
+        tc::fence_async_smem();
         bar_epi();
-        tc::tmem_fence_before();
-        mbar_arrive(&bar_of[n & 1]);  // the O buffer and the staging memory are free
+        if (tid == kEpiThread0) {
+          tc::tma_store_4d(&maps.o, stg, 0, ck.h, ck.c0 + 32 * hf, ck.b);
+          tc::bulk_commit_group();
+        }
       }
+      if (tid == kEpiThread0) tc::bulk_wait_read_all();
+      bar_epi();
+      tc::tmem_fence_before();
+      mbar_arrive(&bar_of[n & 1]);  // the O buffer and the staging memory are free
     }
     if (tid == kEpiThread0) tc::bulk_wait_all();  // output stores complete before the CTA ends
   }
@@ -799,6 +769,293 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
   __syncthreads();
   tc::tmem_fence_after();
   if (warp == kIssuerWarp) tc::tmem_dealloc(tb, kTmemCols);
+}
+
+// ---------------------------------------------------------------------------------------------
+// Segment summaries (segmented runs). For every segment of a (b,h) stream but the last, the
+// state the recurrence reaches at the segment end from a zero start, and the product of the
+// segment's decays:
+//   D[i] = e^{Lam_i},  Lam_i = sum of lam_{t,i} over the segment's tokens
+//   U    = sum_t Wr_t^T v_t,  Wr_{t,i} = w_{t,i} e^{sum of lam_{s,i} over the segment's tokens s > t}
+// Referenced to the segment end, every exponent is <= 0: no division, no fast/exact split, and no
+// decay of an accumulator between chunks, so U is a single accumulation of V^T Wr over the
+// segment (one TMEM accumulator, chunk tiles double-buffered). The chunks are visited from the
+// segment's last to its first, so the exponent of a token is the running sum of the lam of the
+// tokens after it.
+//
+// Warp roles (one CTA per segment at a time, 9 warps):
+//   warps 0-7  row workers; warp w owns tokens 8w..8w+7 of the chunk, lane l slots 4l..4l+3 of
+//              the lam table. Per chunk: scatter the rows' lam into the table, walk the rows from
+//              the last to the first (exclusive in-warp suffix sums in place), exchange the warp
+//              totals, write Wr^T at the selected entries, convert the warp's tokens of the v
+//              tile into V^T; at the segment's end read U out of TMEM and write U and D.
+//   warp 8     MMA issuer (one thread): the v tile loads (two chunks ahead) and the 8 MMAs of
+//              each chunk, U^T += V^T Wr (M = value columns, N = slots, K = tokens).
+constexpr int kSumThreads = (kRWarps + 1) * 32;
+constexpr int kSumOffRawV = 0;                       // v tiles from TMA, [2][64 t][128 dv] bf16
+constexpr int kSumOffVt = kSumOffRawV + 32768;       // V^T  [2][128 dv][64 t] (A)
+constexpr int kSumOffWt = kSumOffVt + 2 * 32768;     // Wr^T [2][128 slot][64 t] (B)
+constexpr int kSumOffTab = kSumOffWt + 2 * 32768;    // lam table [64 t][128 slot], then exponents
+constexpr int kSumOffTot = kSumOffTab + 32768;       // per-warp lam sums [2][8][128]
+constexpr int kSumOffSuf = kSumOffTot + 2 * kRWarps * kM * 4;  // per-warp exponent offsets [8][128]
+constexpr int kSumSmemBytes = kSumOffSuf + kRWarps * kM * 4 + 1024;
+constexpr int kSumTmemCols = 128;
+static_assert(kSumSmemBytes <= 232448, "shared memory budget");
+
+// The summary pass visits item (pair, seg) = blockIdx.x + j*gridDim.x, seg < nseg - 1, and the
+// item's chunks from the last to the first; first/last refer to that visiting order.
+struct SumWalker {
+  int item, pair, seg, b, h, t0, nch, i;
+  __device__ void set_item(const Params& p, int items) {
+    if (item >= items) return;
+    const int pairs = p.B * p.H;
+    seg = item / pairs;
+    pair = item - seg * pairs;
+    b = pair / p.H;
+    h = pair - b * p.H;
+    t0 = seg * p.seg_chunks * kC;
+    const int t1 = min(p.T, t0 + p.seg_chunks * kC);
+    nch = (t1 - t0 + kC - 1) / kC;
+    i = 0;
+  }
+  __device__ void start(const Params& p, int items) {
+    item = blockIdx.x;
+    set_item(p, items);
+  }
+  __device__ bool valid(int items) const { return item < items; }
+  __device__ Chunk get(const Params& p) const {
+    Chunk c;
+    c.pair = pair;
+    c.seg = seg;
+    c.b = b;
+    c.h = h;
+    c.c0 = t0 + (nch - 1 - i) * kC;
+    c.nrows = min(kC, min(p.T, t0 + p.seg_chunks * kC) - c.c0);
+    c.first = i == 0;
+    c.last = i == nch - 1;
+    return c;
+  }
+  __device__ void next(const Params& p, int items) {
+    if (++i >= nch) {
+      item += gridDim.x;
+      set_item(p, items);
+    }
+  }
+};
+
+template <int KP>
+__global__ void __launch_bounds__(kSumThreads, 1) segment_summary_kernel(const __grid_constant__ Maps maps,
+                                                                          const Params p) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* sm = reinterpret_cast<unsigned char*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  unsigned char* sRawV = sm + kSumOffRawV;
+  unsigned char* sVt = sm + kSumOffVt;
+  unsigned char* sWt = sm + kSumOffWt;
+  float* sTab = reinterpret_cast<float*>(sm + kSumOffTab);
+  float* sTot = reinterpret_cast<float*>(sm + kSumOffTot);
+  float* sSuf = reinterpret_cast<float*>(sm + kSumOffSuf);
+
+  __shared__ __align__(8) uint64_t bar_rdy[2],  // tiles of chunk n in buffer n&1 written (row threads)
+      bar_tma[2],                                // raw v tile of chunk n landed          (TMA)
+      bar_mma[2],                                // MMAs of chunk n done, buffer n&1 free (MMA commit)
+      bar_out,                                   // U of an item read out of TMEM         (row threads)
+      bar_fin;                                   // issuer only: every MMA issued is done (MMA commit)
+  __shared__ uint32_t s_tbase;
+  __shared__ int s_abort;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int K = p.K;
+  const int items = p.B * p.H * (p.nseg - 1);
+
+  if (warp == kIssuerWarp) tc::tmem_alloc(&s_tbase, kSumTmemCols);
+  if (tid == 0) {
+    for (int b = 0; b < 2; ++b) {
+      tc::mbar_init(&bar_rdy[b], kRThreads);
+      tc::mbar_init(&bar_tma[b], 1);
+      tc::mbar_init(&bar_mma[b], 1);
+    }
+    tc::mbar_init(&bar_out, kRThreads);
+    tc::mbar_init(&bar_fin, 1);
+    tc::fence_mbar_init();
+    s_abort = 0;
+  }
+  if (warp == kIssuerWarp && lane == 0) tc::tma_prefetch_desc(&maps.v);
+  tc::tmem_fence_before();
+  __syncthreads();
+  tc::tmem_fence_after();
+  const uint32_t tb = s_tbase;
+  volatile int* abort_flag = &s_abort;
+
+  SumWalker wk;
+  wk.start(p, items);
+
+  if (warp < kRWarps) {
+    // =========================================================================== row workers
+    const int w = warp;
+    float* tab = sTab + w * kRowsPerWarp * kM;  // this warp's rows of the table
+    float lamS[4] = {0.f, 0.f, 0.f, 0.f};      // Lam of the item's tokens after this chunk (slots 4l..)
+    RowInputs<KP> cur;
+    if (wk.valid(items)) load_rows<true, KP>(p, wk.get(p), w, lane, cur);
+    for (uint32_t n = 0; wk.valid(items); ++n, wk.next(p, items)) {
+      const Chunk ck = wk.get(p);
+      const int buf = n & 1;
+      const int nrows_w = ck.nrows - w * kRowsPerWarp;
+      if (ck.first) lamS[0] = lamS[1] = lamS[2] = lamS[3] = 0.f;
+      // the next chunk's records start loading (they have this whole chunk to arrive)
+      RowInputs<KP> nxt;
+      {
+        SumWalker nx = wk;
+        nx.next(p, items);
+        if (nx.valid(items)) load_rows<true, KP>(p, nx.get(p), w, lane, nxt);
+      }
+      // ---- the warp's rows of the table: lam at the selected entries, 0 elsewhere
+#pragma unroll
+      for (int i = 0; i < kRowsPerWarp; ++i)
+        reinterpret_cast<float4*>(tab)[lane + 32 * i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      __syncwarp();
+      for_entries(cur, lane, K, nrows_w, [&](int r, int slot, float lam, float) { tab[r * kM + slot] = lam; });
+      __syncwarp();
+      // ---- walk the rows from the last: each entry becomes the sum of lam below it in the warp
+      float run[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int r = kRowsPerWarp - 1; r >= 0; --r) {
+        float4* row = reinterpret_cast<float4*>(tab + r * kM) + lane;
+        const float4 x = *row;
+        *row = make_float4(run[0], run[1], run[2], run[3]);
+        run[0] += x.x; run[1] += x.y; run[2] += x.z; run[3] += x.w;
+      }
+      reinterpret_cast<float4*>(sTot + (buf * kRWarps + w) * kM)[lane] = make_float4(run[0], run[1], run[2], run[3]);
+      if (bar_rows_or(*abort_flag != 0)) break;  // every row worker takes the same decision
+      // ---- exponent offset of the warp's rows (lam of the later warps' rows and later chunks), and
+      // Lam past the next chunk (every row warp sums in the same order, so all hold the same value)
+      float suf[4] = {lamS[0], lamS[1], lamS[2], lamS[3]}, tot[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int w2 = 0; w2 < kRWarps; ++w2) {
+        const float4 t4 = reinterpret_cast<const float4*>(sTot + (buf * kRWarps + w2) * kM)[lane];
+        const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if (w2 > w) suf[e] += tv[e];
+          tot[e] += tv[e];
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) lamS[e] += tot[e];
+      reinterpret_cast<float4*>(sSuf + w * kM)[lane] = make_float4(suf[0], suf[1], suf[2], suf[3]);
+      // ---- tile buffer `buf` is free once the MMAs of chunk n-2 are done
+      if (n >= 2) wait_or_abort(&bar_mma[buf], ((n - 2) >> 1) & 1, abort_flag);
+      unsigned char* wt = sWt + buf * 32768;
+      unsigned char* vt = sVt + buf * 32768;
+      // the warp's token columns of Wr^T start at zero (rows slot = lane + 32e: 4-way stores)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int slot = lane + 32 * e;
+        *reinterpret_cast<float4*>(wt + tc::swz_offset(kM, slot, w * kRowsPerWarp)) = make_float4(0.f, 0.f, 0.f, 0.f);
+        *reinterpret_cast<float4*>(wt + tc::swz_offset(kM, slot, w * kRowsPerWarp + 4)) =
+            make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      __syncwarp();
+      // ---- each entry's owner: Wr = w e^{exponent} (exponent <= 0)
+      for_entries(cur, lane, K, nrows_w, [&](int r, int slot, float, float wv) {
+        const float x = tab[r * kM + slot] + sSuf[w * kM + slot];
+        *reinterpret_cast<float*>(wt + tc::swz_offset(kM, slot, w * kRowsPerWarp + r)) = tc::to_tf32(wv * expf(x));
+      });
+      // ---- V^T of the warp's 8 tokens (value columns lane + 32e; rows past the sequence end are
+      // zero in the tile)
+      wait_or_abort(&bar_tma[buf], (n >> 1) & 1, abort_flag);
+      const uint16_t* raw = reinterpret_cast<const uint16_t*>(sRawV + buf * (kC * kDV * 2));
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int dv = lane + 32 * e;
+        float x[kRowsPerWarp];
+#pragma unroll
+        for (int r = 0; r < kRowsPerWarp; ++r)
+          x[r] = __uint_as_float((uint32_t)raw[(w * kRowsPerWarp + r) * kDV + dv] << 16);
+        *reinterpret_cast<float4*>(vt + tc::swz_offset(kDV, dv, w * kRowsPerWarp)) = make_float4(x[0], x[1], x[2], x[3]);
+        *reinterpret_cast<float4*>(vt + tc::swz_offset(kDV, dv, w * kRowsPerWarp + 4)) =
+            make_float4(x[4], x[5], x[6], x[7]);
+      }
+      tc::fence_async_smem();
+      mbar_arrive(&bar_rdy[buf]);
+      // ---- the item's last chunk: U out of TMEM (warp w: lanes 32(w%4).., slot columns
+      // 64(w/4)..), D = e^Lam
+      if (ck.last) {
+        wait_or_abort(&bar_mma[buf], (n >> 1) & 1, abort_flag);
+        tc::tmem_fence_after();
+        const int64_t slot_base = ((int64_t)ck.pair * p.nseg + ck.seg + 1);
+        float* dst = p.ws_state + slot_base * kM * kDV;
+        const int dv = (w & 3) * 32 + lane;
+        const int c0 = (w >> 2) * 64;
+        float u[2][32];
+        tc::tmem_ld32(tc::tmem_addr(tb, (uint32_t)((w & 3) * 32), (uint32_t)c0), u[0]);
+        tc::tmem_ld32(tc::tmem_addr(tb, (uint32_t)((w & 3) * 32), (uint32_t)(c0 + 32)), u[1]);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) dst[(int64_t)(c0 + 32 * g + j) * kDV + dv] = u[g][j];
+        }
+        if (w == 0) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) p.ws_D[slot_base * kM + lane * 4 + e] = expf(lamS[e]);
+        }
+        tc::tmem_fence_before();
+        mbar_arrive(&bar_out);
+      }
+      cur = nxt;
+    }
+  } else if (warp == kIssuerWarp) {
+    // =========================================================================== MMA issuer
+    if (lane == 0) {
+      uint32_t n = 0, n_tma = 0, n_items = 0;
+      auto load_v = [&](const SumWalker& at, uint32_t j) {  // v tile of the walker's chunk, as chunk j
+        if (!at.valid(items)) return;
+        const Chunk c = at.get(p);
+        tc::mbar_arrive_expect_tx(&bar_tma[j & 1], kC * kDV * 2);
+        tc::tma_load_4d(sRawV + (j & 1) * (kC * kDV * 2), &maps.v, &bar_tma[j & 1], 0, c.h, c.c0, c.b);
+        ++n_tma;
+      };
+      {
+        SumWalker nx = wk;
+        load_v(nx, 0);
+        nx.next(p, items);
+        load_v(nx, 1);
+      }
+      auto kstep = [](int R, int j) -> uint64_t { return (uint64_t)(((j >> 2) * (R * 128) + (j & 3) * 32) >> 4); };
+      constexpr uint32_t kIdC = tc::idesc_tf32(kDV, kM, 0, 0);
+      const uint64_t dVt0 = tc::smem_desc(tc::smem_u32(sVt), 16, 1024), dWt0 = tc::smem_desc(tc::smem_u32(sWt), 16, 1024);
+      for (; wk.valid(items) && !*abort_flag; ++n, wk.next(p, items)) {
+        const Chunk ck = wk.get(p);
+        const int buf = n & 1;
+        wait_or_abort(&bar_rdy[buf], (n >> 1) & 1, abort_flag);  // tiles written, raw v consumed
+        {
+          SumWalker nx = wk;  // the raw v buffer is free again: the chunk two ahead
+          nx.next(p, items);
+          nx.next(p, items);
+          load_v(nx, n + 2);
+        }
+        // the accumulator of the item before has been read out
+        if (ck.first && n_items > 0) wait_or_abort(&bar_out, (n_items - 1) & 1, abort_flag);
+        tc::tmem_fence_after();
+        const uint64_t dVt = dVt0 + (uint64_t)((buf * 32768) >> 4), dWt = dWt0 + (uint64_t)((buf * 32768) >> 4);
+#pragma unroll
+        for (int j = 0; j < kC / 8; ++j)
+          tc::mma_tf32_ss(tb, dVt + kstep(kDV, j), dWt + kstep(kM, j), kIdC, (ck.first && j == 0) ? 0u : 1u);
+        tc::mma_commit(&bar_mma[buf]);
+        if (ck.last) ++n_items;
+      }
+      // nothing may still be running when the CTA releases its memory
+      tc::mma_commit(&bar_fin);
+      tc::mbar_wait(&bar_fin, 0);
+      for (uint32_t j = n; j < n_tma; ++j) tc::mbar_wait(&bar_tma[j & 1], (j >> 1) & 1);
+    }
+    __syncwarp();
+  }
+
+  tc::tmem_fence_before();
+  __syncthreads();
+  tc::tmem_fence_after();
+  if (warp == kIssuerWarp) tc::tmem_dealloc(tb, kSumTmemCols);
 }
 
 // Combines the segment summaries of each (b,h) into start states:
@@ -906,14 +1163,14 @@ WsLayout ws_layout(const rsm_forward_args& a, const Plan& pl) {
 template <int KP>
 cudaError_t launch_passes(const Maps& maps, const Params& p, const Plan& pl, int64_t pairs, int sms,
                           cudaStream_t stream) {
-  cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel<false, KP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       kSmemBytes);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(prefill_tc_kernel<true, KP>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  cudaError_t e =
+      cudaFuncSetAttribute(prefill_tc_kernel<KP>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
   if (pl.nseg > 1) {
+    e = cudaFuncSetAttribute(segment_summary_kernel<KP>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSumSmemBytes);
+    if (e != cudaSuccess) return e;
     const int items = (int)(pairs * (pl.nseg - 1));
-    prefill_tc_kernel<true, KP><<<std::min(items, sms), kThreads, kSmemBytes, stream>>>(maps, p);
+    segment_summary_kernel<KP><<<std::min(items, sms), kSumThreads, kSumSmemBytes, stream>>>(maps, p);
     e = cudaGetLastError();
     if (e == cudaSuccess) e = profile_mark(stream);
     if (e != cudaSuccess) return e;
@@ -924,7 +1181,7 @@ cudaError_t launch_passes(const Maps& maps, const Params& p, const Plan& pl, int
     if (e != cudaSuccess) return e;
   }
   const int64_t items = pairs * pl.nseg;
-  prefill_tc_kernel<false, KP><<<(unsigned)std::min<int64_t>(items, sms), kThreads, kSmemBytes, stream>>>(maps, p);
+  prefill_tc_kernel<KP><<<(unsigned)std::min<int64_t>(items, sms), kThreads, kSmemBytes, stream>>>(maps, p);
   e = cudaGetLastError();
   if (e == cudaSuccess) e = profile_mark(stream);
   return e;
