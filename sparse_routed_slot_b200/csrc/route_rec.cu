@@ -12,10 +12,12 @@
 //   Entries are in rank order (logit descending, slot ascending) except that logits agreeing in
 //   their upper 25 key bits may be listed in slot order; the set is always exact.
 //
-// Two threads per row. A warp takes 16 consecutive rows and copies them into shared memory with
-// asynchronous 16-byte copies (one 512-byte row per warp instruction), into one of two buffers per
-// warp, so the next 16 rows arrive while the current ones are ranked. Each thread of the pair
-// ranks half of the row's slots; the two sorted halves are merged through shuffles. Selection (router scores are monotone in the
+// Two threads per row. A warp takes 16 consecutive rows and copies them into its shared-memory
+// buffer with asynchronous 16-byte copies (one 512-byte row per warp instruction). One buffer per
+// warp keeps a CTA at 34 KB, so six CTAs (24 warps) share an SM and hide each other's copy
+// latency, which measured faster than double-buffering at half the warps. Each thread of the
+// pair ranks half of the row's slots; the two sorted halves are merged through shuffles.
+// Selection (router scores are monotone in the
 // logits, so TopK of the scores = TopK of the logits; -0 ties +0): each logit becomes a packed
 // 32-bit key, its order-preserving bit pattern with the low 7 bits replaced by (127 - slot), which
 // makes every key distinct and breaks ties to the lower slot. The top N (N = 16 or 32 >= K) keys
@@ -40,10 +42,16 @@ constexpr int kWarps = 4;              // warps per CTA
 constexpr int kThreads = kWarps * 32;
 constexpr int kRowsPerTask = 16;       // rows per warp task (two threads per row)
 constexpr int kBufBytes = kRowsPerTask * kRowFloats * 4;  // one warp's staged rows
-constexpr int kSmem = kWarps * 2 * kBufBytes;
+constexpr int kSmem = kWarps * kBufBytes;
 constexpr uint32_t kCoarse = ~0x7Fu;   // key bits above the slot field
 
-RSM_DEV uint32_t packed_key(float x, int slot) { return (order_key(x) & kCoarse) | (uint32_t)(127 - slot); }
+// The order key of common.cuh with -0 folded into +0 by an add (x + 0 is +0 for x = -0 and x
+// otherwise), which runs on the FMA pipe and leaves two logic operations for the ALU.
+RSM_DEV uint32_t packed_key(float x, int slot) {
+  const uint32_t b = __float_as_uint(x + 0.0f);
+  const uint32_t key = b ^ ((uint32_t)((int32_t)b >> 31) | 0x80000000u);
+  return (key & kCoarse) | (uint32_t)(127 - slot);
+}
 
 // Full bitonic sort of N keys, descending.
 template <int N>
@@ -88,7 +96,6 @@ RSM_DEV void cp_async16(void* smem, const void* gmem) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(tc::smem_u32(smem)), "l"(gmem) : "memory");
 }
 RSM_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-RSM_DEV void cp_async_wait_prev() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 RSM_DEV void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 struct Rows {
@@ -121,7 +128,7 @@ __global__ void __launch_bounds__(kThreads) route_rec_kernel(const Rows R) {
   const int64_t rows = R.B * R.H * R.T;
   const int64_t tasks = (rows + kRowsPerTask - 1) / kRowsPerTask;
   const int64_t stride = (int64_t)gridDim.x * kWarps;
-  unsigned char* wbuf = smem + warp * 2 * kBufBytes;
+  unsigned char* wbuf = smem + warp * kBufBytes;
   // input row index (in the [B, T, H] layout) of row p = 16*task + r of the [B, H, T] order:
   // one division per warp and task (lane 0), then a walk along the stream
   auto input_row = [&](int64_t task, int r) {
@@ -145,29 +152,27 @@ __global__ void __launch_bounds__(kThreads) route_rec_kernel(const Rows R) {
     }
     return (b * R.T + t) * R.H + h;
   };
-  // the warp copies the 16 rows of task `task` into buffer j&1 (16 bytes per lane per row)
-  auto stage = [&](int64_t task, uint32_t j) {
+  // the warp copies the 16 rows of task `task` into its buffer (16 bytes per lane per row)
+  auto stage = [&](int64_t task) {
     if (task < tasks) {
       const int64_t ir0 = input_row(task, lane & 15);  // lane r (r < 16) knows row r's index
       for (int r = 0; r < kRowsPerTask; ++r) {
         const int64_t irr = __shfl_sync(kFull, ir0, r);
         if (task * kRowsPerTask + r < rows)
-          cp_async16(wbuf + (j & 1) * kBufBytes + (r * kRowFloats + lane * 4) * 4, R.logits + irr * kRM + lane * 4);
+          cp_async16(wbuf + (r * kRowFloats + lane * 4) * 4, R.logits + irr * kRM + lane * 4);
       }
     }
     cp_async_commit();
   };
   const int64_t task0 = (int64_t)blockIdx.x * kWarps + warp;
-  stage(task0, 0);
-  uint32_t j = 0;
-  for (int64_t task = task0; task < tasks; task += stride, ++j) {
-    stage(task + stride, j + 1);  // the next rows arrive while these are ranked
-    cp_async_wait_prev();
+  for (int64_t task = task0; task < tasks; task += stride) {
+    stage(task);
+    cp_async_wait_all();
     __syncwarp();
     const int64_t p = task * kRowsPerTask + rl;
     const int64_t ir = input_row(task, rl);
     const bool live = p < rows;  // both lanes of a pair agree
-    const float* xr = reinterpret_cast<const float*>(wbuf + (j & 1) * kBufBytes) + rl * kRowFloats;
+    const float* xr = reinterpret_cast<const float*>(wbuf) + rl * kRowFloats;
     const float fh = (R.decay_slot || !live) ? 0.f : __ldg(R.f + ir);
 
     // ---- top N packed keys of this thread's half of the row, then of the whole row
@@ -234,9 +239,7 @@ __global__ void __launch_bounds__(kThreads) route_rec_kernel(const Rows R) {
 #pragma unroll
       for (int q = 0; q < KH; ++q) {
         const int r = half * KH + q;
-        uint32_t key = 0u;
-#pragma unroll
-        for (int rr = 0; rr < N; ++rr) key = rr == r ? top[rr] : key;
+        const uint32_t key = half ? top[KH + q] : top[q];
         lam[q] = 0.f;
         wv[q] = 0.f;
         if (r < K) {
@@ -269,7 +272,7 @@ __global__ void __launch_bounds__(kThreads) route_rec_kernel(const Rows R) {
       const int src = __ffs(pending) - 1;
       pending &= pending - 1u;
       const int r = src >> 1;
-      const float* xw = reinterpret_cast<const float*>(wbuf + (j & 1) * kBufBytes) + r * kRowFloats;
+      const float* xw = reinterpret_cast<const float*>(wbuf) + r * kRowFloats;
       float x4[kRM / 32];
 #pragma unroll
       for (int e = 0; e < kRM / 32; ++e) x4[e] = xw[lane * (kRM / 32) + e];
