@@ -894,6 +894,26 @@ __global__ void __launch_bounds__(kSumThreads, 1) segment_summary_kernel(const _
     const int w = warp;
     float* tab = sTab + w * kRowsPerWarp * kM;  // this warp's rows of the table
     float lamS[4] = {0.f, 0.f, 0.f, 0.f};      // Lam of the item's tokens after this chunk (slots 4l..)
+    // The table rows and the warp's token columns of both Wr^T buffers start at zero; afterwards each
+    // entry's owner clears what it wrote (sparse), so no chunk fills them densely.
+    uint32_t es2[RowInputs<KP>::kGroups], es1[RowInputs<KP>::kGroups];  // entry slots of chunks n-2, n-1
+#pragma unroll
+    for (int i = 0; i < kRowsPerWarp; ++i)
+      reinterpret_cast<float4*>(tab)[lane + 32 * i] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int slot = lane + 32 * e;
+        unsigned char* wt = sWt + b * 32768;
+        *reinterpret_cast<float4*>(wt + tc::swz_offset(kM, slot, w * kRowsPerWarp)) = make_float4(0.f, 0.f, 0.f, 0.f);
+        *reinterpret_cast<float4*>(wt + tc::swz_offset(kM, slot, w * kRowsPerWarp + 4)) =
+            make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+#pragma unroll
+    for (int g = 0; g < RowInputs<KP>::kGroups; ++g) es2[g] = es1[g] = 0u;
+    __syncwarp();
     RowInputs<KP> cur;
     if (wk.valid(items)) load_rows<true, KP>(p, wk.get(p), w, lane, cur);
     for (uint32_t n = 0; wk.valid(items); ++n, wk.next(p, items)) {
@@ -908,20 +928,18 @@ __global__ void __launch_bounds__(kSumThreads, 1) segment_summary_kernel(const _
         nx.next(p, items);
         if (nx.valid(items)) load_rows<true, KP>(p, nx.get(p), w, lane, nxt);
       }
-      // ---- the warp's rows of the table: lam at the selected entries, 0 elsewhere
-#pragma unroll
-      for (int i = 0; i < kRowsPerWarp; ++i)
-        reinterpret_cast<float4*>(tab)[lane + 32 * i] = make_float4(0.f, 0.f, 0.f, 0.f);
-      __syncwarp();
+      // ---- the warp's rows of the table (all zero): lam at the selected entries
       for_entries(cur, lane, K, nrows_w, [&](int r, int slot, float lam, float) { tab[r * kM + slot] = lam; });
       __syncwarp();
-      // ---- walk the rows from the last: each entry becomes the sum of lam below it in the warp
+      // ---- walk the rows from the last: each nonzero entry becomes the sum of lam below it in the
+      // warp, zeros stay (an entry with lam = 0 has w = k (1 - e^0) = 0, so its exponent is not used)
       float run[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int r = kRowsPerWarp - 1; r >= 0; --r) {
         float4* row = reinterpret_cast<float4*>(tab + r * kM) + lane;
         const float4 x = *row;
-        *row = make_float4(run[0], run[1], run[2], run[3]);
+        *row = make_float4(x.x != 0.f ? run[0] : 0.f, x.y != 0.f ? run[1] : 0.f, x.z != 0.f ? run[2] : 0.f,
+                           x.w != 0.f ? run[3] : 0.f);
         run[0] += x.x; run[1] += x.y; run[2] += x.z; run[3] += x.w;
       }
       reinterpret_cast<float4*>(sTot + (buf * kRWarps + w) * kM)[lane] = make_float4(run[0], run[1], run[2], run[3]);
@@ -946,18 +964,27 @@ __global__ void __launch_bounds__(kSumThreads, 1) segment_summary_kernel(const _
       if (n >= 2) wait_or_abort(&bar_mma[buf], ((n - 2) >> 1) & 1, abort_flag);
       unsigned char* wt = sWt + buf * 32768;
       unsigned char* vt = sVt + buf * 32768;
-      // the warp's token columns of Wr^T start at zero (rows slot = lane + 32e: 4-way stores)
+      // the entries of chunk n-2 leave this buffer (rows past a chunk's end hold slot 0, which
+      // clears a zero)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int slot = lane + 32 * e;
-        *reinterpret_cast<float4*>(wt + tc::swz_offset(kM, slot, w * kRowsPerWarp)) = make_float4(0.f, 0.f, 0.f, 0.f);
-        *reinterpret_cast<float4*>(wt + tc::swz_offset(kM, slot, w * kRowsPerWarp + 4)) =
-            make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int g = 0; g < RowInputs<KP>::kGroups; ++g) {
+        int r, j0;
+        entry_pos(lane, g, KP, r, j0);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if (r < kRowsPerWarp && j0 + e < K) {
+            const int slot = (int)((es2[g] >> (8 * e)) & 255u);
+            *reinterpret_cast<float*>(wt + tc::swz_offset(kM, slot, w * kRowsPerWarp + r)) = 0.f;
+          }
+        }
+        es2[g] = es1[g];
+        es1[g] = cur.es[g];
       }
       __syncwarp();
-      // ---- each entry's owner: Wr = w e^{exponent} (exponent <= 0)
+      // ---- each entry's owner: Wr = w e^{exponent} (exponent <= 0); its table entry back to zero
       for_entries(cur, lane, K, nrows_w, [&](int r, int slot, float, float wv) {
         const float x = tab[r * kM + slot] + sSuf[w * kM + slot];
+        tab[r * kM + slot] = 0.f;
         *reinterpret_cast<float*>(wt + tc::swz_offset(kM, slot, w * kRowsPerWarp + r)) = tc::to_tf32(wv * expf(x));
       });
       // ---- V^T of the warp's 8 tokens (value columns lane + 32e; rows past the sequence end are
