@@ -205,12 +205,8 @@ def oracle_sample(w, seconds_target: float = 3.0) -> dict:
 
 def _sources_digest() -> str:
     """sha256 of the CUDA sources (used to tell whether stored ncu counters are still current)."""
-    import glob
-    import hashlib
-    h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(ROOT, "sparse_routed_slot_b200", "csrc", "*"))):
-        h.update(open(f, "rb").read())
-    return h.hexdigest()
+    from sparse_routed_slot_b200.profile_case import sources_digest
+    return sources_digest()
 
 
 def stored_traffic(key: str):

@@ -161,6 +161,13 @@ __global__ void __launch_bounds__(kThreads) route_rec_kernel(const Rows R) {
         if (task * kRowsPerTask + r < rows)
           cp_async16(wbuf + (r * kRowFloats + lane * 4) * 4, R.logits + irr * kRM + lane * 4);
       }
+      // the k rows (gathered at the selected slots once the rows are ranked) start moving into L2:
+      // lane 2r + e fetches the e-th 128-byte half of row r's 256 bytes
+      {
+        const int64_t irk = __shfl_sync(kFull, ir0, lane >> 1);
+        if (task * kRowsPerTask + (lane >> 1) < rows)
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(R.k + irk * kRM + (lane & 1) * (kRM / 2)));
+      }
     }
     cp_async_commit();
   };

@@ -1,0 +1,147 @@
+"""Profiling case for ncu, and the summary of its DRAM counters.
+
+Run a fixed case through the public API (on cuda:0, synthetic inputs):
+
+    python -m sparse_routed_slot_b200.profile_case run [--workload long_ctx_bf16] [--forwards 2]
+                                                      [--decode-steps 2]
+
+Each forward makes rsm_forward_kernel_launches() launches (routing records, segment summary,
+segment scan, chunk scan on the tensor path); the decode steps use decode_256x16. Capture with
+
+    ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum \\
+        --clock-control none --csv --log-file traffic.csv \\
+        python -m sparse_routed_slot_b200.profile_case run
+
+then write the per-call DRAM bytes of the LAST forward and the LAST decode step, keyed to the
+current CUDA sources, to profiles/traffic.json:
+
+    python -m sparse_routed_slot_b200.profile_case traffic traffic.csv
+
+bench.py reads that file and reports its bytes only while the sources still hash the same.
+"""
+
+from __future__ import annotations
+
+import argparse
+import collections
+import csv
+import glob
+import hashlib
+import json
+import os
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+FORWARD_KERNELS = ("route_rec_kernel", "segment_summary_kernel", "segment_scan_kernel", "prefill_tc_kernel",
+                   "prefill_simt_kernel")
+DECODE_KERNELS = ("decode_kernel",)
+
+
+def sources_digest() -> str:
+    """sha256 of the CUDA sources (the key under which measured counters stay valid)."""
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "sparse_routed_slot_b200", "csrc", "*"))):
+        h.update(open(f, "rb").read())
+    return h.hexdigest()
+
+
+def run_case(workload: str, forwards: int, decode_steps: int) -> None:
+    import torch
+
+    import sparse_routed_slot_b200 as rsm
+    from sparse_routed_slot_b200.workloads import WORKLOADS, make_inputs
+
+    dev = torch.device("cuda", 0)
+    w = WORKLOADS[workload]
+    x = make_inputs(w.B, w.T, w.H, w.M, w.Dv, w.torch_dtype, w.decay, seed=w.seed, device=dev)
+    for _ in range(forwards):
+        out = rsm.forward(x["q"], x["k"], x["v"], x["logits"], x["f"], w.K)
+    torch.cuda.synchronize()
+    del x, out
+    if decode_steps > 0:
+        d = WORKLOADS["decode_256x16"]
+        state = torch.randn(d.B, d.H, d.M, d.Dv, device=dev)
+        y = make_inputs(decode_steps, d.B, d.H, d.M, d.Dv, d.torch_dtype, d.decay, seed=9, device=dev)
+        for i in range(decode_steps):
+            rsm.decode_step(y["q"][i], y["k"][i], y["v"][i], y["logits"][i], y["f"][i], d.K, state)
+        torch.cuda.synchronize()
+
+
+def read_ncu_csv(path: str):
+    """[(kernel name, {metric: value})] in launch order from an ncu --csv log."""
+    rows = list(csv.reader(open(path)))
+    hi = next(i for i, r in enumerate(rows) if "Kernel Name" in r and "Metric Name" in r)
+    h = rows[hi]
+    ki, ii, mi, vi = h.index("Kernel Name"), h.index("ID"), h.index("Metric Name"), h.index("Metric Value")
+    launches: "collections.OrderedDict[str, tuple]" = collections.OrderedDict()
+    for r in rows[hi + 1:]:
+        if len(r) <= vi:
+            continue
+        name, metrics = launches.setdefault(r[ii], (r[ki].split("(")[0], {}))
+        metrics[r[mi]] = float(r[vi].replace(",", ""))
+    return list(launches.values())
+
+
+def summarize_traffic(csv_path: str, workload: str, out_path: str) -> dict:
+    launches = read_ncu_csv(csv_path)
+
+    def last_group(kinds):
+        """The last maximal run of consecutive launches whose names match `kinds` (one call)."""
+        idx = [i for i, (n, _) in enumerate(launches) if any(k in n for k in kinds)]
+        if not idx:
+            return []
+        group = [idx[-1]]
+        for i in reversed(idx[:-1]):
+            if i != group[-1] - 1:
+                break
+            # a forward starts with the routing kernel: stop after including it
+            if "route_rec_kernel" in launches[group[-1]][0]:
+                break
+            group.append(i)
+        return [launches[i] for i in reversed(group)]
+
+    fwd = last_group(FORWARD_KERNELS)
+    dec = last_group(DECODE_KERNELS)[-1:]
+
+    def total(group):
+        return int(sum(m.get("dram__bytes_read.sum", 0) + m.get("dram__bytes_write.sum", 0) for _, m in group))
+
+    per_kernel = {}
+    for name, m in fwd + dec:
+        per_kernel[name] = {"read": int(m.get("dram__bytes_read.sum", 0)), "write": int(m.get("dram__bytes_write.sum", 0)),
+                            "ns": int(m.get("gpu__time_duration.sum", 0))}
+    d = {
+        "sources_sha256": sources_digest(),
+        "how": ("ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum --clock-control none "
+                f"python -m sparse_routed_slot_b200.profile_case run --workload {workload}; the last forward "
+                f"({len(fwd)} launches, summed) and the last decode step"),
+        "bytes": {f"{workload}/forward": total(fwd), "decode_256x16/step": total(dec)},
+        "per_kernel": per_kernel,
+    }
+    with open(out_path, "w") as fh:
+        json.dump(d, fh, indent=1)
+        fh.write("\n")
+    return d
+
+
+def main(argv=None) -> None:
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    sub = ap.add_subparsers(dest="cmd", required=True)
+    r = sub.add_parser("run")
+    r.add_argument("--workload", default="long_ctx_bf16")
+    r.add_argument("--forwards", type=int, default=2)
+    r.add_argument("--decode-steps", type=int, default=2)
+    t = sub.add_parser("traffic")
+    t.add_argument("csv")
+    t.add_argument("--workload", default="long_ctx_bf16")
+    t.add_argument("--out", default=os.path.join(ROOT, "profiles", "traffic.json"))
+    a = ap.parse_args(argv)
+    if a.cmd == "run":
+        run_case(a.workload, a.forwards, a.decode_steps)
+        print("ok")
+    else:
+        d = summarize_traffic(a.csv, a.workload, a.out)
+        print(json.dumps(d["bytes"]))
+
+
+if __name__ == "__main__":
+    main()
