@@ -45,8 +45,8 @@
 //              from TMEM, staged in halves through the A tile's memory and written by bulk tensor
 //              stores.
 // Per chunk the issuer runs S = Qh Wh^T (as soon as the row tiles are ready), then, once the
-// state is decayed and the V^T tile is there, O^T = H^T Qh^T and the carry H^T += V^T Wh, and
-// finally O^T += V^T A^T when the epilogue has masked S into A. An exact-path chunk carries into
+// state is decayed, O^T = H^T Qh^T, then (the V^T conversion overlaps the read) the carry
+// H^T += V^T Wh, and finally O^T += V^T A^T when the epilogue has masked S into A. An exact-path chunk carries into
 // U^T = V^T Wh_end (end-referenced weights) and the epilogue forms H = D H + U.
 // Every mbarrier is waited on by a role that the barrier's next phase depends on, so no waiter
 // can fall two phases behind (which a parity wait cannot tell from zero).
@@ -413,7 +413,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         // this warp's token columns of Wh^T start at zero
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int slot = lane * 4 + e;
+          const int slot = lane + 32 * e;  // 8 consecutive rows per 8 lanes: 4-way stores (no conflicts)
           *reinterpret_cast<float4*>(sWt + tc::swz_offset(kM, slot, w * kRowsPerWarp)) = make_float4(0.f, 0.f, 0.f, 0.f);
           *reinterpret_cast<float4*>(sWt + tc::swz_offset(kM, slot, w * kRowsPerWarp + 4)) =
               make_float4(0.f, 0.f, 0.f, 0.f);
@@ -470,7 +470,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         }
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int slot = lane * 4 + e;
+          const int slot = lane + 32 * e;  // 8 consecutive rows per 8 lanes: 4-way stores (no conflicts)
           *reinterpret_cast<float4*>(sWt + tc::swz_offset(kM, slot, w * kRowsPerWarp)) = make_float4(0.f, 0.f, 0.f, 0.f);
           *reinterpret_cast<float4*>(sWt + tc::swz_offset(kM, slot, w * kRowsPerWarp + 4)) =
               make_float4(0.f, 0.f, 0.f, 0.f);
@@ -590,6 +590,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         tc::mma_commit(&bar_s);  // every main-pass chunk: tells the epilogue the chunk is ready
         wait_or_abort(&bar_h, n & 1, abort_flag);  // state ready
         if (n >= 2) wait_or_abort(&bar_of[n & 1], ((n - 2) >> 1) & 1, abort_flag);  // O buffer free
+        tc::tmem_fence_after();
+        mma_read(ob);  // needs no V^T: the conversion overlaps it
         wait_or_abort(&bar_vt, n & 1, abort_flag);  // V^T written
         tc::tmem_fence_after();
         {
@@ -599,7 +601,6 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
           nx.next(p, items);
           load_v(nx, n + 2);
         }
-        mma_read(ob);
         mma_carry(fast ? kColH : kColU, fast);
         tc::mma_commit(&bar_t);
         wait_or_abort(&bar_a, n & 1, abort_flag);
