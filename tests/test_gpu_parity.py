@@ -276,6 +276,43 @@ def test_tensor_segments_with_aliased_state(rsm):
     assert rel(st.cpu().numpy(), r["HT"]) <= TOL_BF16
 
 
+def test_tensor_segments_unselected_slots_keep_bits(rsm):
+    """A long sequence split into segments: slots that no token selects pass the initial state
+    through every segment summary (D = 1, U = 0) and the scan bit for bit."""
+    B, T, H, M, K, Dv = 1, 4096 + 77, 2, 128, 16, 128
+    x = make_inputs(B, T, H, M, Dv, torch.bfloat16, "head", seed=19, device="cuda", h0=True)
+    x["logits"][..., M // 2:] = -100.0
+    out = rsm.forward(x["q"], x["k"], x["v"], x["logits"], x["f"], K, x["H0"], path="tensor")
+    torch.cuda.synchronize()
+    a = out["HT"][:, :, M // 2:].cpu().numpy().view(np.uint32)
+    b = x["H0"][:, :, M // 2:].cpu().numpy().view(np.uint32)
+    assert np.array_equal(a, b)
+
+
+def test_tensor_segments_window_limit(rsm):
+    """The window-limit case (K=1, one-hot cyclic router, f = -1e4) over a sequence long enough to
+    be split into segments: the segment summaries see decays of e^-10000 and still give the window
+    form o_t = sum_{s=t-M+1..t} q_{t, s mod M} v_s."""
+    B, T, H, M, Dv = 1, 2000, 2, 128, 128
+    dev = torch.device("cuda")
+    g = torch.Generator(device=dev).manual_seed(6)
+    q = torch.randn(B, T, H, M, generator=g, device=dev).bfloat16()
+    v = torch.randn(B, T, H, Dv, generator=g, device=dev).bfloat16()
+    k = torch.ones(B, T, H, M, device=dev).bfloat16()
+    logits = torch.zeros(B, T, H, M, device=dev)
+    t = torch.arange(T, device=dev)
+    logits[:, t, :, t % M] = 10.0
+    f = torch.full((B, T, H), -1e4, device=dev)
+    out = rsm.forward(q, k, v, logits, f, 1, path="tensor")
+    torch.cuda.synchronize()
+    from oracle import brute
+    qc, vc = q.float().cpu().numpy(), v.float().cpu().numpy()
+    for h in range(H):
+        ow, HTw = brute.window_form(qc[0, :, h], vc[0, :, h], M)
+        assert rel(out["o"][0, :, h].cpu().numpy(), ow) <= TOL_FP32
+        assert rel(out["HT"][0, h].cpu().numpy(), HTw) <= TOL_FP32
+
+
 def test_tensor_mixed_fast_and_exact_chunks(rsm):
     """Some tokens forget almost everything (f = -1e4): their chunks take the exact path while
     the others take the tensor-core path; results still match the oracle."""
