@@ -85,15 +85,17 @@ constexpr int kColH = 0, kColHr = 128, kColO = 256, kColS = 384, kColU = 384, kT
 
 // Dynamic shared memory (offsets from a 1024-byte aligned base). Operand tiles are K-major in the
 // swizzled format of tc.cuh; Wh^T and V^T are stored transposed because they are contracted over
-// tokens (a tf32 operand cannot be MN-major in this swizzle).
-constexpr int kOffQ = 0;                   // Qh   [64 t][128 slot]   (A of S, B of the read)
-constexpr int kOffW = kOffQ + 32768;       // Wh   [64 s][128 slot]   (B of S); exact path: dense g
+// tokens and every operand tile here is K-major. Qh is double-buffered (chunk n&1), so the row
+// workers can build the next chunk's Qh while this chunk's read still uses its own. The Wh tile
+// also holds the chunk's decay table before the walk turns it into G (in place) and the post-pass
+// into Wh; an exact-path chunk keeps lam and then the dense g there (plain [64][128] layout).
+constexpr int kOffQ = 0;                   // Qh   [2][64 t][128 slot] (A of S, B of the read)
+constexpr int kOffW = kOffQ + 2 * 32768;   // Wh   [64 s][128 slot]   (B of S); decay table before
 constexpr int kOffWt = kOffW + 32768;      // Wh^T [128 slot][64 s]   (B of the carry)
 constexpr int kOffVt = kOffWt + 32768;     // V^T  [128 dv][64 s]     (A of carry and A.V)
 constexpr int kOffA = kOffVt + 32768;      // A    [64 t][64 s]       (B of A.V)
 constexpr int kOffRawV = kOffA + 16384;    // v tiles from TMA, [2][64][128] bf16
-constexpr int kOffTab = kOffRawV + 32768;  // decay table [64 t][128 slot] fp32 (exact path: lam)
-constexpr int kOffTot = kOffTab + 32768;   // per-warp slot products (sums), [2][8][128]
+constexpr int kOffTot = kOffRawV + 32768;  // per-warp slot products (sums), [2][8][128]
 constexpr int kOffSmall = kOffTot + 2 * kRWarps * kM * 4;
 // D[2][M], fast[2]
 constexpr int kSmallBytes = 2 * kM * 4 + 16;
@@ -283,7 +285,6 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
   unsigned char* sVt = sm + kOffVt;
   unsigned char* sA = sm + kOffA;
   unsigned char* sRawV = sm + kOffRawV;
-  float* sTab = reinterpret_cast<float*>(sm + kOffTab);
   float* sTot = reinterpret_cast<float*>(sm + kOffTot);
   float* sDc = reinterpret_cast<float*>(sm + kOffSmall);    // [2][M]
   int* sFast = reinterpret_cast<int*>(sDc + 2 * kM);         // [2]
@@ -338,7 +339,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     // =========================================================================== row workers
     const int w = warp;
     const int RB = p.rec_bytes;
-    float* tab = sTab + w * kRowsPerWarp * kM;  // this warp's rows of the decay table
+    // the decay table lives in the Wh tile: row t = w*8 + r of the warp, 4 slots per lane
+    auto tab_row = [&](int r) -> float4* {
+      return reinterpret_cast<float4*>(sW + tc::swz_offset(kC, w * kRowsPerWarp + r, lane * 4));
+    };
 
     RowInputs<KP> cur;
     if (wk.valid(items)) load_rows<false, KP>(p, wk.get(p), w, lane, cur);
@@ -346,20 +350,22 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       const Chunk ck = wk.get(p);
       const int buf = n & 1;
       const int nrows_w = ck.nrows - w * kRowsPerWarp;  // rows of this warp inside the chunk
+      // ---- the previous chunk's S has read the Wh tile (and, issued before it, the read of the
+      // chunk before that has read this chunk's Qh buffer)
+      if (n > 0) wait_or_abort(&bar_s, (n - 1) & 1, abort_flag);
       // ---- this warp's rows of the decay table: 1 everywhere, -a at the selected entries
 #pragma unroll
-      for (int i = 0; i < kRowsPerWarp; ++i)
-        reinterpret_cast<float4*>(tab)[lane + 32 * i] = make_float4(1.f, 1.f, 1.f, 1.f);
+      for (int r = 0; r < kRowsPerWarp; ++r) *tab_row(r) = make_float4(1.f, 1.f, 1.f, 1.f);
       __syncwarp();
       for_entries(cur, lane, K, nrows_w, [&](int r, int slot, float lam, float) {
-        tab[r * kM + slot] = -expf(lam);
+        *reinterpret_cast<float*>(sW + tc::swz_offset(kC, w * kRowsPerWarp + r, slot)) = -expf(lam);
       });
       __syncwarp();
       // ---- product of the decays over the warp's rows, per slot
       float P[4] = {1.f, 1.f, 1.f, 1.f};
 #pragma unroll
       for (int r = 0; r < kRowsPerWarp; ++r) {
-        const float4 a4 = reinterpret_cast<const float4*>(tab + r * kM)[lane];
+        const float4 a4 = *tab_row(r);
         P[0] *= fabsf(a4.x); P[1] *= fabsf(a4.y); P[2] *= fabsf(a4.z); P[3] *= fabsf(a4.w);
       }
       reinterpret_cast<float4*>(sTot + (buf * kRWarps + w) * kM)[lane] = make_float4(P[0], P[1], P[2], P[3]);
@@ -380,24 +386,26 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
 #pragma unroll
       for (int e = 0; e < 4; ++e) ok &= gend[e] >= kDMin;
       const bool fast = __all_sync(kFull, ok);
-      // ---- the previous chunk's read and carry have consumed the operand tiles (and the epilogue
-      // has decayed the state of the chunk before it, whose decay buffer this chunk reuses)
-      if (n > 0) wait_or_abort(&bar_t, (n - 1) & 1, abort_flag);
-      if (w == 0) {
+      // the chunk's decays and path, once the epilogue has used those of the chunk before the
+      // previous one (its decay of the state precedes the previous chunk's read, and so the carry)
+      auto put_decays = [&]() {
+        if (w == 0) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int slot = lane * 4 + e;
-          sDc[buf * kM + slot] = gend[e];
+          for (int e = 0; e < 4; ++e) {
+            const int slot = lane * 4 + e;
+            sDc[buf * kM + slot] = gend[e];
+          }
+          if (lane == 0) sFast[buf] = fast;
         }
-        if (lane == 0) sFast[buf] = fast;
-      }
+      };
+      unsigned char* sQb = sQ + buf * 32768;  // this chunk's Qh buffer
       if (fast) {
         // ---- walk the warp's rows: Qh = q G, and G at the selected entries (0 elsewhere)
         float G[4] = {off[0], off[1], off[2], off[3]};
 #pragma unroll
         for (int r = 0; r < kRowsPerWarp; ++r) {
           const int t = w * kRowsPerWarp + r;
-          const float4 a4 = reinterpret_cast<const float4*>(tab + r * kM)[lane];
+          const float4 a4 = *tab_row(r);
           const float av[4] = {a4.x, a4.y, a4.z, a4.w};
           const float4 q4 = bf16x4_to_f32(cur.q[r]);
           float qh[4], gw[4];
@@ -407,9 +415,13 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             qh[e] = tc::to_tf32(fget(q4, e) * G[e]);
             gw[e] = sign_set(av[e]) ? G[e] : 0.f;
           }
-          *reinterpret_cast<float4*>(sQ + tc::swz_offset(kC, t, lane * 4)) = make_float4(qh[0], qh[1], qh[2], qh[3]);
+          *reinterpret_cast<float4*>(sQb + tc::swz_offset(kC, t, lane * 4)) = make_float4(qh[0], qh[1], qh[2], qh[3]);
           *reinterpret_cast<float4*>(sW + tc::swz_offset(kC, t, lane * 4)) = make_float4(gw[0], gw[1], gw[2], gw[3]);
         }
+        // the previous carry has read Wh^T (and the epilogue has used the decays this chunk's
+        // buffer held before)
+        if (n > 0) wait_or_abort(&bar_t, (n - 1) & 1, abort_flag);
+        put_decays();
         // this warp's token columns of Wh^T start at zero
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -436,6 +448,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         // A.V of the chunk before is done with A, and the epilogue has staged that chunk's output
         // through the A tile's memory
         if (n > 0) wait_or_abort(&bar_of[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag);
+        put_decays();
+        // lam, then the dense g, in the Wh tile's memory in plain [64][128] layout (this warp: rows
+        // 8w..8w+7); every row worker is past the swizzled decay table first
+        float* tab = reinterpret_cast<float*>(sW) + w * kRowsPerWarp * kM;
         bar_rows();  // every row worker is past the product totals
 #pragma unroll
         for (int i = 0; i < kRowsPerWarp; ++i)
@@ -464,7 +480,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
           g[0] += l4.x; g[1] += l4.y; g[2] += l4.z; g[3] += l4.w;
           reinterpret_cast<float4*>(dg + t * kM)[lane] = make_float4(g[0], g[1], g[2], g[3]);
           const float4 q4 = bf16x4_to_f32(cur.q[r]);
-          *reinterpret_cast<float4*>(sQ + tc::swz_offset(kC, t, lane * 4)) =
+          *reinterpret_cast<float4*>(sQb + tc::swz_offset(kC, t, lane * 4)) =
               make_float4(tc::to_tf32(q4.x * expf(g[0])), tc::to_tf32(q4.y * expf(g[1])),
                           tc::to_tf32(q4.z * expf(g[2])), tc::to_tf32(q4.w * expf(g[3])));
         }
@@ -556,15 +572,15 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       auto kstep = [](int R, int j) -> uint64_t { return (uint64_t)(((j >> 2) * (R * 128) + (j & 3) * 32) >> 4); };
       constexpr uint32_t kIdS = tc::idesc_tf32(64, kC, 0, 0), kIdO = tc::idesc_tf32(kDV, kC, 0, 0),
                          kIdC = tc::idesc_tf32(kDV, kM, 0, 0);
-      auto mma_s = [&]() {  // S = Qh Wh^T
+      auto mma_s = [&](uint64_t dQn) {  // S = Qh Wh^T
 #pragma unroll
         for (int j = 0; j < kM / 8; ++j)
-          tc::mma_tf32_ss(tb + kColS, dQ + kstep(kC, j), dW + kstep(kC, j), kIdS, j > 0);
+          tc::mma_tf32_ss(tb + kColS, dQn + kstep(kC, j), dW + kstep(kC, j), kIdS, j > 0);
       };
-      auto mma_read = [&](uint32_t ob) {  // O^T = H^T Qh^T (state read from TMEM)
+      auto mma_read = [&](uint32_t ob, uint64_t dQn) {  // O^T = H^T Qh^T (state read from TMEM)
 #pragma unroll
         for (int j = 0; j < kM / 8; ++j)
-          tc::mma_tf32_ts(tb + kColO + ob, tb + kColHr + 8 * j, dQ + kstep(kC, j), kIdO, j > 0);
+          tc::mma_tf32_ts(tb + kColO + ob, tb + kColHr + 8 * j, dQn + kstep(kC, j), kIdO, j > 0);
       };
       auto mma_carry = [&](uint32_t col, bool acc) {  // H^T += V^T Wh, or U^T = V^T Wh
 #pragma unroll
@@ -586,12 +602,13 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
           wait_or_abort(&bar_h, n & 1, abort_flag);
           tc::tmem_fence_after();
         }
-        if (fast) mma_s();
+        const uint64_t dQn = dQ + (uint64_t)(((n & 1) * 32768) >> 4);  // this chunk's Qh buffer
+        if (fast) mma_s(dQn);
         tc::mma_commit(&bar_s);  // every main-pass chunk: tells the epilogue the chunk is ready
         wait_or_abort(&bar_h, n & 1, abort_flag);  // state ready
         if (n >= 2) wait_or_abort(&bar_of[n & 1], ((n - 2) >> 1) & 1, abort_flag);  // O buffer free
         tc::tmem_fence_after();
-        mma_read(ob);  // needs no V^T: the conversion overlaps it
+        mma_read(ob, dQn);  // needs no V^T: the conversion overlaps it
         wait_or_abort(&bar_vt, n & 1, abort_flag);  // V^T written
         tc::tmem_fence_after();
         {
