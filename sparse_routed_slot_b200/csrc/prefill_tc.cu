@@ -35,11 +35,11 @@
 //              along its rows, and exchanges the per-warp products for the in-chunk prefix at its
 //              first row. It then walks its rows: the running product G gives Qh = q G and, at
 //              the selected entries, G itself, from which each entry's owner forms Wh = w / G in
-//              the Wh and Wh^T tiles. q and the records of the next chunk are loaded while this one
+//              the Wh and Wh^T tiles. Once a chunk's tiles are handed over, the row workers convert
+//              its v tile into V^T. q and the records of the next chunk are loaded while this one
 //              is processed.
 //   warp 8     MMA issuer (one thread): v tile loads (two chunks ahead) and the tcgen05.mma of
 //              every chunk, as soon as their operands are ready.
-//              Once a chunk's tiles are handed over, they also convert its v tile into V^T.
 //   warps 9-12 epilogue (one per TMEM lane quarter): S -> A masking, the decay of the state after
 //              the carry (and the state in and out at item boundaries), the output of the chunk
 //              from TMEM, staged in halves through the A tile's memory and written by bulk tensor
@@ -820,7 +820,7 @@ constexpr int kSumSmemBytes = kSumOffSuf + kRWarps * kM * 4 + 1024;
 constexpr int kSumTmemCols = 128;
 static_assert(kSumSmemBytes <= 232448, "shared memory budget");
 
-// The summary pass visits item (pair, seg) = blockIdx.x + j*gridDim.x, seg < nseg - 1, and the
+// The summary kernel visits item (pair, seg) = blockIdx.x + j*gridDim.x, seg < nseg - 1, and the
 // item's chunks from the last to the first; first/last refer to that visiting order.
 struct SumWalker {
   int item, pair, seg, b, h, t0, nch, i;

@@ -249,8 +249,8 @@ def test_workload_parity(rsm, name):
 @pytest.mark.parametrize("T", [1000, 4096 + 77])
 @pytest.mark.parametrize("decay", ["head", "slot"])
 def test_tensor_segments_match_oracle(rsm, T, decay):
-    """Few (b,h) streams and a long sequence: the sequence is split into segments (summary pass,
-    scan of segment states, main pass). Random initial state."""
+    """Few (b,h) streams and a long sequence: the sequence is split into segments (segment
+    summaries, scan of segment states, chunk scan). Random initial state."""
     B, H, M, K, Dv = 1, 2, 128, 16, 128
     x = make_inputs(B, T, H, M, Dv, torch.bfloat16, decay, seed=T, device="cuda", h0=True)
     out = rsm.forward(x["q"], x["k"], x["v"], x["logits"], x["f"], K, x["H0"], routing=True, path="tensor")
