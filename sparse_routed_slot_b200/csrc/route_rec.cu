@@ -10,7 +10,8 @@
 //     float  lam[KP]    lam = sigmoid(logit[slot]) * f, the log of the slot's decay (<= 0)
 //     float  w[KP]      w = k[slot] * (1 - e^lam), the slot's write weight
 //   Entries are in rank order (logit descending, slot ascending) except that logits agreeing in
-//   their upper 25 key bits may be listed in slot order; the set is always exact.
+//   their upper 25 key bits may be listed in slot order; when no ranked output is requested and
+//   K equals KP, they come in no particular order. The set is always exact.
 //
 // Two threads per row. A warp takes 16 consecutive rows and copies them into its shared-memory
 // buffer with asynchronous 16-byte copies (one 512-byte row per warp instruction). One buffer per
@@ -85,8 +86,8 @@ RSM_DEV void sort_desc(uint32_t (&a)[N]) {
 }
 
 // top <- the N largest of top and g (both sorted descending); the largest dropped key is folded
-// into `dropped`.
-template <int N>
+// into `dropped`. Without SORT the N keys are left as a bitonic sequence (the right set, unordered).
+template <int N, bool SORT = true>
 RSM_DEV void merge_top(uint32_t (&top)[N], const uint32_t (&g)[N], uint32_t& dropped) {
 #pragma unroll
   for (int i = 0; i < N; ++i) {
@@ -94,12 +95,14 @@ RSM_DEV void merge_top(uint32_t (&top)[N], const uint32_t (&g)[N], uint32_t& dro
     top[i] = max(a, b);
     dropped = max(dropped, min(a, b));
   }
+  if constexpr (SORT) {
 #pragma unroll
-  for (int j = N >> 1; j > 0; j >>= 1) {
+    for (int j = N >> 1; j > 0; j >>= 1) {
 #pragma unroll
-    for (int i = 0; i < N; ++i) {
-      const int l = i ^ j;
-      if (l > i) cas_desc(top[i], top[l]);
+      for (int i = 0; i < N; ++i) {
+        const int l = i ^ j;
+        if (l > i) cas_desc(top[i], top[l]);
+      }
     }
   }
 }
@@ -219,7 +222,12 @@ __global__ void __launch_bounds__(kThreads) route_rec_kernel(const Rows R) {
     }
 #pragma unroll
     for (int i = 0; i < N; ++i) g[i] = __shfl_xor_sync(kFull, top[i], 1);  // the partner's half
-    merge_top<N>(top, g, dropped);  // both lanes now hold the row's top N
+    // both lanes now hold the row's top N; sorted only where the order is used (ranked outputs, or
+    // K < N, where the first K must be the K largest)
+    const bool ranked = R.idx_out || R.score_out;
+    const bool sorted = ranked || K < N;
+    if (sorted) merge_top<N, true>(top, g, dropped);
+    else merge_top<N, false>(top, g, dropped);  // lane 2r+1 holds lane 2r's keys in reverse
     dropped = max(dropped, __shfl_xor_sync(kFull, dropped, 1));
     if (VALIDATE && live) {
       if (R.decay_slot) {
@@ -242,7 +250,6 @@ __global__ void __launch_bounds__(kThreads) route_rec_kernel(const Rows R) {
       next = max(next, r < K ? 0u : top[r]);
       if (r + 1 < N && r + 1 < K) near_tie |= ((top[r] ^ top[r + 1]) & kCoarse) == 0u;
     }
-    const bool ranked = R.idx_out || R.score_out;
     const bool exact = ((next ^ kth) & kCoarse) == 0u || (ranked && near_tie);
     unsigned char* rp = R.rec + p * (int64_t)(9 * KP);
     int32_t* io = R.idx_out ? R.idx_out + ir * K : nullptr;
@@ -258,7 +265,9 @@ __global__ void __launch_bounds__(kThreads) route_rec_kernel(const Rows R) {
 #pragma unroll
       for (int q = 0; q < KH; ++q) {
         const int r = half * KH + q;
-        const uint32_t key = half ? top[KH + q] : top[q];
+        // sorted: lane `half` takes rank positions half*KH + q; unsorted, the partner's array is
+        // this lane's reversed, so each lane takes its own first half
+        const uint32_t key = (sorted && half) ? top[KH + q] : top[q];
         lam[q] = 0.f;
         wv[q] = 0.f;
         if (r < K) {
