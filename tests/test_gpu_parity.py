@@ -241,6 +241,11 @@ def test_workload_parity(rsm, name):
     eo, eh = rel(out["o"].cpu().numpy(), r["o"]), rel(out["HT"].cpu().numpy(), r["HT"])
     print(f"{name}: o {eo:.3e} H_T {eh:.3e}")
     assert eo <= tol and eh <= tol
+    # the benchmark's call: no routing outputs (the routing records then hold the selected set
+    # without ranking it)
+    out2 = rsm.forward(x["q"], x["k"], x["v"], x["logits"], x["f"], w.K)
+    torch.cuda.synchronize()
+    assert rel(out2["o"].cpu().numpy(), r["o"]) <= tol and rel(out2["HT"].cpu().numpy(), r["HT"]) <= tol
 
 
 # ------------------------------------------------------------------------------------ tensor path
