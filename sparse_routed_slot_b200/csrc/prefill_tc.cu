@@ -801,15 +801,19 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
 // segment's last to its first, so the exponent of a token is the running sum of the lam of the
 // tokens after it.
 //
-// Warp roles (one CTA per segment at a time, 9 warps):
+// Warp roles (one CTA per segment at a time, 13 warps):
 //   warps 0-7  row workers; warp w owns tokens 8w..8w+7 of the chunk, lane l slots 4l..4l+3 of
 //              the lam table. Per chunk: scatter the rows' lam into the table, walk the rows from
 //              the last to the first (exclusive in-warp suffix sums in place), exchange the warp
-//              totals, write Wr^T at the selected entries, convert the warp's tokens of the v
-//              tile into V^T; at the segment's end read U out of TMEM and write U and D.
+//              totals, write Wr^T at the selected entries; at the segment's end read U out of TMEM
+//              and write U and D.
 //   warp 8     MMA issuer (one thread): the v tile loads (two chunks ahead) and the 8 MMAs of
 //              each chunk, U^T += V^T Wr (M = value columns, N = slots, K = tokens).
-constexpr int kSumThreads = (kRWarps + 1) * 32;
+//   warps 9-12 converters: each chunk's v tile into V^T (warp c: tokens 16c..16c+15), beside the
+//              row workers' chain instead of at its end.
+constexpr int kSumConvWarps = 4;
+constexpr int kSumConvThreads = kSumConvWarps * 32;
+constexpr int kSumThreads = (kRWarps + 1 + kSumConvWarps) * 32;
 constexpr int kSumOffRawV = 0;                       // v tiles from TMA, [2][64 t][128 dv] bf16
 constexpr int kSumOffVt = kSumOffRawV + 32768;       // V^T  [2][128 dv][64 t] (A)
 constexpr int kSumOffWt = kSumOffVt + 2 * 32768;     // Wr^T [2][128 slot][64 t] (B)
@@ -873,7 +877,8 @@ __global__ void __launch_bounds__(kSumThreads, 1) segment_summary_kernel(const _
   float* sTot = reinterpret_cast<float*>(sm + kSumOffTot);
   float* sSuf = reinterpret_cast<float*>(sm + kSumOffSuf);
 
-  __shared__ __align__(8) uint64_t bar_rdy[2],  // tiles of chunk n in buffer n&1 written (row threads)
+  __shared__ __align__(8) uint64_t bar_rdy[2],  // Wr^T of chunk n in buffer n&1 written (row threads)
+      bar_vt[2],                                 // V^T of chunk n in buffer n&1 written  (converters)
       bar_tma[2],                                // raw v tile of chunk n landed          (TMA)
       bar_mma[2],                                // MMAs of chunk n done, buffer n&1 free (MMA commit)
       bar_out,                                   // U of an item read out of TMEM         (row threads)
@@ -889,6 +894,7 @@ __global__ void __launch_bounds__(kSumThreads, 1) segment_summary_kernel(const _
   if (tid == 0) {
     for (int b = 0; b < 2; ++b) {
       tc::mbar_init(&bar_rdy[b], kRThreads);
+      tc::mbar_init(&bar_vt[b], kSumConvThreads);
       tc::mbar_init(&bar_tma[b], 1);
       tc::mbar_init(&bar_mma[b], 1);
     }
@@ -978,10 +984,9 @@ __global__ void __launch_bounds__(kSumThreads, 1) segment_summary_kernel(const _
 #pragma unroll
       for (int e = 0; e < 4; ++e) lamS[e] += tot[e];
       reinterpret_cast<float4*>(sSuf + w * kM)[lane] = make_float4(suf[0], suf[1], suf[2], suf[3]);
-      // ---- tile buffer `buf` is free once the MMAs of chunk n-2 are done
+      // ---- Wr^T buffer `buf` is free once the MMAs of chunk n-2 are done
       if (n >= 2) wait_or_abort(&bar_mma[buf], ((n - 2) >> 1) & 1, abort_flag);
       unsigned char* wt = sWt + buf * 32768;
-      unsigned char* vt = sVt + buf * 32768;
       // the entries of chunk n-2 leave this buffer (rows past a chunk's end hold slot 0, which
       // clears a zero)
 #pragma unroll
@@ -1005,21 +1010,6 @@ __global__ void __launch_bounds__(kSumThreads, 1) segment_summary_kernel(const _
         tab[r * kM + slot] = 0.f;
         *reinterpret_cast<float*>(wt + tc::swz_offset(kM, slot, w * kRowsPerWarp + r)) = tc::to_tf32(wv * expf(x));
       });
-      // ---- V^T of the warp's 8 tokens (value columns lane + 32e; rows past the sequence end are
-      // zero in the tile)
-      wait_or_abort(&bar_tma[buf], (n >> 1) & 1, abort_flag);
-      const uint16_t* raw = reinterpret_cast<const uint16_t*>(sRawV + buf * (kC * kDV * 2));
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int dv = lane + 32 * e;
-        float x[kRowsPerWarp];
-#pragma unroll
-        for (int r = 0; r < kRowsPerWarp; ++r)
-          x[r] = __uint_as_float((uint32_t)raw[(w * kRowsPerWarp + r) * kDV + dv] << 16);
-        *reinterpret_cast<float4*>(vt + tc::swz_offset(kDV, dv, w * kRowsPerWarp)) = make_float4(x[0], x[1], x[2], x[3]);
-        *reinterpret_cast<float4*>(vt + tc::swz_offset(kDV, dv, w * kRowsPerWarp + 4)) =
-            make_float4(x[4], x[5], x[6], x[7]);
-      }
       tc::fence_async_smem();
       mbar_arrive(&bar_rdy[buf]);
       // ---- the item's last chunk: U out of TMEM (warp w: lanes 32(w%4).., slot columns
@@ -1072,7 +1062,8 @@ __global__ void __launch_bounds__(kSumThreads, 1) segment_summary_kernel(const _
       for (; wk.valid(items) && !*abort_flag; ++n, wk.next(p, items)) {
         const Chunk ck = wk.get(p);
         const int buf = n & 1;
-        wait_or_abort(&bar_rdy[buf], (n >> 1) & 1, abort_flag);  // tiles written, raw v consumed
+        wait_or_abort(&bar_rdy[buf], (n >> 1) & 1, abort_flag);  // Wr^T written
+        wait_or_abort(&bar_vt[buf], (n >> 1) & 1, abort_flag);   // V^T written, raw v consumed
         {
           SumWalker nx = wk;  // the raw v buffer is free again: the chunk two ahead
           nx.next(p, items);
@@ -1095,6 +1086,32 @@ __global__ void __launch_bounds__(kSumThreads, 1) segment_summary_kernel(const _
       for (uint32_t j = n; j < n_tma; ++j) tc::mbar_wait(&bar_tma[j & 1], (j >> 1) & 1);
     }
     __syncwarp();
+  } else {
+    // =========================================================================== converters
+    const int c = warp - (kRWarps + 1);  // tokens 16c..16c+15 of each chunk
+    for (uint32_t n = 0; wk.valid(items) && !*abort_flag; ++n, wk.next(p, items)) {
+      const int buf = n & 1;
+      if (n >= 2) wait_or_abort(&bar_mma[buf], ((n - 2) >> 1) & 1, abort_flag);  // V^T buffer free
+      wait_or_abort(&bar_tma[buf], (n >> 1) & 1, abort_flag);                    // v tile landed
+      const uint16_t* raw = reinterpret_cast<const uint16_t*>(sRawV + buf * (kC * kDV * 2));
+      unsigned char* vt = sVt + buf * 32768;
+      // value columns lane + 32e (8 consecutive rows per 8 lanes: 4-way stores); rows past the
+      // sequence end are zero in the tile
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int dv = lane + 32 * e;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const int t0 = 16 * c + 4 * g;
+          float x[4];
+#pragma unroll
+          for (int r = 0; r < 4; ++r) x[r] = __uint_as_float((uint32_t)raw[(t0 + r) * kDV + dv] << 16);
+          *reinterpret_cast<float4*>(vt + tc::swz_offset(kDV, dv, t0)) = make_float4(x[0], x[1], x[2], x[3]);
+        }
+      }
+      tc::fence_async_smem();
+      mbar_arrive(&bar_vt[buf]);
+    }
   }
 
   tc::tmem_fence_before();
