@@ -4,8 +4,14 @@
 
 A step is one chunked prefill (rsm_forward) of the chosen workload, inputs resident in HBM
 (default: the 32K-token long-context prefill, B=1 T=32768 H=16 M=128 K=16 Dv=128, bf16 q/k/v,
-fp32 logits/state/output). The line also carries the generation-decode measurement
-(rsm_decode_step on 256 sequences x 16 heads, M=128 K=16 Dv=128, state from a 2048-token prefill).
+fp32 logits/state/output). The JSON line also carries
+  - `configs`: the other prefill workloads (tiny fp32 check, the pages' small training shape, the
+    mid-size per-slot-decay prefill), each with its time, roofline and the oracle beside it;
+  - `decode`: the generation workload (rsm_decode_step on 256 sequences x 16 heads, M=128 K=16
+    Dv=128, state from a 2048-token prefill), all 1024 steps timed on the device, an end-to-end
+    figure with each step's inputs copied in from host memory, and the oracle on its first steps.
+Roofline bytes are the path's algorithmic bytes (o counted in v's dtype); the extra bytes of the
+library's fp32 o are reported beside them.
 
 Under torchrun (N > 1) every rank runs its own replica on its own GPU with its own inputs (the
 path shards by sequence with no data exchange), timing is taken on the device with CUDA events,
@@ -41,14 +47,22 @@ def load_peaks() -> dict:
 # --------------------------------------------------------------------------- work accounting
 
 def prefill_bytes(w) -> int:
-    """Algorithmic bytes of one prefill: every input read once, o and H_T written once."""
+    """Algorithmic bytes of one prefill (the per-token-head figure of the path's scope table):
+    every input read once, o written once in v's dtype, H_T written once."""
     es = 2 if w.dtype == "bf16" else 4
     th = w.B * w.T * w.H
     b = th * (2 * w.M * es + w.Dv * es + w.M * 4)          # q, k, v, logits
     b += th * (w.M * 4 if w.decay == "slot" else 4)        # f
-    b += th * w.Dv * 4                                     # o (fp32)
+    b += th * w.Dv * es                                    # o in v's dtype
     b += w.B * w.H * w.M * w.Dv * 4                        # H_T
     return b
+
+
+def o_fp32_extra_bytes(w) -> int:
+    """Bytes the library writes beyond prefill_bytes(): it returns o in fp32 for every input dtype
+    (a bf16 o alone would take most of the bf16 error bar on heavy-tailed outputs)."""
+    es = 2 if w.dtype == "bf16" else 4
+    return w.B * w.T * w.H * w.Dv * (4 - es)
 
 
 def prefill_flops(w, chunk=64) -> int:
@@ -203,6 +217,24 @@ def oracle_sample(w, seconds_target: float = 3.0) -> dict:
                       f"{used} threads over heads; {dt1:.1f} s", "seconds": dt1, "tokens": T1 * reps}
 
 
+def oracle_decode_sample(w, state, steps, state_bytes) -> dict:
+    """Times the fp64 CPU oracle on the first steps of the generation workload, every stream,
+    starting from the device's post-prefill state (upcast), and reports the state rate it reaches
+    per step in the decode line's unit."""
+    from oracle import oracle
+    cores = oracle.default_threads()
+    n = steps["q"].shape[0]
+    t0 = time.perf_counter()
+    for i in range(n):
+        state = oracle.decode_step(steps["q"][i], steps["k"][i], steps["v"][i], steps["logits"][i], steps["f"][i],
+                                   w.K, state, nthreads=cores)["state"]
+    dt = (time.perf_counter() - t0) / n
+    return {"value": state_bytes / dt / 1e9, "unit": "GB/s (state)", "cores": min(cores, w.B * w.H),
+            "kind": "oracle", "ms_per_step": dt * 1e3,
+            "sample": f"first {n} of {w.decode_steps} steps, all {w.B}x{w.H} streams, from the device's "
+                      f"post-prefill state, fp64, {min(cores, w.B * w.H)} threads over streams"}
+
+
 def _sources_digest() -> str:
     """sha256 of the CUDA sources (used to tell whether stored ncu counters are still current)."""
     from sparse_routed_slot_b200.profile_case import sources_digest
@@ -226,81 +258,124 @@ def stored_traffic(key: str):
 
 KERNEL_NAMES = {4: ["route records", "segment summary", "segment scan", "chunk scan"],
                 2: ["route records", "chunk scan"], 1: ["chunk scan (CUDA cores)"]}
+L2_FLUSH_BYTES = 256 << 20  # written between timed steps of workloads smaller than L2 (126 MB)
+
+
+class PrefillCase:
+    """One prefill workload on the device: inputs, outputs, workspace and the timed call."""
+
+    def __init__(self, w, dev, rank, path):
+        import torch
+        from sparse_routed_slot_b200 import api
+        from sparse_routed_slot_b200.workloads import make_inputs
+        self.w, self.path = w, path
+        self.x = make_inputs(w.B, w.T, w.H, w.M, w.Dv, w.torch_dtype, w.decay,
+                             seed=replica_seed(w.seed, rank), device=dev)
+        self.o = torch.empty(w.B, w.T, w.H, w.Dv, dtype=torch.float32, device=dev)
+        self.HT = torch.empty(w.B, w.H, w.M, w.Dv, dtype=torch.float32, device=dev)
+        a = api._forward_args(self.x["q"], self.x["k"], self.x["v"], self.x["logits"], self.x["f"], w.K, None,
+                              self.o, self.HT, None, None, path, False)
+        self.path_used = api.selected_path(a)
+        self.launches = api.kernel_launches(a)
+        self.ws = torch.empty(max(api.workspace_bytes(a), 1), dtype=torch.uint8, device=dev)
+        self.nbytes = prefill_bytes(w)
+        self.flush = None if self.nbytes + o_fp32_extra_bytes(w) > L2_FLUSH_BYTES else \
+            torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step(self, x=None):
+        import sparse_routed_slot_b200 as rsm
+        x = self.x if x is None else x
+        rsm.forward(x["q"], x["k"], x["v"], x["logits"], x["f"], self.w.K, out={"o": self.o, "HT": self.HT},
+                    workspace=self.ws, path=self.path)
+
+    def time(self, steps, warmup, world, stream, kernel_split=True):
+        """Mean device time of one call (ms) and the per-kernel split (ms), CUDA events on the
+        launching stream; the L2 is flushed between timed calls when the workload fits in it."""
+        import ctypes
+        import torch
+        from sparse_routed_slot_b200 import _lib
+        L = _lib.load()
+        for _ in range(warmup):
+            self.step()
+        n = self.launches
+        kev = [[torch.cuda.Event(enable_timing=True) for _ in range(n + 1)] for _ in range(steps)]
+        for row in kev:  # torch creates the CUDA event on its first record
+            for e in row:
+                e.record(stream)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for a, b in ev:
+            a.record(stream)
+            b.record(stream)
+        kev_ptrs = [(ctypes.c_void_p * (n + 1))(*[e.cuda_event for e in row]) for row in kev]
+        torch.cuda.synchronize()
+        barrier(world)
+        for i in range(steps):
+            if self.flush is not None:
+                self.flush.zero_()
+            if kernel_split:
+                _lib.check(L.rsm_forward_set_profile_events(kev_ptrs[i], n + 1))
+            ev[i][0].record(stream)
+            self.step()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        _lib.check(L.rsm_forward_set_profile_events(None, 0))
+        barrier(world)
+        ms = sum(a.elapsed_time(b) for a, b in ev) / steps
+        kms = [sum(row[j].elapsed_time(row[j + 1]) for row in kev) / steps for j in range(n)] if kernel_split else []
+        return ms, kms
+
+    def roofline(self, ms, peaks, traffic_key):
+        achieved = self.nbytes / (ms * 1e-3) / 1e9
+        w = self.w
+        return {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": stored_traffic(traffic_key),
+                "algorithmic_bytes": self.nbytes, "o_fp32_extra_bytes": o_fp32_extra_bytes(w),
+                "frac_with_o_fp32": (self.nbytes + o_fp32_extra_bytes(w)) / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                "peak_source": peaks["source"] + " (burst copy)",
+                "tensor_tflops": prefill_flops(w) / (ms * 1e-3) / 1e12}
+
+
+def config_of(w, case, world, extra=None):
+    c = {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "M": w.M, "K": w.K, "Dv": w.Dv,
+         "decay": w.decay, "qkv_dtype": w.dtype, "state_dtype": "f32", "o_dtype": "f32",
+         "path": case.path_used, "parallelism": f"replicas{world}",
+         "l2": (f"L2 flushed between timed calls ({L2_FLUSH_BYTES >> 20} MB written)" if case.flush is not None
+                else f"inputs larger than L2 ({case.nbytes / 1e6:.0f} MB per step, no flush)")}
+    c.update(extra or {})
+    return c
 
 
 def run_ours(args, world, rank, local):
-    import ctypes
     import torch
     import sparse_routed_slot_b200 as rsm
-    from sparse_routed_slot_b200 import _lib, api
-    from sparse_routed_slot_b200.workloads import WORKLOADS, make_inputs
+    from sparse_routed_slot_b200.workloads import WORKLOADS
 
     w = WORKLOADS[args.workload]
     dev = torch.device("cuda", local)
     peaks = load_peaks()
-    x = make_inputs(w.B, w.T, w.H, w.M, w.Dv, w.torch_dtype, w.decay, seed=replica_seed(w.seed, rank), device=dev)
-    o = torch.empty(w.B, w.T, w.H, w.Dv, dtype=torch.float32, device=dev)
-    HT = torch.empty(w.B, w.H, w.M, w.Dv, dtype=torch.float32, device=dev)
-    outs = {"o": o, "HT": HT}
-    a = api._forward_args(x["q"], x["k"], x["v"], x["logits"], x["f"], w.K, None, o, HT, None, None,
-                          args.path, False)
-    ws_bytes = api.workspace_bytes(a)
-    path_used = api.selected_path(a)
-    launches = api.kernel_launches(a)
-    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
-    L = _lib.load()
-
-    def step():
-        rsm.forward(x["q"], x["k"], x["v"], x["logits"], x["f"], w.K, out=outs, workspace=ws,
-                    path=args.path)
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    barrier(world)
     stream = torch.cuda.current_stream(dev)
-    # per-kernel events inside every timed call (recorded by the library on this stream)
-    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(launches + 1)] for _ in range(args.steps)]
-    for row in kev:  # torch creates the CUDA event on its first record
-        for e in row:
-            e.record(stream)
-    torch.cuda.synchronize()
-    kev_ptrs = [(ctypes.c_void_p * (launches + 1))(*[e.cuda_event for e in row]) for row in kev]
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    case = PrefillCase(w, dev, rank, args.path)
     clocks = ClockSampler(local)
-    torch.cuda.synchronize()
-    barrier(world)
-    ev[0].record(stream)
-    for i in range(args.steps):
-        _lib.check(L.rsm_forward_set_profile_events(kev_ptrs[i], launches + 1))
-        step()
-        ev[i + 1].record(stream)
-    torch.cuda.synchronize()
-    _lib.check(L.rsm_forward_set_profile_events(None, 0))
-    barrier(world)
+    ms, kms = case.time(args.steps, args.warmup, world, stream)
     clk = clocks.stop()
-    per = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
-    ms = sum(per) / len(per)
-    kms = [sum(row[j].elapsed_time(row[j + 1]) for row in kev) / args.steps for j in range(launches)]
-    names = KERNEL_NAMES.get(launches, [f"kernel {j}" for j in range(launches)])
+    names = KERNEL_NAMES.get(case.launches, [f"kernel {j}" for j in range(case.launches)])
     tokens = w.B * w.T
     value, ms_max = job_throughput(tokens, ms, world)
 
     # end to end through the public call with host buffers: pinned inputs copied in, result out
-    host_in = {n: t.cpu().pin_memory() for n, t in x.items()}
-    dev_in = {n: torch.empty_like(t) for n, t in x.items()}
-    host_o = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-    host_HT = torch.empty(HT.shape, dtype=HT.dtype).pin_memory()
+    host_in = {n: t.cpu().pin_memory() for n, t in case.x.items()}
+    dev_in = {n: torch.empty_like(t) for n, t in case.x.items()}
+    host_o = torch.empty(case.o.shape, dtype=case.o.dtype).pin_memory()
+    host_HT = torch.empty(case.HT.shape, dtype=case.HT.dtype).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in host_in.values())
     d2h = host_o.numel() * 4 + host_HT.numel() * 4
 
     def e2e_step():
         for n in dev_in:
             dev_in[n].copy_(host_in[n], non_blocking=True)
-        rsm.forward(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["logits"], dev_in["f"], w.K,
-                    out=outs, workspace=ws, path=args.path)
-        host_o.copy_(o, non_blocking=True)
-        host_HT.copy_(HT, non_blocking=True)
+        case.step(dev_in)
+        host_o.copy_(case.o, non_blocking=True)
+        host_HT.copy_(case.HT, non_blocking=True)
 
     for _ in range(max(1, args.warmup)):
         e2e_step()
@@ -315,62 +390,83 @@ def run_ours(args, world, rank, local):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
     del host_in, dev_in
 
-    nbytes = prefill_bytes(w)
-    achieved = nbytes / (ms * 1e-3) / 1e9
+    roof = case.roofline(ms, peaks, f"{w.name}/forward")
+    roof["kernel"] = f"rsm_forward, all {case.launches} launches of the step (" + ", ".join(names) + ")"
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32" if path_used == "simt" else "tf32", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "M": w.M, "K": w.K, "Dv": w.Dv,
-                   "decay": w.decay, "qkv_dtype": w.dtype, "state_dtype": "f32", "o_dtype": "f32",
-                   "path": path_used, "parallelism": f"replicas{world}",
-                   "l2": f"inputs larger than L2 ({nbytes / 1e6:.0f} MB per step, no flush)"},
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": achieved / peaks["hbm_gbs"],
-                     "traffic": stored_traffic(f"{w.name}/forward"),
-                     "algorithmic_bytes": nbytes,
-                     "kernel": f"rsm_forward, all {launches} launches of the step (" + ", ".join(names) + ")",
-                     "peak_source": peaks["source"] + " (burst copy)",
-                     "tensor_tflops": prefill_flops(w) / (ms * 1e-3) / 1e12},
+        "vs_baseline": None, "dtype": "f32" if case.path_used == "simt" else "tf32", "data": "synthetic",
+        "config": config_of(w, case, world),
+        "roofline": roof,
         "kernels": [{"name": n, "ms": t, "share": t / sum(kms) if sum(kms) > 0 else None}
                     for n, t in zip(names, kms)],
         "e2e": {"value": tokens * world / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": args.steps * launches,
+        "gpu_launches": 2 * args.steps * case.launches,  # device-timed steps and end-to-end steps
         "clocks": clk,
     }
-    if not args.no_decode:
-        line["decode"] = run_decode(args, world, rank, local, peaks)
-        line["gpu_launches"] += line["decode"]["steps_timed"]
+    del case
     if rank == 0 and not args.no_cpu:
         line["cpu_baseline"] = oracle_sample(w)
+    if not args.no_configs:
+        line["configs"] = []
+        for name in ("tiny_fp32", "small_bf16", "mid_gla_bf16"):
+            sub = run_prefill_config(args, WORKLOADS[name], world, rank, local, peaks)
+            line["gpu_launches"] += sub.pop("launches_timed")
+            line["configs"].append(sub)
+    if not args.no_decode:
+        line["decode"] = run_decode(args, world, rank, local, peaks)
+        line["gpu_launches"] += line["decode"].pop("launches_timed")
     return line
 
 
+def run_prefill_config(args, w, world, rank, local, peaks) -> dict:
+    """A sub-line for another prefill workload: device time, roofline and the oracle beside it."""
+    import torch
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    case = PrefillCase(w, dev, rank, args.path)
+    steps = max(args.steps, 20)
+    clocks = ClockSampler(local)
+    ms, kms = case.time(steps, args.warmup, world, stream)
+    clk = clocks.stop()
+    value, ms_max = job_throughput(w.B * w.T, ms, world)
+    names = KERNEL_NAMES.get(case.launches, [f"kernel {j}" for j in range(case.launches)])
+    roof = case.roofline(ms, peaks, f"{w.name}/forward")
+    roof["kernel"] = f"rsm_forward, all {case.launches} launches of the step (" + ", ".join(names) + ")"
+    sub = {"workload": w.name, "value": value, "unit": "tokens/s", "ms_per_step": ms_max, "steps": steps,
+           "dtype": "f32" if case.path_used == "simt" else "tf32", "config": config_of(w, case, world),
+           "roofline": roof,
+           "kernels": [{"name": n, "ms": t} for n, t in zip(names, kms)], "clocks": clk,
+           "launches_timed": steps * case.launches}
+    if rank == 0 and not args.no_cpu:
+        sub["cpu_baseline"] = oracle_sample(w)
+    return sub
+
+
 def run_decode(args, world, rank, local, peaks) -> dict:
-    """Generation decode: 256 sequences x 16 heads, state from a 2048-token prefill, then
-    `decode_steps` timed rsm_decode_step calls (default 256 of the 1024-step workload)."""
+    """Generation decode: 256 sequences x 16 heads, state from a 2048-token prefill, then every
+    step of the workload (1024 rsm_decode_step calls, one launch each) timed on the device."""
     import torch
     import sparse_routed_slot_b200 as rsm
-    from sparse_routed_slot_b200.workloads import WORKLOADS, make_inputs
+    from sparse_routed_slot_b200.workloads import DECODE_PREFILL_GROUP, WORKLOADS, decode_prefill_group, \
+        decode_step_inputs
 
     w = WORKLOADS["decode_256x16"]
     dev = torch.device("cuda", local)
     state = torch.zeros(w.B, w.H, w.M, w.Dv, dtype=torch.float32, device=dev)
-    # prefill in groups of 32 sequences (bounded input memory)
-    for b0 in range(0, w.B, 32):
-        x = make_inputs(32, w.decode_prefill_T, w.H, w.M, w.Dv, w.torch_dtype, w.decay,
-                        seed=w.seed + b0 + 1000 * rank, device=dev)
+    for b0 in range(0, w.B, DECODE_PREFILL_GROUP):
+        x = decode_prefill_group(w, b0, rank, device=dev)
         out = rsm.forward(x["q"], x["k"], x["v"], x["logits"], x["f"], w.K, state=True, path=args.path)
-        state[b0:b0 + 32].copy_(out["HT"])
+        state[b0:b0 + DECODE_PREFILL_GROUP].copy_(out["HT"])
         del x, out
+    state0 = state.clone() if rank == 0 and not args.no_cpu else None
     nsteps = args.decode_steps
-    d = make_inputs(nsteps, w.B, w.H, w.M, w.Dv, w.torch_dtype, w.decay, seed=w.seed + 7 + 1000 * rank,
-                    device=dev)
+    d = decode_step_inputs(w, nsteps, rank, device=dev)
     o = torch.empty(w.B, w.H, w.Dv, dtype=torch.float32, device=dev)
 
-    def step(i):
-        rsm.decode_step(d["q"][i], d["k"][i], d["v"][i], d["logits"][i], d["f"][i], w.K, state, o=o)
+    def step(i, x=d):
+        rsm.decode_step(x["q"][i], x["k"][i], x["v"][i], x["logits"][i], x["f"][i], w.K, state, o=o)
 
     for i in range(3):
         step(i)
@@ -389,16 +485,52 @@ def run_decode(args, world, rank, local, peaks) -> dict:
     sb, tb = decode_bytes(w.B, w.H, w.M, w.K, w.Dv, 2, w.decay == "slot")
     state_gbs = sb / (ms * 1e-3) / 1e9
     total_gbs = tb / (ms * 1e-3) / 1e9
-    return {"value": state_gbs * world, "unit": "GB/s (state, all GPUs)", "ms_per_step": ms,
-            "steps_timed": nsteps, "total_gbs": total_gbs * world,
-            "roofline": {"bound": "hbm", "achieved": total_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": total_gbs / peaks["hbm_gbs"],
-                         "traffic": stored_traffic("decode_256x16/step"),
-                         "algorithmic_bytes": tb, "kernel": "rsm decode step (one launch)"},
-            "clocks": clk, "traffic_note": "single launch per step",
-            "config": {"workload": w.name, "B": w.B, "H": w.H, "M": w.M, "K": w.K, "Dv": w.Dv,
-                       "prefill_T": w.decode_prefill_T, "graph": False,
-                       "l2": f"state {w.B * w.H * w.M * w.Dv * 4 / 1e6:.0f} MB > L2"}}
+
+    # end to end: every step's inputs copied in from pinned host memory and o read back; the
+    # carried state stays on the device (it is the recurrence's own memory)
+    e2e_steps = min(nsteps, 256)
+    host_in = {n: t[:e2e_steps].cpu().pin_memory() for n, t in d.items()}
+    dev_in = {n: torch.empty_like(t[0]) for n, t in d.items()}
+    host_o = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    h2d = sum(t[0].numel() * t.element_size() for t in host_in.values())
+
+    def e2e_step(i):
+        for n in dev_in:
+            dev_in[n].copy_(host_in[n][i], non_blocking=True)
+        rsm.decode_step(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["logits"], dev_in["f"], w.K, state, o=o)
+        host_o.copy_(o, non_blocking=True)
+
+    for i in range(3):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0.record(stream)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
+    cpu_steps = {n: t[:8].float().cpu().numpy() for n, t in d.items()} if state0 is not None else None
+    del host_in, dev_in, d
+
+    res = {"value": state_gbs * world, "unit": "GB/s (state, all GPUs)", "ms_per_step": ms,
+           "steps_timed": nsteps, "total_gbs": total_gbs * world,
+           "tokens_per_s": w.B * world / (ms * 1e-3),
+           "roofline": {"bound": "hbm", "achieved": total_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                        "frac": total_gbs / peaks["hbm_gbs"],
+                        "traffic": stored_traffic("decode_256x16/step"),
+                        "algorithmic_bytes": tb, "kernel": "rsm_decode_step (one launch per step)",
+                        "peak_source": peaks["source"] + " (burst copy)"},
+           "e2e": {"value": sb * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s (state, all GPUs)",
+                   "ms_per_step": e2e_ms, "steps": e2e_steps,
+                   "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": host_o.numel() * 4},
+           "clocks": clk, "launches_timed": nsteps + e2e_steps,
+           "config": {"workload": w.name, "B": w.B, "H": w.H, "M": w.M, "K": w.K, "Dv": w.Dv,
+                      "decay": w.decay, "qkv_dtype": w.dtype, "prefill_T": w.decode_prefill_T,
+                      "graph": False, "l2": f"state {w.B * w.H * w.M * w.Dv * 4 / 1e6:.0f} MB > L2, no flush"}}
+    if state0 is not None:
+        res["cpu_baseline"] = oracle_decode_sample(w, state0.double().cpu().numpy(), cpu_steps, sb)
+    return res
 
 
 # --------------------------------------------------------------------------- reference arm
@@ -436,8 +568,9 @@ def main():
     ap.add_argument("--workload", default="long_ctx_bf16")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--path", default="auto", choices=["auto", "simt", "tensor"])
-    ap.add_argument("--decode-steps", type=int, default=256)
+    ap.add_argument("--decode-steps", type=int, default=1024)
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-configs", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:

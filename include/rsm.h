@@ -66,7 +66,16 @@ typedef enum rsm_path {
   RSM_PATH_TENSOR = 2   /* tcgen05/TMEM tensor-core path; RSM_ERR_UNSUPPORTED when not available */
 } rsm_path;
 
-enum { RSM_FLAG_VALIDATE = 1 };
+enum {
+  /* Device-side check of the preconditions: a non-finite logit or a non-finite or positive f is
+   * reported as RSM_ERR_NONFINITE by rsm_get_device_status (results are then undefined). */
+  RSM_FLAG_VALIDATE = 1,
+  /* Testing aid for the bounded-wait error path (no counterpart on the pages; never set in normal
+   * use): in rsm_decode_step the routing warps hand over no routing slot and the warps waiting for
+   * one give up after a short bound, so every CTA takes its timeout exit, the call writes neither o
+   * nor the state, and rsm_get_device_status reports RSM_ERR_TIMEOUT. Other calls ignore it. */
+  RSM_FLAG_TEST_STALL_ROUTING = 256
+};
 
 /* ---------------------------------------------------------------------------------------------
  * rsm_route -- TopK routing of router logits.
@@ -148,18 +157,20 @@ RSM_API rsm_status rsm_forward_set_profile_events(void* const* events, int n_eve
  *   The pages have no counterpart to this call; it exists for callers with no way to allocate:
  *   work recorded into a CUDA graph capture (an allocation would break the capture), programs
  *   whose allocator owns every byte of the device, or runtimes with a fixed memory plan. Where
- *   rsm_forward needs a caller-supplied workspace (long sequences split into segments), this call
- *   uses a scratch array built into the library instead; the caller passes only the inputs and
- *   outputs (args->workspace and args->workspace_bytes are ignored). Results are those of
- *   rsm_forward.
- *   Limit: the scratch holds rsm_forward_noalloc_max_scratch() bytes (16 MiB); sizes whose
- *   workspace would exceed it return RSM_ERR_WORKSPACE with the sizes in rsm_last_error().
+ *   rsm_forward needs a caller-supplied workspace (the tensor-core path: routing records of every
+ *   token, 144 bytes per token and head for K <= 16 and 288 for K <= 32, plus the segment states
+ *   when a long sequence is split), this call uses a scratch array built into the library instead;
+ *   the caller passes only the inputs and outputs (args->workspace and args->workspace_bytes are
+ *   ignored). Results are bit-identical to those of rsm_forward.
+ *   Limit: the scratch holds rsm_forward_noalloc_max_scratch() bytes (16 MiB), about 116,000
+ *   token-heads (B*T*H) at K <= 16 before segment states; sizes whose workspace would exceed it
+ *   return RSM_ERR_WORKSPACE with the sizes in rsm_last_error(), before anything is launched.
  *   The array occupies device memory on every GPU that loads the library, until exit. The first
- *   call on each device looks up the array's device address (cudaGetSymbolAddress) with that
- *   device current; make that first call before any stream capture. All calls share the array
- *   and it keeps the last call's contents (nothing in it needs to start at zero): calls whose
- *   GPU work overlaps in time, on any streams or host threads of one device, race and must not
- *   be issued. No CUDA allocation routine is called.
+ *   call on each device (and the first after a device reset) looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call before any stream
+ *   capture. All calls share the array and it keeps the last call's contents (nothing in it needs
+ *   to start at zero): calls whose GPU work overlaps in time, on any streams or host threads of
+ *   one device, race and must not be issued. No CUDA allocation routine is called.
  * ------------------------------------------------------------------------------------------- */
 RSM_API rsm_status rsm_forward_noalloc(const rsm_forward_args* args, void* stream);
 RSM_API size_t rsm_forward_noalloc_max_scratch(void);

@@ -17,6 +17,7 @@ RSM_F32, RSM_BF16 = 0, 1
 RSM_DECAY_HEAD, RSM_DECAY_SLOT = 0, 1
 RSM_PATH_AUTO, RSM_PATH_SIMT, RSM_PATH_TENSOR = 0, 1, 2
 RSM_FLAG_VALIDATE = 1
+RSM_FLAG_TEST_STALL_ROUTING = 256
 
 # Every symbol include/rsm.h declares (the CPU tests check the library exports all of them).
 EXPORTED = ("rsm_route", "rsm_forward_workspace_size", "rsm_forward", "rsm_forward_selected_path",

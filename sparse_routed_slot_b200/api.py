@@ -136,9 +136,10 @@ def forward(q, k, v, logits, f, K: int, H0=None, *, state: bool = True, routing:
 
 
 def decode_step(q, k, v, logits, f, K: int, state, *, routing: bool = False, validate: bool = False,
-                o=None):
+                o=None, flags: int = 0):
     """One token per (b,h). q, k [B,H,M]; v [B,H,Dv]; logits [B,H,M]; f [B,H] or [B,H,M];
-    state [B,H,M,Dv] fp32 updated in place. Returns dict(o [B,H,Dv] fp32, idx, score)."""
+    state [B,H,M,Dv] fp32 updated in place. Returns dict(o [B,H,Dv] fp32, idx, score).
+    `flags` are extra RSM_FLAG_* bits passed through unchanged."""
     B, H, M = q.shape
     Dv = v.shape[-1]
     if q.dtype not in _DTYPES:
@@ -168,7 +169,7 @@ def decode_step(q, k, v, logits, f, K: int, state, *, routing: bool = False, val
     a.state, a.o = state.data_ptr(), o.data_ptr()
     a.idx_out = None if idx is None else idx.data_ptr()
     a.score_out = None if sc is None else sc.data_ptr()
-    a.flags = _lib.RSM_FLAG_VALIDATE if validate else 0
+    a.flags = (_lib.RSM_FLAG_VALIDATE if validate else 0) | flags
     _lib.check(_lib.load().rsm_decode_step(ctypes.byref(a), _stream(dev)))
     return {"o": o, "idx": idx, "score": sc}
 

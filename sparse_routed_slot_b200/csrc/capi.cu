@@ -81,7 +81,7 @@ rsm_status check_forward(const rsm_forward_args* a) {
   RSM_OPTIONAL_PTR(a->score_out, "score_out");
   if (a->path == RSM_PATH_TENSOR && !rsm::prefill_tc_supported(*a))
     return fail(RSM_ERR_UNSUPPORTED,
-                "the tensor-core path needs bf16 q/k/v, M in {64,128}, Dv in {64,128}");
+                "the tensor-core path needs bf16 q/k/v, M = Dv = 128 and K <= 32");
   return RSM_OK;
 }
 

@@ -19,7 +19,9 @@
 //   whether to write the row and by how much to decay it.
 //
 // Every wait is bounded; on expiry the CTA records RSM_ERR_TIMEOUT, stops, and the producer waits
-// (bounded) for its copies still in flight before the CTA exits.
+// (bounded) for its copies still in flight before the CTA exits. RSM_FLAG_TEST_STALL_ROUTING
+// exercises that path on purpose: the routers hand over nothing and the consumers' wait for the
+// first routing slot uses a short limit, so every CTA takes the timeout exit.
 #include "common.cuh"
 #include "kernels.h"
 #include "tc.cuh"
@@ -149,7 +151,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(rsm_decode_args a) 
   } else if (warp >= kRouterWarp0) {
     // ------------------------------------------------------------------------------ routers
     const int r = warp - kRouterWarp0;
-    for (int m = r; m < nitems && !*abort_flag; m += kRouters) {
+    // testing aid: no routing slot is ever handed over, so the consumers' bounded wait expires
+    const int route_items = (a.flags & RSM_FLAG_TEST_STALL_ROUTING) ? 0 : nitems;
+    for (int m = r; m < route_items && !*abort_flag; m += kRouters) {
       const int slot = m % nslots;
       if (m >= nslots && !tc::mbar_wait(&rempty[slot], ((m / nslots) - 1) & 1)) {
         fail();
@@ -206,13 +210,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(rsm_decode_args a) 
     const int RG = kConsumers / CG;  // row groups
     const int cg = tid % CG, rg = tid / CG;
     const bool active = rg < RG;
+    // the hand-off wait's poll limit: the default bound, or a short one under the testing aid
+    const uint32_t rfull_limit = (a.flags & RSM_FLAG_TEST_STALL_ROUTING) ? (1u << 10) : (1u << 22);
     int n = 0;
     for (int m = 0; m < nitems; ++m) {
       // A thread that sees a failure stops waiting and computing but still reaches the item's
       // barrier, which ORs the failure over all consumers, so that they leave together.
       bool ab = false;
       const int slot = m % nslots;
-      if (!tc::mbar_wait(&rfull[slot], (m / nslots) & 1)) {
+      if (!tc::mbar_wait(&rfull[slot], (m / nslots) & 1, rfull_limit)) {
         fail();
         ab = true;
       }

@@ -94,10 +94,21 @@ def make_workload_inputs(w: Workload, device="cpu", h0: bool = False) -> dict:
     return make_inputs(w.B, w.T, w.H, w.M, w.Dv, w.torch_dtype, w.decay, w.seed, device, h0)
 
 
-def make_decode_inputs(B: int, H: int, M: int, Dv: int, steps: int, dtype: torch.dtype,
-                       decay: str, seed: int, device="cpu") -> dict:
-    """Per-step decode inputs stacked on a leading step axis: q, k, logits [S,B,H,M], v [S,B,H,Dv],
-    f [S,B,H] or [S,B,H,M]. Same recipe as the prefill inputs."""
-    d = make_inputs(steps, B, H, M, Dv, dtype, decay, seed, device)
-    # make_inputs lays out [B',T',H,...]; here B' = steps and T' = the batch of sequences.
-    return d
+# The generation-decode workload: its state comes from a prefill of `decode_prefill_T` random
+# tokens for every sequence, drawn in groups of `DECODE_PREFILL_GROUP` sequences (bounded input
+# memory), then `decode_steps` single-token steps. The benchmark and the tests draw the same
+# tensors through these two functions.
+DECODE_PREFILL_GROUP = 32
+
+
+def decode_prefill_group(w: Workload, b0: int, rank: int = 0, device="cpu") -> dict:
+    """Prefill inputs of sequences b0 .. b0 + DECODE_PREFILL_GROUP - 1 of a decode workload."""
+    return make_inputs(DECODE_PREFILL_GROUP, w.decode_prefill_T, w.H, w.M, w.Dv, w.torch_dtype,
+                       w.decay, seed=w.seed + b0 + 1000 * rank, device=device)
+
+
+def decode_step_inputs(w: Workload, steps: int, rank: int = 0, device="cpu") -> dict:
+    """Inputs of `steps` decode steps, stacked on a leading step axis: q, k, logits [S,B,H,M],
+    v [S,B,H,Dv], f [S,B,H] or [S,B,H,M]."""
+    return make_inputs(steps, w.B, w.H, w.M, w.Dv, w.torch_dtype, w.decay,
+                       seed=w.seed + 7 + 1000 * rank, device=device)
