@@ -12,6 +12,9 @@ These restate the RSM mixer in closed forms that do not run the token-by-token r
   is a gated linear-attention recurrence with per-slot gate (paperlayer.ai summary, sections
   3.4 "State-Space Models as RSMs" and A.5 "Efficient Training using Gated Linear Attention");
   computed as a masked matrix product with cumulative log-gates.
+* ``router_scores`` / ``selection_counts``: the router variants' scores (sigmoid or softmax over the
+  row, optionally normalised over the TopK set) and the per-slot selection counts, from library
+  routines (scipy's expit and softmax, numpy sums and bincount).
 * ``window_form``: the one-hot cyclic router with full overwrite, which turns the slot store into
   a window of the last M tokens ("Raven Part 1 -- Memory as a Set of Slots", "Key claims": a
   one-hot cyclic router recovers sliding-window attention; paperlayer.ai summary section 2.2).
@@ -30,7 +33,22 @@ def topk_stable(logits: np.ndarray, K: int) -> np.ndarray:
     return order[..., :K].astype(np.int32)
 
 
-def gates(logits, f, K: int):
+def router_scores(logits, K: int, router: str = "sigmoid"):
+    """Scores of every slot under a router variant, zero off the TopK set, with library routines:
+    scipy's expit (sigmoid) or softmax over the row's M slots, then, for the normalised variants,
+    division by the sum over the selected slots. Returns (selected mask, scores) [T,M]."""
+    from scipy.special import expit, softmax
+    lg = np.asarray(logits, dtype=np.float32).astype(np.float64)
+    sel = np.zeros(lg.shape, dtype=bool)
+    np.put_along_axis(sel, topk_stable(lg, K), True, axis=-1)
+    s = softmax(lg, axis=-1) if router.startswith("softmax") else expit(lg)
+    s = np.where(sel, s, 0.0)
+    if router.endswith("_norm"):
+        s = s / s.sum(axis=-1, keepdims=True)
+    return sel, s
+
+
+def gates(logits, f, K: int, router: str = "sigmoid"):
     """Per-(token, slot) decay a (1 off the selected set) and write weight (1-a) (0 off it).
 
     logits: [T,M] fp32; f: [T] or [T,M]. Returns (a, one_minus_a) as float64 [T,M].
@@ -40,16 +58,13 @@ def gates(logits, f, K: int):
     fx = np.asarray(f, dtype=np.float32).astype(np.float64)
     if fx.ndim == 1:
         fx = np.repeat(fx[:, None], M, axis=1)
-    sel = np.zeros((T, M), dtype=bool)
-    idx = topk_stable(lg, K)
-    np.put_along_axis(sel, idx, True, axis=1)
-    s = 1.0 / (1.0 + np.exp(-lg))
+    sel, s = router_scores(lg, K, router)
     a = np.where(sel, np.exp(s * fx), 1.0)
     one_minus_a = np.where(sel, 1.0 - np.exp(s * fx), 0.0)
     return a, one_minus_a
 
 
-def quadratic_form(q, k, v, logits, f, K: int, H0=None):
+def quadratic_form(q, k, v, logits, f, K: int, H0=None, router: str = "sigmoid"):
     """Unrolled closed form for one (b,h) stream. q,k,logits [T,M]; v [T,Dv]; f [T] or [T,M].
 
     Returns (o [T,Dv], HT [M,Dv]) in float64. O(T^2 M Dv): tiny inputs only.
@@ -59,7 +74,7 @@ def quadratic_form(q, k, v, logits, f, K: int, H0=None):
     v = np.asarray(v, np.float32).astype(np.float64)
     T, M = q.shape
     Dv = v.shape[1]
-    a, oma = gates(logits, f, K)
+    a, oma = gates(logits, f, K, router)
     h0 = np.zeros((M, Dv)) if H0 is None else np.asarray(H0, np.float64)
     o = np.zeros((T, Dv))
     for t in range(T):
@@ -113,6 +128,12 @@ def dense_masked_form(q, k, v, logits, f, H0=None):
     HT = (np.exp(G[-1])[:, None] * (np.zeros((M, v.shape[1])) if H0 is None else np.asarray(H0, np.float64))
           + (W * np.exp(G[-1][None, :] - G)).T @ v)
     return o, HT
+
+
+def selection_counts(logits, K: int):
+    """Tokens that select each slot: a bincount of the stable library sort's TopK. logits [T,M]."""
+    lg = np.asarray(logits, dtype=np.float32)
+    return np.bincount(topk_stable(lg, K).ravel(), minlength=lg.shape[-1]).astype(np.int32)
 
 
 def window_form(q, v, M: int):

@@ -34,18 +34,26 @@ def build(force: bool = False) -> str:
     return _LIB_PATH
 
 
+def bind(lib):
+    """Declares the C signatures on a loaded oracle library (also used for test mutants)."""
+    f32p = np.ctypeslib.ndpointer(np.float32, flags="C_CONTIGUOUS")
+    vp = ctypes.c_void_p
+    lib.rsmo_forward.argtypes = [ctypes.c_int] * 7 + [f32p] * 5 + [vp] * 5 + [ctypes.c_int]
+    lib.rsmo_forward.restype = ctypes.c_int
+    lib.rsmo_route.argtypes = [f32p, ctypes.c_longlong, ctypes.c_int, ctypes.c_int, vp, vp]
+    lib.rsmo_route.restype = ctypes.c_int
+    lib.rsmo_forward_ex.argtypes = [ctypes.c_int] * 7 + [f32p] * 5 + [vp] * 5 + [ctypes.c_int, vp, ctypes.c_int]
+    lib.rsmo_forward_ex.restype = ctypes.c_int
+    lib.rsmo_route_ex.argtypes = [f32p, ctypes.c_longlong, ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, vp]
+    lib.rsmo_route_ex.restype = ctypes.c_int
+    return lib
+
+
 def _load():
     global _lib
     with _lock:
         if _lib is None:
-            lib = ctypes.CDLL(build())
-            f32p = np.ctypeslib.ndpointer(np.float32, flags="C_CONTIGUOUS")
-            vp = ctypes.c_void_p
-            lib.rsmo_forward.argtypes = [ctypes.c_int] * 7 + [f32p] * 5 + [vp] * 5 + [ctypes.c_int]
-            lib.rsmo_forward.restype = ctypes.c_int
-            lib.rsmo_route.argtypes = [f32p, ctypes.c_longlong, ctypes.c_int, ctypes.c_int, vp, vp]
-            lib.rsmo_route.restype = ctypes.c_int
-            _lib = lib
+            _lib = bind(ctypes.CDLL(build()))
     return _lib
 
 
@@ -57,16 +65,23 @@ def _ptr(a):
     return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
 
 
+# Router variants: the score of a selected slot is its sigmoid (default) or its softmax over all M
+# slots of the row, optionally normalised over the K selected slots to sum to one.
+ROUTERS = {"sigmoid": 0, "softmax": 1, "sigmoid_norm": 2, "softmax_norm": 3}
+
+
 def default_threads() -> int:
     return max(1, os.cpu_count() or 1)
 
 
-def forward(q, k, v, logits, f, K: int, H0=None, want_idx: bool = True, nthreads: int | None = None):
+def forward(q, k, v, logits, f, K: int, H0=None, want_idx: bool = True, nthreads: int | None = None,
+            router: str = "sigmoid", want_counts: bool = False):
     """Sequential fp64 recurrence over all tokens.
 
     q, k, logits: [B,T,H,M]; v: [B,T,H,Dv]; f: [B,T,H] (per-head decay) or [B,T,H,M] (per-slot).
-    H0: optional [B,H,M,Dv] (zeros when None). Returns dict(o, HT, idx, score) with o [B,T,H,Dv]
-    float64, HT [B,H,M,Dv] float64, idx [B,T,H,K] int32, score [B,T,H,K] float64.
+    H0: optional [B,H,M,Dv] (zeros when None). router: a key of ROUTERS. Returns dict(o, HT, idx,
+    score, counts) with o [B,T,H,Dv] float64, HT [B,H,M,Dv] float64, idx [B,T,H,K] int32,
+    score [B,T,H,K] float64, counts [B,H,M] int32 (tokens that selected each slot) or None.
     """
     q, k, v, logits, f = map(_f32, (q, k, v, logits, f))
     B, T, H, M = q.shape
@@ -85,14 +100,16 @@ def forward(q, k, v, logits, f, K: int, H0=None, want_idx: bool = True, nthreads
     HT = np.zeros((B, H, M, Dv), np.float64)
     idx = np.zeros((B, T, H, K), np.int32) if want_idx else None
     score = np.zeros((B, T, H, K), np.float64) if want_idx else None
-    rc = _load().rsmo_forward(B, T, H, M, K, Dv, per_slot, q, k, v, logits, f, _ptr(h0), _ptr(o),
-                              _ptr(HT), _ptr(idx), _ptr(score), nthreads or default_threads())
+    counts = np.zeros((B, H, M), np.int32) if want_counts else None
+    rc = _load().rsmo_forward_ex(B, T, H, M, K, Dv, per_slot, q, k, v, logits, f, _ptr(h0), _ptr(o),
+                                 _ptr(HT), _ptr(idx), _ptr(score), ROUTERS[router], _ptr(counts),
+                                 nthreads or default_threads())
     if rc != 0:
         raise ValueError("oracle rejected the sizes")
-    return {"o": o, "HT": HT, "idx": idx, "score": score}
+    return {"o": o, "HT": HT, "idx": idx, "score": score, "counts": counts}
 
 
-def decode_step(q, k, v, logits, f, K: int, state, nthreads: int | None = None):
+def decode_step(q, k, v, logits, f, K: int, state, nthreads: int | None = None, router: str = "sigmoid"):
     """One generation step on a carried state (returns a new state; the argument is not changed).
 
     q, k, logits: [B,H,M]; v: [B,H,Dv]; f: [B,H] or [B,H,M]; state: [B,H,M,Dv].
@@ -100,17 +117,18 @@ def decode_step(q, k, v, logits, f, K: int, state, nthreads: int | None = None):
     q, k, v, logits, f = map(_f32, (q, k, v, logits, f))
     fx = f[:, None] if f.ndim in (2, 3) else f
     out = forward(q[:, None], k[:, None], v[:, None], logits[:, None], fx, K, H0=state,
-                  nthreads=nthreads)
+                  nthreads=nthreads, router=router, want_counts=True)
     return {"o": out["o"][:, 0], "state": out["HT"], "idx": out["idx"][:, 0],
-            "score": out["score"][:, 0]}
+            "score": out["score"][:, 0], "counts": out["counts"]}
 
 
-def route(logits, K: int):
-    """TopK (rank order: logit desc, index asc) and fp64 sigmoid scores for rows [N, M]."""
+def route(logits, K: int, router: str = "sigmoid"):
+    """TopK (rank order: logit desc, index asc) and fp64 scores of the router variant for rows
+    [N, M]."""
     lg = _f32(logits)
     N, M = lg.shape
     idx = np.zeros((N, K), np.int32)
     score = np.zeros((N, K), np.float64)
-    if _load().rsmo_route(lg, N, M, K, _ptr(idx), _ptr(score)) != 0:
+    if _load().rsmo_route_ex(lg, N, M, K, ROUTERS[router], _ptr(idx), _ptr(score)) != 0:
         raise ValueError("oracle rejected the sizes")
     return idx, score

@@ -19,6 +19,17 @@
  *      with zero routing is carried over unchanged).
  *   5. o_t = sum_i q_i * H[i,:], read after the write (README, "How Raven Works").
  *
+ * Router variants (rsmo_forward_ex, rsmo_route_ex; the default above is RSMO_SIGMOID):
+ *   - softmax scores: s_i = e^{l_i} / sum_{j=1..M} e^{l_j}, over all M slots of the row, in
+ *     place of the sigmoid (README, "Model Structure": top-k sigmoid/softmax router; "Usage":
+ *     router_score 'sigmoid' or 'softmax'; paperlayer.ai summary, section 6.2.1). The selected
+ *     set does not change: softmax, like sigmoid, is monotone in the logit.
+ *   - normalised scores: after the TopK cut, s_i = s_i / sum_{j in S_t} s_j, so the selected
+ *     weights sum to one (paperlayer.ai summary, section 4.1).
+ * Selection counts (rsmo_forward_ex): counts[b,h,i] += number of tokens t with i in S_t, the
+ * per-slot count behind the "effective sequence length" analysis (paperlayer.ai summary,
+ * section 7.1 and Figure 5: how much each slot processes).
+ *
  * Layouts (row-major, contiguous): q, k, logits [B,T,H,M]; v [B,T,H,Dv]; f [B,T,H] (per head)
  * or [B,T,H,M] (per slot); H0, HT [B,H,M,Dv]; o [B,T,H,Dv]; idx, score [B,T,H,K].
  * Inputs are the exact fp32 values the device sees (bf16 inputs are widened exactly beforehand).
@@ -56,6 +67,27 @@ void rsmo_topk(const float* row, int M, int K, int32_t* idx_out) {
 
 double rsmo_sigmoid(double x) { return 1.0 / (1.0 + exp(-x)); }
 
+enum { RSMO_SIGMOID = 0, RSMO_SOFTMAX = 1, RSMO_NORMALISE = 2 };
+
+/* Scores of the K selected slots sel[0..K) of one row of M logits, for a router variant. */
+void rsmo_scores(const float* row, int M, int K, const int32_t* sel, int router, double* s) {
+  if (router & RSMO_SOFTMAX) {
+    double mx = (double)row[0];
+    for (int j = 1; j < M; ++j)
+      if ((double)row[j] > mx) mx = (double)row[j];
+    double z = 0.0;
+    for (int j = 0; j < M; ++j) z += exp((double)row[j] - mx);
+    for (int r = 0; r < K; ++r) s[r] = exp((double)row[sel[r]] - mx) / z;
+  } else {
+    for (int r = 0; r < K; ++r) s[r] = rsmo_sigmoid((double)row[sel[r]]);
+  }
+  if (router & RSMO_NORMALISE) {
+    double sum = 0.0;
+    for (int r = 0; r < K; ++r) sum += s[r];
+    for (int r = 0; r < K; ++r) s[r] /= sum;
+  }
+}
+
 typedef struct {
   int B, T, H, M, K, Dv, per_slot;
   const float *q, *k, *v, *logits, *f;
@@ -63,6 +95,8 @@ typedef struct {
   double *o, *HT;
   int32_t* idx;
   double* score;
+  int router;
+  int32_t* counts;
   int pair_begin, pair_end; /* range of flattened (b,h) pairs handled by one worker */
 } rsmo_job;
 
@@ -72,6 +106,7 @@ static void rsmo_run_pair(const rsmo_job* J, int pair) {
   const int M = J->M, K = J->K, Dv = J->Dv, H = J->H, T = J->T;
   double* S = (double*)malloc(sizeof(double) * (size_t)M * (size_t)Dv);
   int32_t* sel = (int32_t*)malloc(sizeof(int32_t) * (size_t)K);
+  double* sc = (double*)malloc(sizeof(double) * (size_t)K);
   if (J->H0)
     memcpy(S, J->H0 + (size_t)pair * M * Dv, sizeof(double) * (size_t)M * Dv);
   else
@@ -84,9 +119,11 @@ static void rsmo_run_pair(const rsmo_job* J, int pair) {
     const float* lg = J->logits + row * M;
     const float* v = J->v + row * Dv;
     rsmo_topk(lg, M, K, sel);
+    rsmo_scores(lg, M, K, sel, J->router, sc);
     for (int r = 0; r < K; ++r) {
       const int i = sel[r];
-      const double s = rsmo_sigmoid((double)lg[i]);
+      const double s = sc[r];
+      if (J->counts) J->counts[(size_t)pair * M + i] += 1;
       const double f = J->per_slot ? (double)J->f[row * M + i] : (double)J->f[row];
       const double a = exp(s * f);
       const double wk = (1.0 - a) * (double)k[i];
@@ -106,6 +143,7 @@ static void rsmo_run_pair(const rsmo_job* J, int pair) {
     }
   }
   if (J->HT) memcpy(J->HT + (size_t)pair * M * Dv, S, sizeof(double) * (size_t)M * Dv);
+  free(sc);
   free(sel);
   free(S);
 }
@@ -117,16 +155,19 @@ static void* rsmo_worker(void* arg) {
 }
 
 /* Runs the recurrence over all (b,h) pairs; pairs are independent, so they are split over
- * nthreads POSIX threads (nthreads <= 1 runs inline). Returns 0 on success, -1 on bad sizes. */
-int rsmo_forward(int B, int T, int H, int M, int K, int Dv, int per_slot,
-                 const float* q, const float* k, const float* v, const float* logits,
-                 const float* f, const double* H0, double* o, double* HT, int32_t* idx,
-                 double* score, int nthreads) {
-  if (B < 0 || T < 0 || H < 0 || M < 1 || K < 1 || K > M || Dv < 1) return -1;
+ * nthreads POSIX threads (nthreads <= 1 runs inline). `router` is a combination of RSMO_SOFTMAX
+ * and RSMO_NORMALISE (0: sigmoid scores); `counts` [B,H,M] (or NULL) is added to.
+ * Returns 0 on success, -1 on bad sizes. */
+int rsmo_forward_ex(int B, int T, int H, int M, int K, int Dv, int per_slot,
+                    const float* q, const float* k, const float* v, const float* logits,
+                    const float* f, const double* H0, double* o, double* HT, int32_t* idx,
+                    double* score, int router, int32_t* counts, int nthreads) {
+  if (B < 0 || T < 0 || H < 0 || M < 1 || K < 1 || K > M || Dv < 1 || router < 0 || router > 3) return -1;
   const int pairs = B * H;
   if (nthreads < 1) nthreads = 1;
   if (nthreads > pairs) nthreads = pairs > 0 ? pairs : 1;
-  rsmo_job base = {B, T, H, M, K, Dv, per_slot, q, k, v, logits, f, H0, o, HT, idx, score, 0, pairs};
+  rsmo_job base = {B, T, H, M, K, Dv, per_slot, q, k, v, logits, f, H0, o, HT, idx, score, router, counts,
+                   0, pairs};
   if (nthreads == 1) {
     rsmo_worker(&base);
     return 0;
@@ -145,6 +186,15 @@ int rsmo_forward(int B, int T, int H, int M, int K, int Dv, int per_slot,
   return 0;
 }
 
+/* The default router (sigmoid scores, not normalised), no counts. */
+int rsmo_forward(int B, int T, int H, int M, int K, int Dv, int per_slot,
+                 const float* q, const float* k, const float* v, const float* logits,
+                 const float* f, const double* H0, double* o, double* HT, int32_t* idx,
+                 double* score, int nthreads) {
+  return rsmo_forward_ex(B, T, H, M, K, Dv, per_slot, q, k, v, logits, f, H0, o, HT, idx, score,
+                         RSMO_SIGMOID, NULL, nthreads);
+}
+
 /* One generation step: the same update and read for a single token per (b,h), applied in
  * place to the carried state (README, "Model Structure": fused recurrent computation for
  * inference). Layouts: q, k, logits [B,H,M]; v [B,H,Dv]; f [B,H] or [B,H,M];
@@ -157,13 +207,19 @@ int rsmo_decode_step(int B, int H, int M, int K, int Dv, int per_slot, const flo
                       score, nthreads);
 }
 
-/* Standalone routing: TopK indices (rank order) and sigmoid scores for rows [rows, M]. */
-int rsmo_route(const float* logits, long long rows, int M, int K, int32_t* idx, double* score) {
-  if (rows < 0 || M < 1 || K < 1 || K > M) return -1;
+/* Standalone routing: TopK indices (rank order) and the router variant's scores, rows [rows, M]. */
+int rsmo_route_ex(const float* logits, long long rows, int M, int K, int router, int32_t* idx,
+                  double* score) {
+  if (rows < 0 || M < 1 || K < 1 || K > M || router < 0 || router > 3) return -1;
   for (long long r = 0; r < rows; ++r) {
     const float* lg = logits + r * M;
     rsmo_topk(lg, M, K, idx + r * K);
-    for (int j = 0; j < K; ++j) score[r * K + j] = rsmo_sigmoid((double)lg[idx[r * K + j]]);
+    rsmo_scores(lg, M, K, idx + r * K, router, score + r * K);
   }
   return 0;
+}
+
+/* Standalone routing with sigmoid scores. */
+int rsmo_route(const float* logits, long long rows, int M, int K, int32_t* idx, double* score) {
+  return rsmo_route_ex(logits, rows, M, K, RSMO_SIGMOID, idx, score);
 }

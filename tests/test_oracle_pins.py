@@ -5,7 +5,9 @@
 * the TopK = M limit against a masked-matrix gated-linear-attention form;
 * the one-hot cyclic router limit against the sliding-window closed form;
 * TopK against a stable library sort, with constructed ties, signed zeros and saturating logits;
-* sigmoid scores against scipy's expit;
+* sigmoid scores against scipy's expit; the router variants (softmax over the row, scores
+  normalised over the TopK set) against scipy's softmax/expit and numpy sums, a hand-derived
+  example and the quadratic form; selection counts against a bincount of a library sort;
 * the invariant that unselected slots keep their bits;
 * mutants of the oracle (planted mistakes, compiled on the CPU) must fail these pins.
 """
@@ -218,6 +220,73 @@ def test_threads_do_not_change_results():
     assert np.array_equal(a["o"], b["o"]) and np.array_equal(a["HT"], b["HT"])
 
 
+# ----------------------------------------------------------------------------- router variants
+
+
+ROUTER_NAMES = ["sigmoid", "softmax", "sigmoid_norm", "softmax_norm"]
+
+
+@pytest.mark.parametrize("router", ROUTER_NAMES)
+def test_golden_router_variants(router):
+    g = json.load(open(os.path.join(GOLDEN, "hand_router_variants_M3.json")))
+    q, k, v, lg = (np.array(g[n], np.float32) for n in ("q", "k", "v", "logits"))
+    H0 = np.array(g["H0"], np.float64)
+    s_hand = g["expect_scores"][router]
+    f = np.array([[math.log(g["decay_targets"][0]) / s_hand[0], math.log(g["decay_targets"][1]) / s_hand[1], -1.0]],
+                 np.float32)
+    out = oracle.forward(q[None, :, None], k[None, :, None], v[None, :, None], lg[None, :, None], f[None, :, None],
+                         g["K"], H0[None, None], nthreads=1, router=router, want_counts=True)
+    assert np.array_equal(out["idx"][0, :, 0], np.array(g["expect_idx"]))
+    assert np.allclose(out["score"][0, 0, 0], s_hand, atol=g["tol"], rtol=0)
+    assert np.allclose(out["o"][0, :, 0], g["expect_o"], atol=g["tol"], rtol=0)
+    assert np.allclose(out["HT"][0, 0], g["expect_HT"], atol=g["tol"], rtol=0)
+    assert np.array_equal(out["counts"][0, 0], g["expect_counts"])
+    idx, sc = oracle.route(lg, g["K"], router)
+    assert np.allclose(sc[0], s_hand, atol=g["tol"], rtol=0)
+
+
+@pytest.mark.parametrize("router", ROUTER_NAMES)
+@pytest.mark.parametrize("M,K", [(8, 3), (32, 8), (64, 64)])
+def test_router_scores_match_library(router, M, K):
+    rng = np.random.default_rng(M + K)
+    lg = (3 * rng.standard_normal((50, M))).astype(np.float32)
+    lg[5] = 0.0                                   # all tied
+    idx, sc = oracle.route(lg, K, router)
+    sel, ref = brute.router_scores(lg, K, router)
+    assert np.array_equal(idx, brute.topk_stable(lg, K))
+    assert np.allclose(sc, np.take_along_axis(ref, idx.astype(np.int64), axis=1), rtol=1e-13, atol=0)
+    if router.endswith("_norm"):
+        assert np.allclose(sc.sum(axis=1), 1.0, rtol=1e-13)
+
+
+@pytest.mark.parametrize("router", ROUTER_NAMES)
+@pytest.mark.parametrize("per_slot", [False, True])
+def test_router_variants_match_quadratic_form(router, per_slot):
+    rng = np.random.default_rng(7 + per_slot)
+    T, M, Dv, K = 9, 6, 3, 2
+    q, k, v, lg, f = _rand_stream(rng, T, M, Dv, per_slot)
+    H0 = rng.standard_normal((M, Dv))
+    out = oracle.forward(q[None, :, None], k[None, :, None], v[None, :, None], lg[None, :, None], f[None, :, None],
+                         K, H0[None, None], nthreads=1, router=router)
+    o_b, HT_b = brute.quadratic_form(q, k, v, lg, f, K, H0, router=router)
+    assert _rel(out["o"][0, :, 0], o_b) <= 1e-12
+    assert _rel(out["HT"][0, 0], HT_b) <= 1e-12
+
+
+def test_selection_counts_match_bincount():
+    rng = np.random.default_rng(3)
+    B, T, H, M, Dv, K = 2, 40, 3, 16, 4, 5
+    x = {n: rng.standard_normal(sh).astype(np.float32) for n, sh in
+         dict(q=(B, T, H, M), k=(B, T, H, M), v=(B, T, H, Dv), logits=(B, T, H, M)).items()}
+    x["logits"][0, :7] = np.round(x["logits"][0, :7])   # exact ties
+    f = -np.abs(rng.standard_normal((B, T, H))).astype(np.float32)
+    out = oracle.forward(x["q"], x["k"], x["v"], x["logits"], f, K, want_counts=True)
+    for b in range(B):
+        for h in range(H):
+            assert np.array_equal(out["counts"][b, h], brute.selection_counts(x["logits"][b, :, h], K))
+    assert int(out["counts"].sum()) == B * T * H * K
+
+
 # ----------------------------------------------------------------------------- mutants
 
 # Each mutant plants one plausible mistake in a copy of the oracle source (compiled here, on the
@@ -234,6 +303,11 @@ MUTANTS = {
                                   "const double wk = (double)k[i];", None, None),
     "q_k_swapped_in_read": ("const double qi = (double)q[i];", "const double qi = (double)k[i];",
                             None, None),
+    "softmax_over_selected_only": ("for (int j = 0; j < M; ++j) z += exp((double)row[j] - mx);",
+                                   "for (int j = 0; j < K; ++j) z += exp((double)row[sel[j]] - mx);", None, None),
+    "normalise_by_first_score": ("for (int r = 0; r < K; ++r) sum += s[r];", "sum = s[0];", None, None),
+    "counts_by_rank": ("J->counts[(size_t)pair * M + i] += 1;", "J->counts[(size_t)pair * M + r] += 1;",
+                       None, None),
 }
 
 
@@ -256,13 +330,11 @@ def _build_mutant(tmp_path, name):
 def _pins_pass_with(lib_path) -> bool:
     saved = oracle._lib
     try:
-        lib = ctypes.CDLL(lib_path)
-        f32p = np.ctypeslib.ndpointer(np.float32, flags="C_CONTIGUOUS")
-        vp = ctypes.c_void_p
-        lib.rsmo_forward.argtypes = [ctypes.c_int] * 7 + [f32p] * 5 + [vp] * 5 + [ctypes.c_int]
-        lib.rsmo_route.argtypes = [f32p, ctypes.c_longlong, ctypes.c_int, ctypes.c_int, vp, vp]
-        oracle._lib = lib
+        oracle._lib = oracle.bind(ctypes.CDLL(lib_path))
         for fn, args in [(test_golden_head_decay, ()), (test_golden_slot_decay, ()),
+                         (test_golden_router_variants, ("softmax",)),
+                         (test_golden_router_variants, ("sigmoid_norm",)),
+                         (test_selection_counts_match_bincount, ()),
                          (test_topk_tie_rules, ()), (test_window_limit_is_sliding_window, ()),
                          (test_recurrence_matches_quadratic_form, (1, 3, True)),
                          (test_recurrence_matches_quadratic_form, (2, 3, False))]:
