@@ -66,6 +66,17 @@ typedef enum rsm_path {
   RSM_PATH_TENSOR = 2   /* tcgen05/TMEM tensor-core path; RSM_ERR_UNSUPPORTED when not available */
 } rsm_path;
 
+/* Router score of a selected slot (the selected set is the same for every variant: both scores
+ * are monotone in the logit). Raven README "Model Structure" (top-k sigmoid/softmax router) and
+ * "Usage" (router_score 'sigmoid' or 'softmax'); paperlayer.ai summary section 6.2.1 (sigmoid vs
+ * softmax scores) and section 4.1 (the selected weights are normalised to sum to one). */
+typedef enum rsm_router {
+  RSM_ROUTER_SIGMOID = 0,       /* s_i = sigmoid(l_i) (default; the README pseudocode)                 */
+  RSM_ROUTER_SOFTMAX = 1,       /* s_i = e^{l_i} / sum over all M slots of e^{l_j}                    */
+  RSM_ROUTER_SIGMOID_NORM = 2,  /* sigmoid scores divided by their sum over the K selected slots      */
+  RSM_ROUTER_SOFTMAX_NORM = 3   /* softmax scores divided by their sum over the K selected slots      */
+} rsm_router;
+
 enum {
   /* Device-side check of the preconditions: a non-finite logit or a non-finite or positive f is
    * reported as RSM_ERR_NONFINITE by rsm_get_device_status (results are then undefined). */
@@ -90,6 +101,11 @@ enum {
  * ------------------------------------------------------------------------------------------- */
 RSM_API rsm_status rsm_route(const float* logits, int64_t rows, int M, int K, int32_t* idx_out,
                      float* score_out, void* stream);
+
+/* rsm_route with a router variant (score_out holds that variant's scores) and RSM_FLAG_* flags
+ * (RSM_FLAG_VALIDATE reports non-finite logits through rsm_get_device_status). */
+RSM_API rsm_status rsm_route_ex(const float* logits, int64_t rows, int M, int K, rsm_router router,
+                                int flags, int32_t* idx_out, float* score_out, void* stream);
 
 /* ---------------------------------------------------------------------------------------------
  * rsm_forward -- chunked prefill over T tokens.
@@ -127,6 +143,10 @@ typedef struct rsm_forward_args {
   size_t workspace_bytes;
   rsm_path path;
   int flags; /* RSM_FLAG_* */
+  rsm_router router;     /* score of the selected slots (RSM_ROUTER_SIGMOID = 0 by default)        */
+  int32_t* slot_counts;  /* [B,H,M] int32 or NULL: the number of tokens of the call that selected
+                            each slot is ADDED to it (the per-slot counts behind the paper's
+                            "effective sequence length" analysis, paperlayer.ai summary 7.1) */
 } rsm_forward_args;
 
 /* Bytes of device workspace rsm_forward needs for these arguments (0 when none). Depends only on
@@ -199,6 +219,8 @@ typedef struct rsm_decode_args {
   int32_t* idx_out;
   float* score_out;
   int flags; /* RSM_FLAG_* */
+  rsm_router router;     /* score of the selected slots (RSM_ROUTER_SIGMOID = 0 by default)        */
+  int32_t* slot_counts;  /* [B,H,M] int32 or NULL: 1 is added for every slot selected at the step */
 } rsm_decode_args;
 
 RSM_API rsm_status rsm_decode_step(const rsm_decode_args* args, void* stream);

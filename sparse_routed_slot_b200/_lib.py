@@ -16,11 +16,14 @@ RSM_OK, RSM_ERR_INVALID_ARG, RSM_ERR_UNSUPPORTED, RSM_ERR_CUDA, RSM_ERR_NONFINIT
 RSM_F32, RSM_BF16 = 0, 1
 RSM_DECAY_HEAD, RSM_DECAY_SLOT = 0, 1
 RSM_PATH_AUTO, RSM_PATH_SIMT, RSM_PATH_TENSOR = 0, 1, 2
+RSM_ROUTER_SIGMOID, RSM_ROUTER_SOFTMAX, RSM_ROUTER_SIGMOID_NORM, RSM_ROUTER_SOFTMAX_NORM = 0, 1, 2, 3
+ROUTERS = {"sigmoid": RSM_ROUTER_SIGMOID, "softmax": RSM_ROUTER_SOFTMAX,
+           "sigmoid_norm": RSM_ROUTER_SIGMOID_NORM, "softmax_norm": RSM_ROUTER_SOFTMAX_NORM}
 RSM_FLAG_VALIDATE = 1
 RSM_FLAG_TEST_STALL_ROUTING = 256
 
 # Every symbol include/rsm.h declares (the CPU tests check the library exports all of them).
-EXPORTED = ("rsm_route", "rsm_forward_workspace_size", "rsm_forward", "rsm_forward_selected_path",
+EXPORTED = ("rsm_route", "rsm_route_ex", "rsm_forward_workspace_size", "rsm_forward", "rsm_forward_selected_path",
             "rsm_forward_kernel_launches", "rsm_forward_set_profile_events",
             "rsm_decode_step",
             "rsm_status_string", "rsm_last_error", "rsm_get_device_status", "rsm_version",
@@ -36,7 +39,7 @@ class ForwardArgs(ctypes.Structure):
                 ("q", _vp), ("k", _vp), ("v", _vp), ("logits", _vp), ("f", _vp), ("H0", _vp),
                 ("o", _vp), ("HT", _vp), ("idx_out", _vp), ("score_out", _vp),
                 ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t),
-                ("path", _int), ("flags", _int)]
+                ("path", _int), ("flags", _int), ("router", _int), ("slot_counts", _vp)]
 
 
 class DecodeArgs(ctypes.Structure):
@@ -44,7 +47,7 @@ class DecodeArgs(ctypes.Structure):
                 ("qkv_dtype", _int), ("decay", _int),
                 ("q", _vp), ("k", _vp), ("v", _vp), ("logits", _vp), ("f", _vp),
                 ("state", _vp), ("o", _vp), ("idx_out", _vp), ("score_out", _vp),
-                ("flags", _int)]
+                ("flags", _int), ("router", _int), ("slot_counts", _vp)]
 
 
 class RSMError(RuntimeError):
@@ -64,6 +67,8 @@ def load() -> ctypes.CDLL:
         lib = ctypes.CDLL(LIB_PATH)
         lib.rsm_route.argtypes = [_vp, ctypes.c_int64, _int, _int, _vp, _vp, _vp]
         lib.rsm_route.restype = _int
+        lib.rsm_route_ex.argtypes = [_vp, ctypes.c_int64, _int, _int, _int, _int, _vp, _vp, _vp]
+        lib.rsm_route_ex.restype = _int
         lib.rsm_forward_workspace_size.argtypes = [ctypes.POINTER(ForwardArgs)]
         lib.rsm_forward_workspace_size.restype = ctypes.c_size_t
         lib.rsm_forward.argtypes = [ctypes.POINTER(ForwardArgs), _vp]

@@ -34,19 +34,27 @@ def _need(t: torch.Tensor, name: str, dtype=None, shape=None):
         raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
 
 
-def route(logits: torch.Tensor, K: int, scores: bool = True):
-    """TopK routing of fp32 logits [..., M]. Returns (idx int32 [..., K], score fp32 [..., K])."""
+def route(logits: torch.Tensor, K: int, scores: bool = True, router: str = "sigmoid",
+          validate: bool = False):
+    """TopK routing of fp32 logits [..., M]. Returns (idx int32 [..., K], score fp32 [..., K]).
+    router: "sigmoid" (default), "softmax", "sigmoid_norm" or "softmax_norm"."""
     _need(logits, "logits", torch.float32)
     M = logits.shape[-1]
     rows = logits.numel() // M if M else 0
     idx = torch.empty(*logits.shape[:-1], K, dtype=torch.int32, device=logits.device)
     sc = torch.empty(*logits.shape[:-1], K, dtype=torch.float32, device=logits.device) if scores else None
-    _lib.check(_lib.load().rsm_route(_ptr(logits), rows, M, K, _ptr(idx), _ptr(sc),
-                                     _stream(logits.device)))
+    L = _lib.load()
+    if router == "sigmoid" and not validate:
+        _lib.check(L.rsm_route(_ptr(logits), rows, M, K, _ptr(idx), _ptr(sc), _stream(logits.device)))
+    else:
+        _lib.check(L.rsm_route_ex(_ptr(logits), rows, M, K, _lib.ROUTERS[router],
+                                  _lib.RSM_FLAG_VALIDATE if validate else 0, _ptr(idx), _ptr(sc),
+                                  _stream(logits.device)))
     return idx, sc
 
 
-def _forward_args(q, k, v, logits, f, K, H0, o, HT, idx, sc, path, validate) -> _lib.ForwardArgs:
+def _forward_args(q, k, v, logits, f, K, H0, o, HT, idx, sc, path, validate, router="sigmoid",
+                  counts=None) -> _lib.ForwardArgs:
     B, T, H, M = q.shape
     Dv = v.shape[-1]
     if q.dtype not in _DTYPES:
@@ -76,6 +84,10 @@ def _forward_args(q, k, v, logits, f, K, H0, o, HT, idx, sc, path, validate) -> 
     a.score_out = None if sc is None else sc.data_ptr()
     a.path = _PATHS[path]
     a.flags = _lib.RSM_FLAG_VALIDATE if validate else 0
+    a.router = _lib.ROUTERS[router]
+    if counts is not None:
+        _need(counts, "slot_counts", torch.int32, (B, H, M))
+    a.slot_counts = None if counts is None else counts.data_ptr()
     return a
 
 
@@ -103,12 +115,15 @@ def kernel_launches(args: _lib.ForwardArgs) -> int:
 
 
 def forward(q, k, v, logits, f, K: int, H0=None, *, state: bool = True, routing: bool = False,
-            path: str = "auto", validate: bool = False, out=None, workspace=None):
+            path: str = "auto", validate: bool = False, out=None, workspace=None, router: str = "sigmoid",
+            slot_counts=None):
     """Chunked prefill. q, k [B,T,H,M]; v [B,T,H,Dv]; logits [B,T,H,M] fp32; f [B,T,H] or
     [B,T,H,M] fp32; H0 [B,H,M,Dv] fp32 or None.
 
     Returns dict(o [B,T,H,Dv] fp32, HT [B,H,M,Dv] fp32 or None, idx, score [B,T,H,K] or None).
     `out` may supply preallocated tensors under the same keys; `workspace` a uint8 CUDA tensor.
+    `router` picks the score variant; `slot_counts` (int32 [B,H,M]) gets the number of tokens
+    that selected each slot added to it.
     """
     B, T, H, M = q.shape
     Dv = v.shape[-1]
@@ -125,7 +140,7 @@ def forward(q, k, v, logits, f, K: int, H0=None, *, state: bool = True, routing:
     if routing:
         idx = idx if idx is not None else torch.empty(B, T, H, K, dtype=torch.int32, device=dev)
         sc = sc if sc is not None else torch.empty(B, T, H, K, dtype=torch.float32, device=dev)
-    a = _forward_args(q, k, v, logits, f, K, H0, o, HT, idx, sc, path, validate)
+    a = _forward_args(q, k, v, logits, f, K, H0, o, HT, idx, sc, path, validate, router, slot_counts)
     need = workspace_bytes(a)
     if need:
         if workspace is None or workspace.numel() < need:
@@ -136,7 +151,7 @@ def forward(q, k, v, logits, f, K: int, H0=None, *, state: bool = True, routing:
 
 
 def decode_step(q, k, v, logits, f, K: int, state, *, routing: bool = False, validate: bool = False,
-                o=None, flags: int = 0):
+                o=None, flags: int = 0, router: str = "sigmoid", slot_counts=None):
     """One token per (b,h). q, k [B,H,M]; v [B,H,Dv]; logits [B,H,M]; f [B,H] or [B,H,M];
     state [B,H,M,Dv] fp32 updated in place. Returns dict(o [B,H,Dv] fp32, idx, score).
     `flags` are extra RSM_FLAG_* bits passed through unchanged."""
@@ -170,6 +185,10 @@ def decode_step(q, k, v, logits, f, K: int, state, *, routing: bool = False, val
     a.idx_out = None if idx is None else idx.data_ptr()
     a.score_out = None if sc is None else sc.data_ptr()
     a.flags = (_lib.RSM_FLAG_VALIDATE if validate else 0) | flags
+    a.router = _lib.ROUTERS[router]
+    if slot_counts is not None:
+        _need(slot_counts, "slot_counts", torch.int32, (B, H, M))
+    a.slot_counts = None if slot_counts is None else slot_counts.data_ptr()
     _lib.check(_lib.load().rsm_decode_step(ctypes.byref(a), _stream(dev)))
     return {"o": o, "idx": idx, "score": sc}
 

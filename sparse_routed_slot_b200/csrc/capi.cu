@@ -33,6 +33,11 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 bool pow2_slots(int M) { return M == 32 || M == 64 || M == 128 || M == 256; }
 
+bool valid_router(rsm_router r) {
+  return r == RSM_ROUTER_SIGMOID || r == RSM_ROUTER_SOFTMAX || r == RSM_ROUTER_SIGMOID_NORM ||
+         r == RSM_ROUTER_SOFTMAX_NORM;
+}
+
 // Shared size checks. Returns RSM_OK or an error with g_err set.
 rsm_status check_sizes(int M, int K, int Dv) {
   if (M < 1 || K < 1 || Dv < 1) return fail(RSM_ERR_INVALID_ARG, "M, K and Dv must be >= 1");
@@ -64,6 +69,7 @@ rsm_status check_forward(const rsm_forward_args* a) {
     return fail(RSM_ERR_INVALID_ARG, "unknown decay %d", (int)a->decay);
   if (a->path != RSM_PATH_AUTO && a->path != RSM_PATH_SIMT && a->path != RSM_PATH_TENSOR)
     return fail(RSM_ERR_INVALID_ARG, "unknown path %d", (int)a->path);
+  if (!valid_router(a->router)) return fail(RSM_ERR_INVALID_ARG, "unknown router %d", (int)a->router);
   if ((int64_t)a->B * a->H > (int64_t)0x7fffffff)
     return fail(RSM_ERR_UNSUPPORTED, "B*H too large");
   const bool tokens = (int64_t)a->B * a->T * a->H > 0;
@@ -79,6 +85,7 @@ rsm_status check_forward(const rsm_forward_args* a) {
   RSM_OPTIONAL_PTR(a->HT, "HT");
   RSM_OPTIONAL_PTR(a->idx_out, "idx_out");
   RSM_OPTIONAL_PTR(a->score_out, "score_out");
+  RSM_OPTIONAL_PTR(a->slot_counts, "slot_counts");
   if (a->path == RSM_PATH_TENSOR && !rsm::prefill_tc_supported(*a))
     return fail(RSM_ERR_UNSUPPORTED,
                 "the tensor-core path needs bf16 q/k/v, M = Dv = 128 and K <= 32");
@@ -126,18 +133,25 @@ const char* rsm_last_error(void) { return g_err; }
 
 int rsm_version(void) { return 100; }
 
-rsm_status rsm_route(const float* logits, int64_t rows, int M, int K, int32_t* idx_out,
-                     float* score_out, void* stream) {
+rsm_status rsm_route_ex(const float* logits, int64_t rows, int M, int K, rsm_router router, int flags,
+                        int32_t* idx_out, float* score_out, void* stream) {
   g_err[0] = 0;
   if (rows < 0) return fail(RSM_ERR_INVALID_ARG, "rows must be >= 0");
   rsm_status s = check_sizes(M, K, 4);
   if (s != RSM_OK) return s;
+  if (!valid_router(router)) return fail(RSM_ERR_INVALID_ARG, "unknown router %d", (int)router);
   if (rows == 0) return RSM_OK;
   RSM_REQUIRE_PTR(logits, "logits");
   RSM_REQUIRE_PTR(idx_out, "idx_out");
   RSM_OPTIONAL_PTR(score_out, "score_out");
-  cudaError_t e = rsm::launch_route(logits, rows, M, K, idx_out, score_out, 0, static_cast<cudaStream_t>(stream));
+  cudaError_t e = rsm::launch_route(logits, rows, M, K, idx_out, score_out, (int)router,
+                                    (flags & RSM_FLAG_VALIDATE) ? 1 : 0, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? RSM_OK : cuda_fail(e, "rsm_route launch");
+}
+
+rsm_status rsm_route(const float* logits, int64_t rows, int M, int K, int32_t* idx_out,
+                     float* score_out, void* stream) {
+  return rsm_route_ex(logits, rows, M, K, RSM_ROUTER_SIGMOID, 0, idx_out, score_out, stream);
 }
 
 size_t rsm_forward_workspace_size(const rsm_forward_args* a) {
@@ -216,6 +230,7 @@ rsm_status rsm_decode_step(const rsm_decode_args* a, void* stream) {
     return fail(RSM_ERR_INVALID_ARG, "unknown qkv_dtype %d", (int)a->qkv_dtype);
   if (a->decay != RSM_DECAY_HEAD && a->decay != RSM_DECAY_SLOT)
     return fail(RSM_ERR_INVALID_ARG, "unknown decay %d", (int)a->decay);
+  if (!valid_router(a->router)) return fail(RSM_ERR_INVALID_ARG, "unknown router %d", (int)a->router);
   if ((int64_t)a->B * a->H == 0) return RSM_OK;
   if ((int64_t)a->B * a->H > (int64_t)0x7fffffff) return fail(RSM_ERR_UNSUPPORTED, "B*H too large");
   RSM_REQUIRE_PTR(a->q, "q");
@@ -227,6 +242,7 @@ rsm_status rsm_decode_step(const rsm_decode_args* a, void* stream) {
   RSM_REQUIRE_PTR(a->o, "o");
   RSM_OPTIONAL_PTR(a->idx_out, "idx_out");
   RSM_OPTIONAL_PTR(a->score_out, "score_out");
+  RSM_OPTIONAL_PTR(a->slot_counts, "slot_counts");
   cudaError_t e = rsm::launch_decode(*a, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? RSM_OK : cuda_fail(e, "rsm_decode_step launch");
 }

@@ -52,6 +52,16 @@ RSM_DEV uint32_t order_key(float x) {
 RSM_DEV float sigmoid_f32(float x) { return 1.0f / (1.0f + expf(-x)); }
 
 // Warp-wide sum / max / min by xor-shuffle butterflies (every lane gets the result).
+RSM_DEV float warp_sum_f(float v) {
+#pragma unroll
+  for (int d = 16; d >= 1; d >>= 1) v += __shfl_xor_sync(kFull, v, d);
+  return v;
+}
+RSM_DEV float warp_max_f(float v) {
+#pragma unroll
+  for (int d = 16; d >= 1; d >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, d));
+  return v;
+}
 RSM_DEV int warp_sum(int v) {
 #pragma unroll
   for (int d = 16; d >= 1; d >>= 1) v += __shfl_xor_sync(kFull, v, d);
@@ -350,6 +360,49 @@ RSM_DEV uint32_t warp_select_guess_rows(const float (&x)[NR][M / 32], int K, flo
     if (ok & (1u << r)) guess = t[r];
   }
   return ok;
+}
+
+// Router variant scores of a row held by a warp (lane: E logits x[e]; sel: the lane's selected
+// elements, bit e). s[e] is the score of each selected element, 0 elsewhere:
+//   RSM_ROUTER_SIGMOID       sigmoid(x)
+//   RSM_ROUTER_SOFTMAX       e^{x - max} / sum over the whole row of e^{x_j - max}
+//   *_NORM                   the above divided by its sum over the selected elements
+// Every lane of the warp must call it (warp reductions).
+template <int E>
+RSM_DEV void warp_router_scores(const float (&x)[E], uint32_t sel, int router, float (&s)[E]) {
+  if (router & RSM_ROUTER_SOFTMAX) {
+    float mx = x[0];
+#pragma unroll
+    for (int e = 1; e < E; ++e) mx = fmaxf(mx, x[e]);
+    mx = warp_max_f(mx);
+    float z = 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      s[e] = expf(x[e] - mx);
+      z += s[e];
+    }
+    const float rz = 1.0f / warp_sum_f(z);
+#pragma unroll
+    for (int e = 0; e < E; ++e) s[e] = (sel >> e) & 1u ? s[e] * rz : 0.f;
+  } else {
+#pragma unroll
+    for (int e = 0; e < E; ++e) s[e] = (sel >> e) & 1u ? sigmoid_f32(x[e]) : 0.f;
+  }
+  if (router & 2) {  // normalised over the selected slots
+    float t = 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) t += s[e];
+    const float rt = 1.0f / warp_sum_f(t);
+#pragma unroll
+    for (int e = 0; e < E; ++e) s[e] *= rt;
+  }
+}
+
+// rank[e] = r for element e (unrolled select, so that a runtime e keeps the array in registers).
+template <int E>
+RSM_DEV void set_rank(int (&rank)[E], int e, int r) {
+#pragma unroll
+  for (int e2 = 0; e2 < E; ++e2) rank[e2] = (e2 == e) ? r : rank[e2];
 }
 
 // Loads the lane's E contiguous logits of a row.

@@ -10,7 +10,8 @@
 //   item) and splits the work among three warp roles that meet at mbarriers in shared memory:
 //     producer  (1 thread)   streams the state of its items, block by block (32 KB of rows per
 //                            block), through a ring of kStages buffers with cp.async.bulk;
-//     routers   (kRouters warps) run ahead of the consumers: TopK of the item's logits, then the
+//     routers   (kRouters warps) run ahead of the consumers: TopK of the item's logits, the
+//                            router scores s (sigmoid or softmax, optionally normalised), then the
 //                            decay a = e^{s f} and write weight w = k (1 - a) of every slot (a = 1,
 //                            w = 0 off the selection), q and v, into a ring of routing slots;
 //     consumers (8 warps)    apply the update to the selected rows of each block, store those rows,
@@ -185,17 +186,23 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(rsm_decode_args a) 
       }
       int32_t* io = a.idx_out ? a.idx_out + pair * K : nullptr;
       float* so = a.score_out ? a.score_out + pair * K : nullptr;
-      const uint32_t sel = warp_topk<M>(x, K, lane, [&](int rank, int slot_i, int e) {
-        if (io) io[rank] = slot_i;
-        if (so) so[rank] = sigmoid_f32(x[e]);
+      int32_t* cnt = a.slot_counts ? a.slot_counts + pair * M : nullptr;
+      int rank[E];
+      const uint32_t sel = warp_topk<M>(x, K, lane, [&](int rk, int slot_i, int e) {
+        if (io) io[rk] = slot_i;
+        if (cnt) cnt[slot_i] += 1;  // one router warp per (b,h): no other writer
+        set_rank<E>(rank, e, rk);
       });
+      float sc[E];
+      warp_router_scores<E>(x, sel, a.router, sc);
 #pragma unroll
       for (int e = 0; e < E; ++e) {
         const int i = lane * E + e;
         if (sel & (1u << e)) {
-          const float lam = sigmoid_f32(x[e]) * fv[e];  // log of the decay, <= 0
-          sa[i] = -expf(lam);                           // sign bit: selected
-          sw[i] = kv[e] * (-expm1f(lam));               // k_i (1 - a_i)
+          if (so) so[rank[e]] = sc[e];
+          const float lam = sc[e] * fv[e];   // log of the decay, <= 0
+          sa[i] = -expf(lam);                // sign bit: selected
+          sw[i] = kv[e] * (-expm1f(lam));    // k_i (1 - a_i)
         } else {
           sa[i] = 1.f;
           sw[i] = 0.f;

@@ -9,7 +9,7 @@
 namespace rsm {
 
 cudaError_t launch_route(const float* logits, int64_t rows, int M, int K, int32_t* idx_out,
-                         float* score_out, int validate, cudaStream_t stream);
+                         float* score_out, int router, int validate, cudaStream_t stream);
 
 // Routing records for the tensor prefill (route_rec.cu, M = 128, K <= 32) over rows given as
 // [B, T, H]: route_record_bytes(K) bytes per row, rows in [B, H, T] order; also the ranked
@@ -17,8 +17,13 @@ cudaError_t launch_route(const float* logits, int64_t rows, int M, int K, int32_
 bool route_records_supported(int M, int K);
 int route_record_bytes(int K);
 cudaError_t launch_route_records(const float* logits, const float* f, const void* k, int64_t B, int64_t T,
-                                 int64_t H, int M, int K, int decay_slot, int validate, unsigned char* rec,
-                                 int32_t* idx_out, float* score_out, cudaStream_t stream);
+                                 int64_t H, int M, int K, int decay_slot, int router, int validate,
+                                 unsigned char* rec, int32_t* idx_out, float* score_out, int32_t* counts,
+                                 cudaStream_t stream);
+
+// Adds the per-slot selection counts of routing records ([pairs, T] rows) to counts[pairs][128].
+cudaError_t launch_record_counts(const unsigned char* rec, int64_t pairs, int64_t T, int K, int32_t* counts,
+                                 cudaStream_t stream);
 
 cudaError_t launch_decode(const rsm_decode_args& a, cudaStream_t stream);
 

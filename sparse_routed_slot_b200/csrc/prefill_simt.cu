@@ -116,17 +116,23 @@ __global__ void __launch_bounds__(kThreads) prefill_simt_kernel(rsm_forward_args
         }
         int32_t* io = (route_owner && a.idx_out) ? a.idx_out + row * K : nullptr;
         float* so = (route_owner && a.score_out) ? a.score_out + row * K : nullptr;
+        int32_t* cnt = (route_owner && a.slot_counts) ? a.slot_counts + (int64_t)pair * M : nullptr;
+        int rank[E];
         const uint32_t sel = warp_topk<M>(x, K, lane, [&](int r, int slot, int e) {
           s_sidx[t * M + r] = (unsigned char)slot;
           if (io) io[r] = slot;
-          if (so) so[r] = sigmoid_f32(x[e]);
+          if (cnt) atomicAdd(cnt + slot, 1);
+          set_rank<E>(rank, e, r);
         });
+        float sc[E];
+        warp_router_scores<E>(x, sel, a.router, sc);
 #pragma unroll
         for (int e = 0; e < E; ++e) {
           const int i = lane * E + e;
           s_q[t * M + i] = In<TIn>::ld(q + row * M + i);
           if (sel & (1u << e)) {
-            const float lam = sigmoid_f32(x[e]) * fv[e];
+            if (so) so[rank[e]] = sc[e];
+            const float lam = sc[e] * fv[e];
             s_g[t * M + i] = lam;
             s_w[t * M + i] = In<TIn>::ld(k + row * M + i) * (-expm1f(lam));
             s_touch[i] = 1;

@@ -1262,7 +1262,7 @@ size_t prefill_tc_workspace_bytes(const rsm_forward_args& a) {
 
 int prefill_tc_launches(const rsm_forward_args& a) {
   if (!prefill_tc_supported(a) || a.T == 0) return 0;
-  return plan_for(a, sm_count()).nseg > 1 ? 4 : 2;
+  return (plan_for(a, sm_count()).nseg > 1 ? 4 : 2) + (a.slot_counts ? 1 : 0);
 }
 
 cudaError_t launch_prefill_tc(const rsm_forward_args& a, cudaStream_t stream) {
@@ -1272,8 +1272,13 @@ cudaError_t launch_prefill_tc(const rsm_forward_args& a, cudaStream_t stream) {
   char* ws = static_cast<char*>(a.workspace);
   unsigned char* rec = reinterpret_cast<unsigned char*>(ws + wl.rec);
   cudaError_t e = launch_route_records(a.logits, a.f, a.k, a.B, a.T, a.H, a.M, a.K, a.decay == RSM_DECAY_SLOT,
-                                       (a.flags & RSM_FLAG_VALIDATE) != 0, rec, a.idx_out, a.score_out, stream);
+                                       (int)a.router, (a.flags & RSM_FLAG_VALIDATE) != 0, rec, a.idx_out,
+                                       a.score_out, a.slot_counts, stream);
   if (e == cudaSuccess) e = profile_mark(stream);
+  if (e == cudaSuccess && a.slot_counts) {
+    e = launch_record_counts(rec, (int64_t)a.B * a.H, a.T, a.K, a.slot_counts, stream);
+    if (e == cudaSuccess) e = profile_mark(stream);
+  }
   if (e != cudaSuccess) return e;
   Maps maps;
   if (!make_map(&maps.v, a.v, a.B, a.T, a.H, kDV, false, kC)) return cudaErrorInvalidValue;

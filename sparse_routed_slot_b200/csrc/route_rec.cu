@@ -7,7 +7,8 @@
 //   record (route_record_bytes(K) = 9 * KP bytes, KP = 16 for K <= 16 else 32; rows in
 //   [B, H, T] order, so the records of one (b,h) stream are contiguous along time):
 //     uint8  slot[KP]   the selected slots (entries >= K: 0)
-//     float  lam[KP]    lam = sigmoid(logit[slot]) * f, the log of the slot's decay (<= 0)
+//     float  lam[KP]    lam = s * f, the log of the slot's decay (<= 0), s the router score
+//                       (sigmoid or softmax of the logit, optionally normalised over the K)
 //     float  w[KP]      w = k[slot] * (1 - e^lam), the slot's write weight
 //   Entries are in rank order (logit descending, slot ascending) except that logits agreeing in
 //   their upper 25 key bits may be listed in slot order; when no ranked output is requested and
@@ -118,15 +119,14 @@ struct Rows {
   const float* f;
   const uint16_t* k;  // bf16 bits
   int64_t B, T, H;
-  int K, decay_slot;
+  int K, decay_slot, router;
   unsigned char* rec;
   int32_t* idx_out;
   float* score_out;
 };
 
-// The score, lam and w of one selected slot of input row `ir` (x = its logit).
-RSM_DEV void entry_values(const Rows& R, int64_t ir, int slot, float x, float fh, float& s, float& lam, float& w) {
-  s = sigmoid_f32(x);
+// lam and w of one selected slot of input row `ir`, from its router score s.
+RSM_DEV void entry_values(const Rows& R, int64_t ir, int slot, float s, float fh, float& lam, float& w) {
   const float fv = R.decay_slot ? __ldg(R.f + ir * kRM + slot) : fh;
   lam = s * fv;
   const float kv = __uint_as_float((uint32_t)__ldg(R.k + ir * kRM + slot) << 16);
@@ -255,28 +255,56 @@ __global__ void __launch_bounds__(kThreads) route_rec_kernel(const Rows R) {
     int32_t* io = R.idx_out ? R.idx_out + ir * K : nullptr;
     float* so = R.score_out ? R.score_out + ir * K : nullptr;
 
+    // softmax scores need the row's maximum and normalising sum (each lane of a pair: its half)
+    float smax = 0.f, rsum = 1.f;
+    if (R.router & RSM_ROUTER_SOFTMAX) {
+      float mx = -3.402823466e38f;
+#pragma unroll 4
+      for (int i = 0; i < kRM / 2; ++i) mx = fmaxf(mx, xr[half * (kRM / 2) + i]);
+      smax = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
+      float z = 0.f;
+#pragma unroll 4
+      for (int i = 0; i < kRM / 2; ++i) z += expf(xr[half * (kRM / 2) + i] - smax);
+      rsum = 1.0f / (z + __shfl_xor_sync(kFull, z, 1));
+    }
+
+    constexpr int KH = KP / 2;
+    uint32_t sw[KH / 4];
+    float sc[KH];
+    int slots[KH];
+#pragma unroll
+    for (int i = 0; i < KH / 4; ++i) sw[i] = 0u;
+#pragma unroll
+    for (int q = 0; q < KH; ++q) {
+      // sorted: lane `half` takes rank positions half*KH + q; unsorted, the partner's array is
+      // this lane's reversed, so each lane takes its own first half
+      const uint32_t key = (sorted && half) ? top[KH + q] : top[q];
+      slots[q] = 127 - (int)(key & 0x7Fu);
+      const float xq = xr[slots[q]];
+      sc[q] = (half * KH + q >= K) ? 0.f : (R.router & RSM_ROUTER_SOFTMAX) ? expf(xq - smax) * rsum : sigmoid_f32(xq);
+    }
+    if (R.router & 2) {  // normalised over the row's K selected slots (both lanes of the pair)
+      float t = 0.f;
+#pragma unroll
+      for (int q = 0; q < KH; ++q) t += sc[q];
+      const float rt = 1.0f / (t + __shfl_xor_sync(kFull, t, 1));
+#pragma unroll
+      for (int q = 0; q < KH; ++q) sc[q] *= rt;
+    }
     if (live && !exact) {
       // ---- entries in rank order from the sorted keys; each lane of the pair computes half
-      constexpr int KH = KP / 2;
-      uint32_t sw[KH / 4];
       float lam[KH], wv[KH];
-#pragma unroll
-      for (int i = 0; i < KH / 4; ++i) sw[i] = 0u;
 #pragma unroll
       for (int q = 0; q < KH; ++q) {
         const int r = half * KH + q;
-        // sorted: lane `half` takes rank positions half*KH + q; unsorted, the partner's array is
-        // this lane's reversed, so each lane takes its own first half
-        const uint32_t key = (sorted && half) ? top[KH + q] : top[q];
         lam[q] = 0.f;
         wv[q] = 0.f;
         if (r < K) {
-          const int slot = 127 - (int)(key & 0x7Fu);
+          const int slot = slots[q];
           sw[q / 4] |= (uint32_t)slot << (8 * (q % 4));
-          float sc;
-          entry_values(R, ir, slot, xr[slot], fh, sc, lam[q], wv[q]);
+          entry_values(R, ir, slot, sc[q], fh, lam[q], wv[q]);
           if (io) io[r] = slot;
-          if (so) so[r] = sc;
+          if (so) so[r] = sc[q];
         }
       }
 #pragma unroll
@@ -310,15 +338,26 @@ __global__ void __launch_bounds__(kThreads) route_rec_kernel(const Rows R) {
       unsigned char* rpw = R.rec + pw * (int64_t)(9 * KP);
       int32_t* iow = R.idx_out ? R.idx_out + irw * K : nullptr;
       float* sow = R.score_out ? R.score_out + irw * K : nullptr;
-      warp_topk<kRM>(x4, K, lane, [&](int rk, int slot, int e) {
-        float sc, lm, wvv;
-        entry_values(R, irw, slot, x4[e], fhw, sc, lm, wvv);
+      int rank[4] = {0, 0, 0, 0};
+      int* rank_p = rank;  // a rare path: local memory is fine here
+      const uint32_t sel = warp_topk<kRM>(x4, K, lane, [&](int rk, int slot, int e) {
         rpw[rk] = (unsigned char)slot;
-        reinterpret_cast<float*>(rpw + KP)[rk] = lm;
-        reinterpret_cast<float*>(rpw + 5 * KP)[rk] = wvv;
         if (iow) iow[rk] = slot;
-        if (sow) sow[rk] = sc;
+        rank_p[e] = rk;
       });
+      float scw[4];
+      const float(&x4c)[4] = x4;  // (binding first sidesteps a front-end crash of this nvcc)
+      warp_router_scores(x4c, sel, (int)R.router, scw);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if ((sel >> e) & 1u) {
+          float lm, wvv;
+          entry_values(R, irw, lane * (kRM / 32) + e, scw[e], fhw, lm, wvv);
+          reinterpret_cast<float*>(rpw + KP)[rank[e]] = lm;
+          reinterpret_cast<float*>(rpw + 5 * KP)[rank[e]] = wvv;
+          if (sow) sow[rank[e]] = scw[e];
+        }
+      }
       if (lane < KP - K) {  // padding entries
         rpw[K + lane] = 0;
         reinterpret_cast<float*>(rpw + KP)[K + lane] = 0.f;
@@ -345,15 +384,45 @@ cudaError_t launch_n(const Rows& R, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+// Per-slot selection counts from the records: block (pair, part) counts the selected slots of a
+// range of the pair's rows in shared memory and adds them to counts[pair][slot].
+__global__ void __launch_bounds__(256) record_counts_kernel(const unsigned char* __restrict__ rec, int64_t T,
+                                                            int K, int rec_bytes, int rows_per_block,
+                                                            int32_t* __restrict__ counts) {
+  __shared__ int hist[kRM];
+  const int pair = blockIdx.y;
+  for (int i = threadIdx.x; i < kRM; i += blockDim.x) hist[i] = 0;
+  __syncthreads();
+  const int64_t t0 = (int64_t)blockIdx.x * rows_per_block;
+  const int64_t t1 = min(T, t0 + rows_per_block);
+  for (int64_t t = t0 + threadIdx.x; t < t1; t += blockDim.x) {
+    const unsigned char* r = rec + ((int64_t)pair * T + t) * rec_bytes;
+    for (int j = 0; j < K; ++j) atomicAdd(&hist[r[j]], 1);
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < kRM; i += blockDim.x)
+    if (hist[i]) atomicAdd(counts + (int64_t)pair * kRM + i, hist[i]);
+}
+
 }  // namespace
 
 int route_record_bytes(int K) { return 9 * (K <= 16 ? 16 : 32); }
 
+cudaError_t launch_record_counts(const unsigned char* rec, int64_t pairs, int64_t T, int K, int32_t* counts,
+                                 cudaStream_t stream) {
+  if (pairs == 0 || T == 0) return cudaSuccess;
+  const int rows_per_block = 4096;
+  dim3 grid((unsigned)((T + rows_per_block - 1) / rows_per_block), (unsigned)pairs);
+  record_counts_kernel<<<grid, 256, 0, stream>>>(rec, T, K, route_record_bytes(K), rows_per_block, counts);
+  return cudaGetLastError();
+}
+
 bool route_records_supported(int M, int K) { return M == kRM && K >= 1 && K <= 32; }
 
 cudaError_t launch_route_records(const float* logits, const float* f, const void* k, int64_t B, int64_t T,
-                                 int64_t H, int M, int K, int decay_slot, int validate, unsigned char* rec,
-                                 int32_t* idx_out, float* score_out, cudaStream_t stream) {
+                                 int64_t H, int M, int K, int decay_slot, int router, int validate,
+                                 unsigned char* rec, int32_t* idx_out, float* score_out, int32_t* counts,
+                                 cudaStream_t stream) {
   if (!route_records_supported(M, K) || !rec || !f || !k) return cudaErrorInvalidValue;
   if (B * T * H == 0) return cudaSuccess;
   Rows R;
@@ -363,11 +432,15 @@ cudaError_t launch_route_records(const float* logits, const float* f, const void
   R.B = B; R.T = T; R.H = H;
   R.K = K;
   R.decay_slot = decay_slot;
+  R.router = router;
   R.rec = rec;
   R.idx_out = idx_out;
   R.score_out = score_out;
-  if (K <= 16) return validate ? launch_n<16, true>(R, stream) : launch_n<16, false>(R, stream);
-  return validate ? launch_n<32, true>(R, stream) : launch_n<32, false>(R, stream);
+  cudaError_t e;
+  if (K <= 16) e = validate ? launch_n<16, true>(R, stream) : launch_n<16, false>(R, stream);
+  else e = validate ? launch_n<32, true>(R, stream) : launch_n<32, false>(R, stream);
+  (void)counts;  // counted by launch_record_counts, a launch of its own
+  return e;
 }
 
 }  // namespace rsm

@@ -51,16 +51,18 @@ def test_struct_layouts_match_c(lib, tmp_path):
     prog = tmp_path / "sizes.c"
     prog.write_text(
         '#include <stdio.h>\n#include <stddef.h>\n#include "rsm.h"\n'
-        "int main(void){printf(\"%zu %zu %zu %zu %zu %zu\\n\", sizeof(rsm_forward_args),"
+        "int main(void){printf(\"%zu %zu %zu %zu %zu %zu %zu %zu %zu %zu\\n\", sizeof(rsm_forward_args),"
         " offsetof(rsm_forward_args, workspace_bytes), offsetof(rsm_forward_args, flags),"
-        " sizeof(rsm_decode_args), offsetof(rsm_decode_args, state), offsetof(rsm_decode_args, flags));"
+        " offsetof(rsm_forward_args, router), offsetof(rsm_forward_args, slot_counts),"
+        " sizeof(rsm_decode_args), offsetof(rsm_decode_args, state), offsetof(rsm_decode_args, flags),"
+        " offsetof(rsm_decode_args, router), offsetof(rsm_decode_args, slot_counts));"
         "return 0;}\n")
     exe = tmp_path / "sizes"
     subprocess.check_call(["gcc", "-I", os.path.join(ROOT, "include"), "-o", str(exe), str(prog)])
     c = list(map(int, subprocess.check_output([str(exe)]).split()))
     F, D = lib.ForwardArgs, lib.DecodeArgs
-    py = [ctypes.sizeof(F), F.workspace_bytes.offset, F.flags.offset,
-          ctypes.sizeof(D), D.state.offset, D.flags.offset]
+    py = [ctypes.sizeof(F), F.workspace_bytes.offset, F.flags.offset, F.router.offset, F.slot_counts.offset,
+          ctypes.sizeof(D), D.state.offset, D.flags.offset, D.router.offset, D.slot_counts.offset]
     assert c == py
 
 
