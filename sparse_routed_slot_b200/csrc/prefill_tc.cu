@@ -163,6 +163,19 @@ RSM_DEV bool bar_rows_or(bool flag) {
 }
 RSM_DEV void bar_rows() { asm volatile("bar.sync 1, %0;" ::"n"(kRThreads) : "memory"); }
 RSM_DEV void bar_epi() { asm volatile("bar.sync 2, %0;" ::"n"(kEpiThreads) : "memory"); }
+// Barrier among the epilogue warps that ORs a flag over them (every epilogue thread sees the same).
+RSM_DEV bool bar_epi_or(bool flag) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.or.pred p, 2, %2, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)flag), "n"(kEpiThreads)
+      : "memory");
+  return r != 0;
+}
 
 // Position of one chunk in the CTA's work list.
 struct Chunk {
@@ -545,13 +558,18 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     }
   } else if (warp == kIssuerWarp) {
     // =========================================================================== MMA issuer
-    if (lane == 0) {
+    // The whole warp runs the issuer's loop, so that its descriptors and addresses are
+    // warp-uniform values; lane 0 alone issues the copies, the MMAs and their commits.
+    const bool leader = lane == 0;
+    {
       uint32_t n = 0, n_tma = 0;
       auto load_v = [&](const Walker& at, uint32_t j) {  // v tile of the walker's chunk, as chunk j
         if (!at.valid(items)) return;
         const Chunk c = at.get(p);
-        tc::mbar_arrive_expect_tx(&bar_tma[j & 1], kC * kDV * 2);
-        tc::tma_load_4d(sRawV + (j & 1) * (kC * kDV * 2), &maps.v, &bar_tma[j & 1], 0, c.h, c.c0, c.b);
+        if (leader) {
+          tc::mbar_arrive_expect_tx(&bar_tma[j & 1], kC * kDV * 2);
+          tc::tma_load_4d(sRawV + (j & 1) * (kC * kDV * 2), &maps.v, &bar_tma[j & 1], 0, c.h, c.c0, c.b);
+        }
         ++n_tma;
       };
       {
@@ -575,22 +593,22 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       auto mma_s = [&](uint64_t dQn) {  // S = Qh Wh^T
 #pragma unroll
         for (int j = 0; j < kM / 8; ++j)
-          tc::mma_tf32_ss(tb + kColS, dQn + kstep(kC, j), dW + kstep(kC, j), kIdS, j > 0);
+          if (leader) tc::mma_tf32_ss(tb + kColS, dQn + kstep(kC, j), dW + kstep(kC, j), kIdS, j > 0);
       };
       auto mma_read = [&](uint32_t ob, uint64_t dQn) {  // O^T = H^T Qh^T (state read from TMEM)
 #pragma unroll
         for (int j = 0; j < kM / 8; ++j)
-          tc::mma_tf32_ts(tb + kColO + ob, tb + kColHr + 8 * j, dQn + kstep(kC, j), kIdO, j > 0);
+          if (leader) tc::mma_tf32_ts(tb + kColO + ob, tb + kColHr + 8 * j, dQn + kstep(kC, j), kIdO, j > 0);
       };
       auto mma_carry = [&](uint32_t col, bool acc) {  // H^T += V^T Wh, or U^T = V^T Wh
 #pragma unroll
         for (int j = 0; j < kC / 8; ++j)
-          tc::mma_tf32_ss(tb + col, dVt + kstep(kM, j), dWt + kstep(kM, j), kIdC, (acc || j > 0) ? 1u : 0u);
+          if (leader) tc::mma_tf32_ss(tb + col, dVt + kstep(kM, j), dWt + kstep(kM, j), kIdC, (acc || j > 0) ? 1u : 0u);
       };
       auto mma_av = [&](uint32_t ob) {  // O^T += V^T A^T
 #pragma unroll
         for (int j = 0; j < kC / 8; ++j)
-          tc::mma_tf32_ss(tb + kColO + ob, dVt + kstep(kDV, j), dA + kstep(kC, j), kIdO, 1);
+          if (leader) tc::mma_tf32_ss(tb + kColO + ob, dVt + kstep(kDV, j), dA + kstep(kC, j), kIdO, 1);
       };
       bool prev_exact = false;
       for (; wk.valid(items) && !*abort_flag; ++n, wk.next(p, items)) {
@@ -604,7 +622,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         }
         const uint64_t dQn = dQ + (uint64_t)(((n & 1) * 32768) >> 4);  // this chunk's Qh buffer
         if (fast) mma_s(dQn);
-        tc::mma_commit(&bar_s);  // every main-pass chunk: tells the epilogue the chunk is ready
+        if (leader) tc::mma_commit(&bar_s);  // every main-pass chunk: tells the epilogue the chunk is ready
         wait_or_abort(&bar_h, n & 1, abort_flag);  // state ready
         if (n >= 2) wait_or_abort(&bar_of[n & 1], ((n - 2) >> 1) & 1, abort_flag);  // O buffer free
         tc::tmem_fence_after();
@@ -619,16 +637,16 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
           load_v(nx, n + 2);
         }
         mma_carry(fast ? kColH : kColU, fast);
-        tc::mma_commit(&bar_t);
+        if (leader) tc::mma_commit(&bar_t);
         wait_or_abort(&bar_a, n & 1, abort_flag);
         tc::tmem_fence_after();
         mma_av(ob);
-        tc::mma_commit(&bar_o);
+        if (leader) tc::mma_commit(&bar_o);
         prev_exact = !fast;
       }
       // no MMA or tile load may still be running when the CTA releases its memory (a barrier of
       // its own: another phase of bar_o could overtake the epilogue's last wait on it)
-      tc::mma_commit(&bar_fin);
+      if (leader) tc::mma_commit(&bar_fin);
       tc::mbar_wait(&bar_fin, 0);
       for (uint32_t j = n; j < n_tma; ++j) tc::mbar_wait(&bar_tma[j & 1], (j >> 1) & 1);
     }
@@ -660,7 +678,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       mbar_arrive(&bar_h);  // phase 0: the first chunk's state
     }
     uint32_t n = 0;
-    for (; wk.valid(items) && !*abort_flag; ++n, wk.next(p, items)) {
+    for (; wk.valid(items); ++n, wk.next(p, items)) {
+      if (bar_epi_or(*abort_flag != 0)) break;  // the epilogue warps leave together (named barriers)
       const Chunk ck = wk.get(p);
       const float* Dn = sDc + (n & 1) * kM;
       wait_or_abort(&bar_s, n & 1, abort_flag);
@@ -1041,13 +1060,18 @@ __global__ void __launch_bounds__(kSumThreads, 1) segment_summary_kernel(const _
     }
   } else if (warp == kIssuerWarp) {
     // =========================================================================== MMA issuer
-    if (lane == 0) {
+    // The whole warp runs the issuer's loop, so that its descriptors and addresses are
+    // warp-uniform values; lane 0 alone issues the copies, the MMAs and their commits.
+    const bool leader = lane == 0;
+    {
       uint32_t n = 0, n_tma = 0, n_items = 0;
       auto load_v = [&](const SumWalker& at, uint32_t j) {  // v tile of the walker's chunk, as chunk j
         if (!at.valid(items)) return;
         const Chunk c = at.get(p);
-        tc::mbar_arrive_expect_tx(&bar_tma[j & 1], kC * kDV * 2);
-        tc::tma_load_4d(sRawV + (j & 1) * (kC * kDV * 2), &maps.v, &bar_tma[j & 1], 0, c.h, c.c0, c.b);
+        if (leader) {
+          tc::mbar_arrive_expect_tx(&bar_tma[j & 1], kC * kDV * 2);
+          tc::tma_load_4d(sRawV + (j & 1) * (kC * kDV * 2), &maps.v, &bar_tma[j & 1], 0, c.h, c.c0, c.b);
+        }
         ++n_tma;
       };
       {
@@ -1076,12 +1100,12 @@ __global__ void __launch_bounds__(kSumThreads, 1) segment_summary_kernel(const _
         const uint64_t dVt = dVt0 + (uint64_t)((buf * 32768) >> 4), dWt = dWt0 + (uint64_t)((buf * 32768) >> 4);
 #pragma unroll
         for (int j = 0; j < kC / 8; ++j)
-          tc::mma_tf32_ss(tb, dVt + kstep(kDV, j), dWt + kstep(kM, j), kIdC, (ck.first && j == 0) ? 0u : 1u);
-        tc::mma_commit(&bar_mma[buf]);
+          if (leader) tc::mma_tf32_ss(tb, dVt + kstep(kDV, j), dWt + kstep(kM, j), kIdC, (ck.first && j == 0) ? 0u : 1u);
+        if (leader) tc::mma_commit(&bar_mma[buf]);
         if (ck.last) ++n_items;
       }
       // nothing may still be running when the CTA releases its memory
-      tc::mma_commit(&bar_fin);
+      if (leader) tc::mma_commit(&bar_fin);
       tc::mbar_wait(&bar_fin, 0);
       for (uint32_t j = n; j < n_tma; ++j) tc::mbar_wait(&bar_tma[j & 1], (j >> 1) & 1);
     }

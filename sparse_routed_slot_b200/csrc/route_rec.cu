@@ -133,9 +133,11 @@ RSM_DEV void entry_values(const Rows& R, int64_t ir, int slot, float s, float fh
   w = kv * (-expm1f(lam));
 }
 
-template <int N, bool VALIDATE>
+template <int N, bool VALIDATE, bool VARIANT>
 __global__ void __launch_bounds__(kThreads) route_rec_kernel(const Rows R) {
   constexpr int KP = N;  // record entries
+  // VARIANT: a router other than plain sigmoid scores (the default compiles without that code)
+  const int router = VARIANT ? R.router : (int)RSM_ROUTER_SIGMOID;
   extern __shared__ __align__(128) unsigned char smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rl = lane >> 1, half = lane & 1;  // row of the task, half of the row (slots 64*half..)
@@ -257,7 +259,7 @@ __global__ void __launch_bounds__(kThreads) route_rec_kernel(const Rows R) {
 
     // softmax scores need the row's maximum and normalising sum (each lane of a pair: its half)
     float smax = 0.f, rsum = 1.f;
-    if (R.router & RSM_ROUTER_SOFTMAX) {
+    if (router & RSM_ROUTER_SOFTMAX) {
       float mx = -3.402823466e38f;
 #pragma unroll 4
       for (int i = 0; i < kRM / 2; ++i) mx = fmaxf(mx, xr[half * (kRM / 2) + i]);
@@ -269,42 +271,38 @@ __global__ void __launch_bounds__(kThreads) route_rec_kernel(const Rows R) {
     }
 
     constexpr int KH = KP / 2;
-    uint32_t sw[KH / 4];
-    float sc[KH];
-    int slots[KH];
-#pragma unroll
-    for (int i = 0; i < KH / 4; ++i) sw[i] = 0u;
-#pragma unroll
-    for (int q = 0; q < KH; ++q) {
-      // sorted: lane `half` takes rank positions half*KH + q; unsorted, the partner's array is
-      // this lane's reversed, so each lane takes its own first half
-      const uint32_t key = (sorted && half) ? top[KH + q] : top[q];
-      slots[q] = 127 - (int)(key & 0x7Fu);
-      const float xq = xr[slots[q]];
-      sc[q] = (half * KH + q >= K) ? 0.f : (R.router & RSM_ROUTER_SOFTMAX) ? expf(xq - smax) * rsum : sigmoid_f32(xq);
-    }
-    if (R.router & 2) {  // normalised over the row's K selected slots (both lanes of the pair)
+    // the key of this lane's q-th entry: sorted, lane `half` takes rank positions half*KH + q;
+    // unsorted, the partner's array is this lane's reversed, so each lane takes its own first half
+    auto entry_key = [&](int q) { return (sorted && half) ? top[KH + q] : top[q]; };
+    float rnorm = 1.f;
+    if (router & 2) {  // normalised scores: 1 / (sum over the row's K selected slots)
       float t = 0.f;
 #pragma unroll
-      for (int q = 0; q < KH; ++q) t += sc[q];
-      const float rt = 1.0f / (t + __shfl_xor_sync(kFull, t, 1));
-#pragma unroll
-      for (int q = 0; q < KH; ++q) sc[q] *= rt;
+      for (int q = 0; q < KH; ++q) {
+        const float xq = xr[127 - (int)(entry_key(q) & 0x7Fu)];
+        if (half * KH + q < K) t += (router & RSM_ROUTER_SOFTMAX) ? expf(xq - smax) * rsum : sigmoid_f32(xq);
+      }
+      rnorm = 1.0f / (t + __shfl_xor_sync(kFull, t, 1));
     }
     if (live && !exact) {
       // ---- entries in rank order from the sorted keys; each lane of the pair computes half
+      uint32_t sw[KH / 4];
       float lam[KH], wv[KH];
+#pragma unroll
+      for (int i = 0; i < KH / 4; ++i) sw[i] = 0u;
 #pragma unroll
       for (int q = 0; q < KH; ++q) {
         const int r = half * KH + q;
         lam[q] = 0.f;
         wv[q] = 0.f;
         if (r < K) {
-          const int slot = slots[q];
+          const int slot = 127 - (int)(entry_key(q) & 0x7Fu);
           sw[q / 4] |= (uint32_t)slot << (8 * (q % 4));
-          entry_values(R, ir, slot, sc[q], fh, lam[q], wv[q]);
+          const float xq = xr[slot];
+          const float sc = rnorm * ((router & RSM_ROUTER_SOFTMAX) ? expf(xq - smax) * rsum : sigmoid_f32(xq));
+          entry_values(R, ir, slot, sc, fh, lam[q], wv[q]);
           if (io) io[r] = slot;
-          if (so) so[r] = sc[q];
+          if (so) so[r] = sc;
         }
       }
 #pragma unroll
@@ -347,7 +345,7 @@ __global__ void __launch_bounds__(kThreads) route_rec_kernel(const Rows R) {
       });
       float scw[4];
       const float(&x4c)[4] = x4;  // (binding first sidesteps a front-end crash of this nvcc)
-      warp_router_scores(x4c, sel, (int)R.router, scw);
+      warp_router_scores(x4c, sel, router, scw);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         if ((sel >> e) & 1u) {
@@ -369,18 +367,18 @@ __global__ void __launch_bounds__(kThreads) route_rec_kernel(const Rows R) {
   cp_async_wait_all();
 }
 
-template <int N, bool V>
+template <int N, bool V, bool VAR>
 cudaError_t launch_n(const Rows& R, cudaStream_t stream) {
-  cudaError_t e = cudaFuncSetAttribute(route_rec_kernel<N, V>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+  cudaError_t e = cudaFuncSetAttribute(route_rec_kernel<N, V, VAR>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148, per_sm = 1;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, route_rec_kernel<N, V>, kThreads, kSmem);
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, route_rec_kernel<N, V, VAR>, kThreads, kSmem);
   const int64_t rows = R.B * R.H * R.T;
   const int64_t tasks = (rows + kRowsPerTask - 1) / kRowsPerTask;
   const int64_t grid = std::min<int64_t>((tasks + kWarps - 1) / kWarps, (int64_t)sms * std::max(per_sm, 1));
-  route_rec_kernel<N, V><<<(unsigned)grid, kThreads, kSmem, stream>>>(R);
+  route_rec_kernel<N, V, VAR><<<(unsigned)grid, kThreads, kSmem, stream>>>(R);
   return cudaGetLastError();
 }
 
@@ -437,8 +435,13 @@ cudaError_t launch_route_records(const float* logits, const float* f, const void
   R.idx_out = idx_out;
   R.score_out = score_out;
   cudaError_t e;
-  if (K <= 16) e = validate ? launch_n<16, true>(R, stream) : launch_n<16, false>(R, stream);
-  else e = validate ? launch_n<32, true>(R, stream) : launch_n<32, false>(R, stream);
+  if (router != RSM_ROUTER_SIGMOID) {
+    if (K <= 16) e = validate ? launch_n<16, true, true>(R, stream) : launch_n<16, false, true>(R, stream);
+    else e = validate ? launch_n<32, true, true>(R, stream) : launch_n<32, false, true>(R, stream);
+  } else {
+    if (K <= 16) e = validate ? launch_n<16, true, false>(R, stream) : launch_n<16, false, false>(R, stream);
+    else e = validate ? launch_n<32, true, false>(R, stream) : launch_n<32, false, false>(R, stream);
+  }
   (void)counts;  // counted by launch_record_counts, a launch of its own
   return e;
 }
