@@ -324,6 +324,41 @@ class PrefillCase:
         kms = [sum(row[j].elapsed_time(row[j + 1]) for row in kev) / steps for j in range(n)] if kernel_split else []
         return ms, kms
 
+    def time_graph(self, steps, warmup, world):
+        """Mean device time of one call (ms) for workloads whose calls are shorter than the host's
+        work to issue them: `steps` calls, each after an L2 flush, are captured in one CUDA graph
+        and replayed; the time of a graph of the flushes alone is subtracted."""
+        import torch
+        for _ in range(warmup):
+            self.step()
+        torch.cuda.synchronize()
+        g_all, g_flush = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_all):
+            for _ in range(steps):
+                self.flush.zero_()
+                self.step()
+        with torch.cuda.graph(g_flush):
+            for _ in range(steps):
+                self.flush.zero_()
+        stream = torch.cuda.current_stream()
+
+        def replay(g, reps=5):
+            g.replay()  # warm
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(reps):
+                g.replay()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            return e0.elapsed_time(e1) / reps
+
+        barrier(world)
+        t_all, t_flush = replay(g_all), replay(g_flush)
+        barrier(world)
+        del g_all, g_flush
+        return max(t_all - t_flush, 1e-6) / steps
+
     def roofline(self, ms, peaks, traffic_key):
         achieved = self.nbytes / (ms * 1e-3) / 1e9
         w = self.w
@@ -429,6 +464,13 @@ def run_prefill_config(args, w, world, rank, local, peaks) -> dict:
     steps = max(args.steps, 20)
     clocks = ClockSampler(local)
     ms, kms = case.time(steps, args.warmup, world, stream)
+    timing = "CUDA events around each call on its stream"
+    if case.flush is not None:
+        # calls this small finish before the host has issued the next one: replay a captured graph
+        ms = case.time_graph(steps, args.warmup, world)
+        kms = []
+        timing = (f"CUDA graph of {steps} calls, each after an L2 flush, replayed; a graph of the flushes "
+                  f"alone subtracted")
     clk = clocks.stop()
     value, ms_max = job_throughput(w.B * w.T, ms, world)
     names = KERNEL_NAMES.get(case.launches, [f"kernel {j}" for j in range(case.launches)])
@@ -437,8 +479,8 @@ def run_prefill_config(args, w, world, rank, local, peaks) -> dict:
     sub = {"workload": w.name, "value": value, "unit": "tokens/s", "ms_per_step": ms_max, "steps": steps,
            "dtype": "f32" if case.path_used == "simt" else "tf32", "config": config_of(w, case, world),
            "roofline": roof,
-           "kernels": [{"name": n, "ms": t} for n, t in zip(names, kms)], "clocks": clk,
-           "launches_timed": steps * case.launches}
+           "kernels": [{"name": n, "ms": t} for n, t in zip(names, kms)], "clocks": clk, "timing": timing,
+           "launches_timed": steps * case.launches * (1 if case.flush is None else 5)}
     if rank == 0 and not args.no_cpu:
         sub["cpu_baseline"] = oracle_sample(w)
     return sub

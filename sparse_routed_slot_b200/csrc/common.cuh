@@ -424,6 +424,32 @@ RSM_DEV void load_row_logits(const float* row, int lane, float (&x)[M / 32]) {
   }
 }
 
+// ---------------------------------------------------------------------------------------------
+// Host-side launch set-up, cached per device: the multiprocessor count, and each kernel's
+// dynamic shared-memory limit (an attribute of the function in the device's context; setting it
+// on every call costs host time that small launches would wait on).
+inline int device_sm_count() {
+  static int cached[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && cached[dev] > 0) return cached[dev];
+  int n = 148;
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  if (dev >= 0 && dev < 64) cached[dev] = n;
+  return n;
+}
+
+template <auto Kernel>
+inline cudaError_t set_smem_limit(int bytes) {
+  static int done[64] = {};  // bytes already allowed, per device
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && done[dev] >= bytes) return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = bytes;
+  return e;
+}
+
 // Validation helpers (used only under RSM_FLAG_VALIDATE).
 RSM_DEV bool finite_f32(float x) { return (__float_as_uint(x) & 0x7f800000u) != 0x7f800000u; }
 

@@ -286,20 +286,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(rsm_decode_args a) 
   }
 }
 
-int sm_count() {
-  int dev = 0, n = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-  return n;
-}
 
 template <int M, typename TIn>
 cudaError_t launch_t(const rsm_decode_args& a, cudaStream_t stream) {
   const int smem = kStages * kStageBytes + route_slots(M, a.Dv) * route_slot_bytes(M, a.Dv) + kRedBytes;
-  cudaError_t e = cudaFuncSetAttribute(decode_kernel<M, TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = set_smem_limit<decode_kernel<M, TIn>>(smem);
   if (e != cudaSuccess) return e;
   const int64_t items = (int64_t)a.B * a.H;
-  const unsigned grid = (unsigned)std::min<int64_t>(items, (int64_t)sm_count());
+  const unsigned grid = (unsigned)std::min<int64_t>(items, (int64_t)device_sm_count());
   decode_kernel<M, TIn><<<grid, kThreads, smem, stream>>>(a);
   return cudaGetLastError();
 }

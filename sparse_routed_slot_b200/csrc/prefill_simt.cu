@@ -21,12 +21,12 @@ namespace rsm {
 namespace {
 
 constexpr int kC = 32;          // tokens per chunk
-constexpr int kThreads = 256;
+constexpr int kThreads = 1024;  // 32 warps: one routing row per warp, and latency hidden by width
 
-__host__ __device__ inline int simt_dt(int M, int Dv) {
-  const int dt = M >= 256 ? 32 : 64;
-  return Dv < dt ? Dv : dt;
-}
+// Value columns per CTA: 64 (32 at M = 256, for shared memory). It divides the thread count, as
+// the register-blocked output and carry loops need; a narrower last tile is masked (DTe).
+__host__ __device__ inline int simt_dt(int M, int /*Dv*/) { return M >= 256 ? 32 : 64; }
+static_assert(kThreads % 64 == 0 && kThreads / 32 <= 32, "tile mapping: G = kThreads / DT groups <= kC");
 
 struct SimtSmem {
   // float offsets into the dynamic shared buffer
@@ -159,42 +159,76 @@ __global__ void __launch_bounds__(kThreads) prefill_simt_kernel(rsm_forward_args
     }
     __syncthreads();
 
-    // --- cumulative log-decay per slot, q scaled to the chunk start, chunk decay
+    // --- cumulative log-decay per slot (a prefix sum down the chunk), chunk decay
     for (int i = tid; i < M; i += kThreads) {
       float g = 0.f;
       for (int t = 0; t < kC; ++t) {
         g += s_g[t * M + i];
         s_g[t * M + i] = g;
-        s_qh[t * M + i] = s_q[t * M + i] * expf(g);
       }
       s_gC[i] = g;
       s_D[i] = expf(g);
     }
     __syncthreads();
+    // --- q scaled to the chunk start, every element in parallel
+    for (int p = tid; p < kC * M; p += kThreads) s_qh[p] = s_q[p] * expf(s_g[p]);
 
-    // --- intra-chunk weights A[t][s], s <= t (sparse over the K slots written at s)
-    for (int p = tid; p < kC * kC; p += kThreads) {
-      const int t = p / kC, s = p % kC;
-      float acc = 0.f;
-      if (s <= t && t < nrows) {
-        for (int r = 0; r < K; ++r) {
-          const int j = s_sidx[s * M + r];
-          acc = fmaf(s_q[t * M + j] * s_w[s * M + j], expf(s_g[t * M + j] - s_g[s * M + j]), acc);
+    // --- intra-chunk weights A[t][s], s <= t (sparse over the K slots written at s); each
+    // thread carries its kC*kC/kThreads pairs together so that their exponentials overlap
+    {
+      constexpr int kPairs = kC * kC / kThreads;  // 1
+      float acc[kPairs];
+      int tt[kPairs], ss[kPairs];
+#pragma unroll
+      for (int k = 0; k < kPairs; ++k) {
+        const int p = tid + k * kThreads;
+        tt[k] = p / kC;
+        ss[k] = p % kC;
+        acc[k] = 0.f;
+      }
+      for (int r = 0; r < K; ++r) {
+#pragma unroll
+        for (int k = 0; k < kPairs; ++k) {
+          const int t = tt[k], s = ss[k];
+          if (s <= t && t < nrows) {
+            const int j = s_sidx[s * M + r];
+            acc[k] = fmaf(s_q[t * M + j] * s_w[s * M + j], expf(s_g[t * M + j] - s_g[s * M + j]), acc[k]);
+          }
         }
       }
-      s_A[p] = acc;
+#pragma unroll
+      for (int k = 0; k < kPairs; ++k) s_A[tid + k * kThreads] = acc[k];
     }
     __syncthreads();
 
-    // --- outputs of the chunk for this column tile
-    for (int p = tid; p < kC * DT; p += kThreads) {
-      const int t = p / DT, dd = p % DT;
-      if (t < nrows && dd < DTe) {
-        float acc = 0.f;
-        const float* qh = s_qh + t * M;
-        for (int i = 0; i < M; ++i) acc = fmaf(qh[i], s_H[i * DT + dd], acc);
-        for (int s = 0; s <= t; ++s) acc = fmaf(s_A[t * kC + s], s_v[s * DT + dd], acc);
-        a.o[(((int64_t)b * T + c0 + t) * H + h) * Dv + d0 + dd] = acc;
+    // --- outputs of the chunk for this column tile: thread (dd, g) computes the tokens
+    // t = g + G k, so that each state and value element it loads serves all of them
+    {
+      constexpr int kMaxNT = kC * 64 / kThreads;  // tokens per thread at DT = 64
+      const int G = kThreads / DT, dd = tid % DT, g = tid / DT, NT = kC / G;  // NT = 1 or 2
+      float acc[kMaxNT];
+#pragma unroll
+      for (int k = 0; k < kMaxNT; ++k) acc[k] = 0.f;
+#pragma unroll 4
+      for (int i = 0; i < M; ++i) {
+        const float hv = s_H[i * DT + dd];
+#pragma unroll
+        for (int k = 0; k < kMaxNT; ++k)
+          if (k < NT) acc[k] = fmaf(s_qh[(g + G * k) * M + i], hv, acc[k]);
+      }
+#pragma unroll 4
+      for (int s = 0; s < kC; ++s) {
+        const float vv = s_v[s * DT + dd];
+#pragma unroll
+        for (int k = 0; k < kMaxNT; ++k) {
+          const int t = g + G * k;
+          if (k < NT && s <= t) acc[k] = fmaf(s_A[t * kC + s], vv, acc[k]);
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < kMaxNT; ++k) {
+        const int t = g + G * k;
+        if (k < NT && t < nrows && dd < DTe) a.o[(((int64_t)b * T + c0 + t) * H + h) * Dv + d0 + dd] = acc[k];
       }
     }
     // --- write weights carried to the chunk end (non-positive exponents)
@@ -205,13 +239,29 @@ __global__ void __launch_bounds__(kThreads) prefill_simt_kernel(rsm_forward_args
     }
     __syncthreads();
 
-    // --- state carry; slots not selected in this chunk are left untouched
-    for (int p = tid; p < M * DT; p += kThreads) {
-      const int i = p / DT, dd = p % DT;
-      if (s_touch[i]) {
-        float acc = s_D[i] * s_H[p];
-        for (int t = 0; t < kC; ++t) acc = fmaf(s_w[t * M + i], s_v[t * DT + dd], acc);
-        s_H[p] = acc;
+    // --- state carry; slots not selected in this chunk are left untouched. Thread (dd, g)
+    // updates the slots i = g + G j, 8 at a time, so that each value element serves all of them
+    {
+      const int G = kThreads / DT, dd = tid % DT, g = tid / DT, NI = M / G;  // NI = 2 .. 8
+      for (int j0 = 0; j0 < NI; j0 += 8) {
+        float acc[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int i = g + G * (j0 + j);
+          acc[j] = (j0 + j < NI) ? s_D[i] * s_H[i * DT + dd] : 0.f;
+        }
+#pragma unroll 4
+        for (int t = 0; t < kC; ++t) {
+          const float vv = s_v[t * DT + dd];
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            if (j0 + j < NI) acc[j] = fmaf(s_w[t * M + g + G * (j0 + j)], vv, acc[j]);
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int i = g + G * (j0 + j);
+          if (j0 + j < NI && s_touch[i]) s_H[i * DT + dd] = acc[j];
+        }
       }
     }
     __syncthreads();
@@ -230,7 +280,7 @@ cudaError_t launch_simt(const rsm_forward_args& a, cudaStream_t stream) {
   const int DT = simt_dt(M, a.Dv);
   const SimtSmem L = simt_layout(M, DT);
   auto kern = prefill_simt_kernel<M, TIn>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L.total);
+  cudaError_t e = set_smem_limit<prefill_simt_kernel<M, TIn>>(L.total);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)(a.B * a.H), (unsigned)((a.Dv + DT - 1) / DT));
   kern<<<grid, kThreads, L.total, stream>>>(a, DT);

@@ -1198,12 +1198,7 @@ bool make_map(CUtensorMap* m, const void* base, int B, int T, int H, int C, bool
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-int sm_count() {
-  int dev = 0, n = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-  return n;
-}
+int sm_count() { return device_sm_count(); }
 
 struct Plan {
   int nseg, seg_chunks;
@@ -1250,10 +1245,10 @@ template <int KP>
 cudaError_t launch_passes(const Maps& maps, const Params& p, const Plan& pl, int64_t pairs, int sms,
                           cudaStream_t stream) {
   cudaError_t e =
-      cudaFuncSetAttribute(prefill_tc_kernel<KP>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+      set_smem_limit<prefill_tc_kernel<KP>>(kSmemBytes);
   if (e != cudaSuccess) return e;
   if (pl.nseg > 1) {
-    e = cudaFuncSetAttribute(segment_summary_kernel<KP>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSumSmemBytes);
+    e = set_smem_limit<segment_summary_kernel<KP>>(kSumSmemBytes);
     if (e != cudaSuccess) return e;
     const int items = (int)(pairs * (pl.nseg - 1));
     segment_summary_kernel<KP><<<std::min(items, sms), kSumThreads, kSumSmemBytes, stream>>>(maps, p);

@@ -46,9 +46,7 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
 cudaError_t launch_route(const float* logits, int64_t rows, int M, int K, int32_t* idx_out,
                          float* score_out, int router, int validate, cudaStream_t stream) {
   if (rows == 0) return cudaSuccess;
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int sms = device_sm_count();
   const int64_t want = (rows + 7) / 8;
   const int grid = (int)(want < (int64_t)sms * 8 ? want : (int64_t)sms * 8);
   switch (M) {

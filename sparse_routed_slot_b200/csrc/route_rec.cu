@@ -369,12 +369,15 @@ __global__ void __launch_bounds__(kThreads) route_rec_kernel(const Rows R) {
 
 template <int N, bool V, bool VAR>
 cudaError_t launch_n(const Rows& R, cudaStream_t stream) {
-  cudaError_t e = cudaFuncSetAttribute(route_rec_kernel<N, V, VAR>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+  cudaError_t e = set_smem_limit<route_rec_kernel<N, V, VAR>>(kSmem);
   if (e != cudaSuccess) return e;
-  int dev = 0, sms = 148, per_sm = 1;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, route_rec_kernel<N, V, VAR>, kThreads, kSmem);
+  const int sms = device_sm_count();
+  static int per_sm_cached = 0;  // the same on every B200 device
+  int per_sm = per_sm_cached;
+  if (per_sm <= 0) {
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, route_rec_kernel<N, V, VAR>, kThreads, kSmem);
+    per_sm_cached = per_sm;
+  }
   const int64_t rows = R.B * R.H * R.T;
   const int64_t tasks = (rows + kRowsPerTask - 1) / kRowsPerTask;
   const int64_t grid = std::min<int64_t>((tasks + kWarps - 1) / kWarps, (int64_t)sms * std::max(per_sm, 1));

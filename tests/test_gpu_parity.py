@@ -377,3 +377,17 @@ def test_forward_profile_events_split_the_call(rsm):
     assert all(p > 0 for p in parts)
     assert abs(sum(parts) - ev[0].elapsed_time(ev[n])) < 1e-3
     assert torch.equal(o, ref["o"]) and torch.equal(HT, ref["HT"])
+
+
+@pytest.mark.parametrize("M,Dv", [(32, 4), (64, 12), (128, 20), (256, 36)])
+def test_simt_narrow_and_ragged_value_tiles(rsm, M, Dv):
+    """The CUDA-core path works in value-column tiles of 64 (32 at M = 256); narrower value
+    widths and ragged last tiles are masked."""
+    B, T, H, K = 2, 75, 2, min(16, M)
+    x = make_inputs(B, T, H, M, Dv, torch.float32, "slot", seed=M + Dv, device="cuda", h0=True)
+    out = rsm.forward(x["q"], x["k"], x["v"], x["logits"], x["f"], K, x["H0"], path="simt")
+    torch.cuda.synchronize()
+    c = host(x)
+    r = oracle.forward(c["q"], c["k"], c["v"], c["logits"], c["f"], K, c["H0"])
+    assert rel(out["o"].cpu().numpy(), r["o"]) <= TOL_FP32
+    assert rel(out["HT"].cpu().numpy(), r["HT"]) <= TOL_FP32
