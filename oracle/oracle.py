@@ -46,6 +46,9 @@ def bind(lib):
     lib.rsmo_forward_ex.restype = ctypes.c_int
     lib.rsmo_route_ex.argtypes = [f32p, ctypes.c_longlong, ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, vp]
     lib.rsmo_route_ex.restype = ctypes.c_int
+    if hasattr(lib, "rsmo_backward"):
+        lib.rsmo_backward.argtypes = [ctypes.c_int] * 7 + [f32p] * 5 + [vp] * 9 + [ctypes.c_int]
+        lib.rsmo_backward.restype = ctypes.c_int
     return lib
 
 
@@ -132,3 +135,26 @@ def route(logits, K: int, router: str = "sigmoid"):
     if _load().rsmo_route_ex(lg, N, M, K, ROUTERS[router], _ptr(idx), _ptr(score)) != 0:
         raise ValueError("oracle rejected the sizes")
     return idx, score
+
+
+def backward(q, k, v, logits, f, K: int, dO=None, dHT=None, H0=None, nthreads: int | None = None):
+    """Gradients of the recurrence (sigmoid router) for the loss whose gradients with respect to
+    o and H_T are dO [B,T,H,Dv] and dHT [B,H,M,Dv] (None = 0). Returns dict(dq, dk, dlogits
+    [B,T,H,M], dv [B,T,H,Dv], df (f's shape), dH0 [B,H,M,Dv]), all float64."""
+    q, k, v, logits, f = map(_f32, (q, k, v, logits, f))
+    B, T, H, M = q.shape
+    Dv = v.shape[-1]
+    per_slot = 1 if f.shape == (B, T, H, M) else 0
+    if not per_slot and f.shape != (B, T, H):
+        raise ValueError(f"bad f shape {f.shape}")
+    def d64(x):
+        return None if x is None else np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+    h0, do, dht = d64(H0), d64(dO), d64(dHT)
+    out = {"dq": np.zeros((B, T, H, M)), "dk": np.zeros((B, T, H, M)), "dlogits": np.zeros((B, T, H, M)),
+           "dv": np.zeros((B, T, H, Dv)), "df": np.zeros(f.shape), "dH0": np.zeros((B, H, M, Dv))}
+    rc = _load().rsmo_backward(B, T, H, M, K, Dv, per_slot, q, k, v, logits, f, _ptr(h0), _ptr(do), _ptr(dht),
+                               _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dlogits"]),
+                               _ptr(out["df"]), _ptr(out["dH0"]), nthreads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle rejected the sizes")
+    return out

@@ -207,6 +207,163 @@ int rsmo_decode_step(int B, int H, int M, int K, int Dv, int per_slot, const flo
                       score, nthreads);
 }
 
+/* ---------------------------------------------------------------------------------------------
+ * Gradients of the recurrence (sigmoid router), by reverse-mode differentiation of the forward
+ * above taken one token at a time. With G = dL/dH (M x Dv), per token t from the last to the
+ * first, selected slots i in S_t, a_i = exp(s_i f), w_i = (1 - a_i) k_i:
+ *   read o_t = sum_i q_i H_t[i]:      dq_t[i] = do_t . H_t[i];  G[i] += q_i do_t  (every slot)
+ *   write H_t[i] = a_i H_{t-1}[i] + w_i v_t (i in S_t):
+ *       dv_t += w_i G[i];  dw_i = G[i] . v_t;  da_i = G[i] . H_{t-1}[i] - k_i dw_i;
+ *       dk_{t,i} = (1 - a_i) dw_i;  dlam_i = a_i da_i  (a = e^lam, lam = s f);
+ *       df += s_i dlam_i (per head; per slot: df_i = s_i dlam_i);  ds_i = f dlam_i;
+ *       dlogit_i = s_i (1 - s_i) ds_i;  then G[i] = a_i G[i]
+ *   unselected slots: G[i] passes unchanged; their dk and dlogit are 0 (the TopK cut is
+ *   piecewise constant in the logits).
+ *   dH0 = G after the first token. H_{t-1} is recovered from H_t by putting back the rows the
+ *   token overwrote, kept from a forward sweep ("tape").
+ * Inputs as rsmo_forward plus dO [B,T,H,Dv] and dHT [B,H,M,Dv] (NULL = 0); outputs (each may be
+ * NULL): dq, dk, dlogits [B,T,H,M]; dv [B,T,H,Dv]; df [B,T,H] or [B,T,H,M]; dH0 [B,H,M,Dv].
+ * ------------------------------------------------------------------------------------------- */
+typedef struct {
+  int B, T, H, M, K, Dv, per_slot;
+  const float *q, *k, *v, *logits, *f;
+  const double *H0, *dO, *dHT;
+  double *dq, *dk, *dv, *dlogits, *df, *dH0;
+  int pair_begin, pair_end;
+} rsmo_bjob;
+
+static void rsmo_backward_pair(const rsmo_bjob* J, int pair) {
+  const int b = pair / J->H, h = pair % J->H;
+  const int M = J->M, K = J->K, Dv = J->Dv, H = J->H, T = J->T;
+  double* S = (double*)malloc(sizeof(double) * (size_t)M * Dv);
+  double* G = (double*)malloc(sizeof(double) * (size_t)M * Dv);
+  int32_t* sel = (int32_t*)malloc(sizeof(int32_t) * (size_t)T * K);
+  double* tape = (double*)malloc(sizeof(double) * (size_t)T * K * Dv); /* H_{t-1} of the rows t overwrote */
+  double* sc = (double*)malloc(sizeof(double) * (size_t)K);
+  if (J->H0)
+    memcpy(S, J->H0 + (size_t)pair * M * Dv, sizeof(double) * (size_t)M * Dv);
+  else
+    memset(S, 0, sizeof(double) * (size_t)M * Dv);
+  /* forward sweep, keeping the overwritten rows */
+  for (int t = 0; t < T; ++t) {
+    const size_t row = ((size_t)b * T + t) * H + h;
+    const float* k = J->k + row * M;
+    const float* lg = J->logits + row * M;
+    const float* v = J->v + row * Dv;
+    int32_t* st = sel + (size_t)t * K;
+    rsmo_topk(lg, M, K, st);
+    rsmo_scores(lg, M, K, st, 0, sc);
+    for (int r = 0; r < K; ++r) {
+      const int i = st[r];
+      const double f = J->per_slot ? (double)J->f[row * M + i] : (double)J->f[row];
+      const double a = exp(sc[r] * f);
+      const double wk = (1.0 - a) * (double)k[i];
+      double* Si = S + (size_t)i * Dv;
+      memcpy(tape + ((size_t)t * K + r) * Dv, Si, sizeof(double) * (size_t)Dv);
+      for (int d = 0; d < Dv; ++d) Si[d] = a * Si[d] + wk * (double)v[d];
+    }
+  }
+  /* reverse sweep */
+  if (J->dHT)
+    memcpy(G, J->dHT + (size_t)pair * M * Dv, sizeof(double) * (size_t)M * Dv);
+  else
+    memset(G, 0, sizeof(double) * (size_t)M * Dv);
+  for (int t = T - 1; t >= 0; --t) {
+    const size_t row = ((size_t)b * T + t) * H + h;
+    const float* q = J->q + row * M;
+    const float* k = J->k + row * M;
+    const float* lg = J->logits + row * M;
+    const float* v = J->v + row * Dv;
+    const double* dO = J->dO ? J->dO + row * Dv : NULL;
+    const int32_t* st = sel + (size_t)t * K;
+    for (int i = 0; i < M; ++i) {
+      double* Gi = G + (size_t)i * Dv;
+      const double* Si = S + (size_t)i * Dv;
+      double dqi = 0.0;
+      if (dO)
+        for (int d = 0; d < Dv; ++d) {
+          dqi += dO[d] * Si[d];
+          Gi[d] += (double)q[i] * dO[d];
+        }
+      if (J->dq) J->dq[row * M + i] = dqi;
+      if (J->dk) J->dk[row * M + i] = 0.0;
+      if (J->dlogits) J->dlogits[row * M + i] = 0.0;
+      if (J->df && J->per_slot) J->df[row * M + i] = 0.0;
+    }
+    if (J->dv)
+      for (int d = 0; d < Dv; ++d) J->dv[row * Dv + d] = 0.0;
+    double dfh = 0.0;
+    rsmo_scores(lg, M, K, st, 0, sc);
+    for (int r = 0; r < K; ++r) {
+      const int i = st[r];
+      const double s = sc[r];
+      const double f = J->per_slot ? (double)J->f[row * M + i] : (double)J->f[row];
+      const double a = exp(s * f);
+      const double wk = (1.0 - a) * (double)k[i];
+      double* Gi = G + (size_t)i * Dv;
+      double* Si = S + (size_t)i * Dv;
+      const double* prev = tape + ((size_t)t * K + r) * Dv;
+      double dw = 0.0, dap = 0.0;
+      for (int d = 0; d < Dv; ++d) {
+        dw += Gi[d] * (double)v[d];
+        dap += Gi[d] * prev[d];
+        if (J->dv) J->dv[row * Dv + d] += wk * Gi[d];
+      }
+      const double da = dap - (double)k[i] * dw;
+      const double dlam = a * da;
+      if (J->dk) J->dk[row * M + i] = (1.0 - a) * dw;
+      if (J->df) {
+        if (J->per_slot) J->df[row * M + i] = s * dlam;
+        else dfh += s * dlam;
+      }
+      if (J->dlogits) J->dlogits[row * M + i] = s * (1.0 - s) * (f * dlam);
+      for (int d = 0; d < Dv; ++d) {
+        Gi[d] *= a;
+        Si[d] = prev[d];
+      }
+    }
+    if (J->df && !J->per_slot) J->df[row] = dfh;
+  }
+  if (J->dH0) memcpy(J->dH0 + (size_t)pair * M * Dv, G, sizeof(double) * (size_t)M * Dv);
+  free(sc);
+  free(tape);
+  free(sel);
+  free(G);
+  free(S);
+}
+
+static void* rsmo_bworker(void* arg) {
+  const rsmo_bjob* J = (const rsmo_bjob*)arg;
+  for (int p = J->pair_begin; p < J->pair_end; ++p) rsmo_backward_pair(J, p);
+  return NULL;
+}
+
+int rsmo_backward(int B, int T, int H, int M, int K, int Dv, int per_slot, const float* q,
+                  const float* k, const float* v, const float* logits, const float* f,
+                  const double* H0, const double* dO, const double* dHT, double* dq, double* dk,
+                  double* dv, double* dlogits, double* df, double* dH0, int nthreads) {
+  if (B < 0 || T < 0 || H < 0 || M < 1 || K < 1 || K > M || Dv < 1) return -1;
+  const int pairs = B * H;
+  if (nthreads < 1) nthreads = 1;
+  if (nthreads > pairs) nthreads = pairs > 0 ? pairs : 1;
+  rsmo_bjob base = {B, T, H, M, K, Dv, per_slot, q, k, v, logits, f, H0, dO, dHT,
+                    dq, dk, dv, dlogits, df, dH0, 0, pairs};
+  pthread_t* th = (pthread_t*)malloc(sizeof(pthread_t) * (size_t)nthreads);
+  rsmo_bjob* jobs = (rsmo_bjob*)malloc(sizeof(rsmo_bjob) * (size_t)nthreads);
+  for (int w = 0; w < nthreads; ++w) {
+    jobs[w] = base;
+    jobs[w].pair_begin = (int)((long long)pairs * w / nthreads);
+    jobs[w].pair_end = (int)((long long)pairs * (w + 1) / nthreads);
+    if (nthreads == 1) rsmo_bworker(&jobs[w]);
+    else pthread_create(&th[w], NULL, rsmo_bworker, &jobs[w]);
+  }
+  if (nthreads > 1)
+    for (int w = 0; w < nthreads; ++w) pthread_join(th[w], NULL);
+  free(jobs);
+  free(th);
+  return 0;
+}
+
 /* Standalone routing: TopK indices (rank order) and the router variant's scores, rows [rows, M]. */
 int rsmo_route_ex(const float* logits, long long rows, int M, int K, int router, int32_t* idx,
                   double* score) {

@@ -9,6 +9,7 @@
   normalised over the TopK set) against scipy's softmax/expit and numpy sums, a hand-derived
   example and the quadratic form; selection counts against a bincount of a library sort;
 * the invariant that unselected slots keep their bits;
+* the backward (gradients of the recurrence) against central finite differences of the forward;
 * mutants of the oracle (planted mistakes, compiled on the CPU) must fail these pins.
 """
 import ctypes
@@ -308,6 +309,11 @@ MUTANTS = {
     "normalise_by_first_score": ("for (int r = 0; r < K; ++r) sum += s[r];", "sum = s[0];", None, None),
     "counts_by_rank": ("J->counts[(size_t)pair * M + i] += 1;", "J->counts[(size_t)pair * M + r] += 1;",
                        None, None),
+    "backward_decay_grad_without_write_term": ("const double da = dap - (double)k[i] * dw;",
+                                               "const double da = dap;", None, None),
+    "backward_state_grad_not_decayed": ("        Gi[d] *= a;\n", "        Gi[d] *= 1.0;\n", None, None),
+    "backward_slot_decay_grad_without_score": ("J->df[row * M + i] = s * dlam;", "J->df[row * M + i] = dlam;",
+                                               None, None),
 }
 
 
@@ -335,6 +341,8 @@ def _pins_pass_with(lib_path) -> bool:
                          (test_golden_router_variants, ("softmax",)),
                          (test_golden_router_variants, ("sigmoid_norm",)),
                          (test_selection_counts_match_bincount, ()),
+                         (test_backward_matches_finite_differences, (False,)),
+                         (test_backward_matches_finite_differences, (True,)),
                          (test_topk_tie_rules, ()), (test_window_limit_is_sliding_window, ()),
                          (test_recurrence_matches_quadratic_form, (1, 3, True)),
                          (test_recurrence_matches_quadratic_form, (2, 3, False))]:
@@ -354,3 +362,65 @@ def test_pins_catch_planted_mistakes(tmp_path, name):
 
 def test_pins_pass_with_the_real_oracle():
     assert _pins_pass_with(oracle.build())
+
+
+# ----------------------------------------------------------------------------- backward
+
+
+def _separated_logits(rng, T, M):
+    """Logits whose neighbours differ by at least 0.25, so that a 2^-10 step never changes TopK."""
+    base = np.arange(M, dtype=np.float64) * 0.25
+    return np.stack([rng.permutation(base) for _ in range(T)]).astype(np.float32) - 0.7
+
+
+def _fd_case(per_slot, seed):
+    rng = np.random.default_rng(seed)
+    T, M, Dv, K = 6, 6, 3, 2
+    q = rng.standard_normal((1, T, 1, M)).astype(np.float32)
+    k = rng.standard_normal((1, T, 1, M)).astype(np.float32)
+    v = rng.standard_normal((1, T, 1, Dv)).astype(np.float32)
+    lg = _separated_logits(rng, T, M)[None, :, None]
+    fs = (1, T, 1, M) if per_slot else (1, T, 1)
+    f = (-0.2 - np.abs(rng.standard_normal(fs))).astype(np.float32)
+    H0 = rng.standard_normal((1, 1, M, Dv))
+    dO = rng.standard_normal((1, T, 1, Dv))
+    dHT = rng.standard_normal((1, 1, M, Dv))
+    return dict(q=q, k=k, v=v, logits=lg, f=f, H0=H0), dO, dHT, K
+
+
+def _loss(x, dO, dHT, K):
+    out = oracle.forward(x["q"], x["k"], x["v"], x["logits"], x["f"], K, x["H0"], want_idx=False, nthreads=1)
+    return float(np.sum(out["o"] * dO) + np.sum(out["HT"] * dHT))
+
+
+@pytest.mark.parametrize("per_slot", [False, True])
+def test_backward_matches_finite_differences(per_slot):
+    """Every gradient component against a central difference of the forward oracle, with a step of
+    2^-10 that is exact in fp32 and never moves the TopK cut."""
+    x, dO, dHT, K = _fd_case(per_slot, 11 + per_slot)
+    g = oracle.backward(x["q"], x["k"], x["v"], x["logits"], x["f"], K, dO=dO, dHT=dHT, H0=x["H0"], nthreads=1)
+    eps = 2.0 ** -10
+    names = {"q": "dq", "k": "dk", "v": "dv", "logits": "dlogits", "f": "df", "H0": "dH0"}
+    for name, gname in names.items():
+        base = x[name]
+        fd = np.zeros(base.shape)
+        for idx in np.ndindex(base.shape):
+            xp = {n: a.copy() for n, a in x.items()}
+            xm = {n: a.copy() for n, a in x.items()}
+            xp[name][idx] += eps
+            xm[name][idx] -= eps
+            fd[idx] = (_loss(xp, dO, dHT, K) - _loss(xm, dO, dHT, K)) / (2 * eps)
+        scale = max(np.max(np.abs(fd)), 1e-12)
+        assert np.max(np.abs(g[gname] - fd)) <= 2e-5 * scale, (name, np.max(np.abs(g[gname] - fd)), scale)
+
+
+def test_backward_unselected_logits_and_keys_get_no_gradient():
+    rng = np.random.default_rng(5)
+    T, M, Dv, K = 9, 8, 4, 3
+    q, k, lg = (rng.standard_normal((1, T, 1, M)).astype(np.float32) for _ in range(3))
+    v = rng.standard_normal((1, T, 1, Dv)).astype(np.float32)
+    f = -np.abs(rng.standard_normal((1, T, 1))).astype(np.float32)
+    g = oracle.backward(q, k, v, lg, f, K, dO=rng.standard_normal((1, T, 1, Dv)), nthreads=1)
+    sel = np.zeros((T, M), bool)
+    np.put_along_axis(sel, brute.topk_stable(lg[0, :, 0], K).astype(np.int64), True, axis=1)
+    assert np.all(g["dk"][0, :, 0][~sel] == 0.0) and np.all(g["dlogits"][0, :, 0][~sel] == 0.0)
