@@ -225,6 +225,51 @@ typedef struct rsm_decode_args {
 
 RSM_API rsm_status rsm_decode_step(const rsm_decode_args* args, void* stream);
 
+/* ---------------------------------------------------------------------------------------------
+ * rsm_backward -- gradients of the prefill (training). Reverse-mode differentiation of the
+ *   recurrence above with the sigmoid router: given dO = dL/do and dHT = dL/dH_T, it returns
+ *   dL/dq, dL/dk, dL/dv, dL/dlogits, dL/df and dL/dH0. The TopK cut is piecewise constant in the
+ *   logits, so unselected slots get no key or logit gradient. Raven README "Model Structure"
+ *   (chunked computation for training) and the fork's reverse-scan backward.
+ *   Inputs as rsm_forward (q, k, v in qkv_dtype; logits, f, H0 fp32; H0 may be NULL = zeros)
+ *   dO    [B,T,H,Dv] fp32, or NULL for zero
+ *   dHT   [B,H,M,Dv] fp32, or NULL for zero
+ *   dq, dk, dlogits [B,T,H,M] fp32; dv [B,T,H,Dv] fp32; df [B,T,H] or [B,T,H,M] fp32;
+ *   dH0 [B,H,M,Dv] fp32 (each output may be NULL to skip it)
+ *   workspace: at least rsm_backward_workspace_size(args) bytes (256-byte aligned): the routing
+ *     of every token and a tape of the K state rows each token overwrites (T*K*Dv*4 bytes per
+ *     (b,h) stream).
+ *   Supported: the sizes of rsm_forward with M*Dv <= 24576 (the state and its gradient stay in
+ *   shared memory), router RSM_ROUTER_SIGMOID. The arithmetic is fp32 on CUDA cores.
+ * ------------------------------------------------------------------------------------------- */
+typedef struct rsm_backward_args {
+  int B, T, H, M, K, Dv;
+  rsm_dtype qkv_dtype;
+  rsm_decay decay;
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* logits;
+  const float* f;
+  const float* H0;
+  const float* dO;
+  const float* dHT;
+  float* dq;
+  float* dk;
+  float* dv;
+  float* dlogits;
+  float* df;
+  float* dH0;
+  void* workspace;
+  size_t workspace_bytes;
+  rsm_router router;
+  int flags; /* RSM_FLAG_* */
+} rsm_backward_args;
+
+/* Bytes of workspace rsm_backward needs, or (size_t)-1 for arguments it rejects. Host-only. */
+RSM_API size_t rsm_backward_workspace_size(const rsm_backward_args* args);
+RSM_API rsm_status rsm_backward(const rsm_backward_args* args, void* stream);
+
 /* Human-readable name of a status code (static storage). */
 RSM_API const char* rsm_status_string(rsm_status status);
 

@@ -6,8 +6,9 @@ a thin ctypes binding with the same three calls:
     route(logits, K)                          -> TopK slot indices and sigmoid scores
     forward(q, k, v, logits, f, K, H0=None)   -> chunked prefill: o and the final state H_T
     decode_step(q, k, v, logits, f, K, state) -> one generation token, state updated in place
+    backward(q, k, v, logits, f, K, dO, dHT)  -> gradients of the prefill (RSMFunction: autograd)
 """
-from .api import decode_step, device_status, forward, route  # noqa: F401
+from .api import RSMFunction, backward, decode_step, device_status, forward, route  # noqa: F401
 from ._lib import RSMError  # noqa: F401
 
-__all__ = ["route", "forward", "decode_step", "device_status", "RSMError"]
+__all__ = ["route", "forward", "backward", "decode_step", "device_status", "RSMFunction", "RSMError"]

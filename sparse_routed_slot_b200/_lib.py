@@ -25,7 +25,7 @@ RSM_FLAG_TEST_STALL_ROUTING = 256
 # Every symbol include/rsm.h declares (the CPU tests check the library exports all of them).
 EXPORTED = ("rsm_route", "rsm_route_ex", "rsm_forward_workspace_size", "rsm_forward", "rsm_forward_selected_path",
             "rsm_forward_kernel_launches", "rsm_forward_set_profile_events",
-            "rsm_decode_step",
+            "rsm_decode_step", "rsm_backward_workspace_size", "rsm_backward",
             "rsm_status_string", "rsm_last_error", "rsm_get_device_status", "rsm_version",
             "rsm_forward_noalloc", "rsm_forward_noalloc_max_scratch")
 
@@ -48,6 +48,16 @@ class DecodeArgs(ctypes.Structure):
                 ("q", _vp), ("k", _vp), ("v", _vp), ("logits", _vp), ("f", _vp),
                 ("state", _vp), ("o", _vp), ("idx_out", _vp), ("score_out", _vp),
                 ("flags", _int), ("router", _int), ("slot_counts", _vp)]
+
+
+class BackwardArgs(ctypes.Structure):
+    _fields_ = [("B", _int), ("T", _int), ("H", _int), ("M", _int), ("K", _int), ("Dv", _int),
+                ("qkv_dtype", _int), ("decay", _int),
+                ("q", _vp), ("k", _vp), ("v", _vp), ("logits", _vp), ("f", _vp), ("H0", _vp),
+                ("dO", _vp), ("dHT", _vp),
+                ("dq", _vp), ("dk", _vp), ("dv", _vp), ("dlogits", _vp), ("df", _vp), ("dH0", _vp),
+                ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t),
+                ("router", _int), ("flags", _int)]
 
 
 class RSMError(RuntimeError):
@@ -83,6 +93,10 @@ def load() -> ctypes.CDLL:
         lib.rsm_forward_noalloc.restype = _int
         lib.rsm_forward_noalloc_max_scratch.argtypes = []
         lib.rsm_forward_noalloc_max_scratch.restype = ctypes.c_size_t
+        lib.rsm_backward_workspace_size.argtypes = [ctypes.POINTER(BackwardArgs)]
+        lib.rsm_backward_workspace_size.restype = ctypes.c_size_t
+        lib.rsm_backward.argtypes = [ctypes.POINTER(BackwardArgs), _vp]
+        lib.rsm_backward.restype = _int
         lib.rsm_decode_step.argtypes = [ctypes.POINTER(DecodeArgs), _vp]
         lib.rsm_decode_step.restype = _int
         lib.rsm_status_string.argtypes = [_int]

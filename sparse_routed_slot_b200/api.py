@@ -197,3 +197,66 @@ def device_status(device=None) -> int:
     """Synchronizes the current stream and returns (and clears) the device status code."""
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
     return _lib.load().rsm_get_device_status(_stream(dev))
+
+
+def backward(q, k, v, logits, f, K: int, dO=None, dHT=None, H0=None, *, validate: bool = False,
+             out=None, workspace=None):
+    """Gradients of rsm_forward (sigmoid router): q, k, v, logits, f, H0 as in forward();
+    dO [B,T,H,Dv] fp32 and dHT [B,H,M,Dv] fp32 (None = zero). Returns dict(dq, dk, dlogits
+    [B,T,H,M], dv [B,T,H,Dv], df (f's shape), dH0 [B,H,M,Dv]), all fp32."""
+    B, T, H, M = q.shape
+    Dv = v.shape[-1]
+    dev = q.device
+    a0 = _forward_args(q, k, v, logits, f, K, H0, torch.empty(1, device=dev), None, None, None, "simt",
+                       validate)  # shape and dtype checks shared with the forward
+    a = _lib.BackwardArgs()
+    for name in ("B", "T", "H", "M", "K", "Dv", "qkv_dtype", "decay", "q", "k", "v", "logits", "f", "H0",
+                 "flags"):
+        setattr(a, name, getattr(a0, name))
+    if dO is not None:
+        _need(dO, "dO", torch.float32, (B, T, H, Dv))
+    if dHT is not None:
+        _need(dHT, "dHT", torch.float32, (B, H, M, Dv))
+    a.dO = None if dO is None else dO.data_ptr()
+    a.dHT = None if dHT is None else dHT.data_ptr()
+    out = dict(out or {})
+    shapes = {"dq": (B, T, H, M), "dk": (B, T, H, M), "dlogits": (B, T, H, M), "dv": (B, T, H, Dv),
+              "df": tuple(f.shape), "dH0": (B, H, M, Dv)}
+    for name, shape in shapes.items():
+        if out.get(name) is None:
+            out[name] = torch.empty(shape, dtype=torch.float32, device=dev)
+        _need(out[name], name, torch.float32, shape)
+        setattr(a, name, out[name].data_ptr())
+    a.router = _lib.RSM_ROUTER_SIGMOID
+    L = _lib.load()
+    need = L.rsm_backward_workspace_size(ctypes.byref(a))
+    if need == ctypes.c_size_t(-1).value:
+        _lib.check(L.rsm_backward(ctypes.byref(a), None))  # raises with the reason
+    if need:
+        if workspace is None or workspace.numel() < need:
+            workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+        a.workspace, a.workspace_bytes = workspace.data_ptr(), workspace.numel()
+    _lib.check(L.rsm_backward(ctypes.byref(a), _stream(dev)))
+    return out
+
+
+class RSMFunction(torch.autograd.Function):
+    """The mixer as an autograd function: forward runs rsm_forward, backward runs rsm_backward.
+    Inputs q, k, v, logits, f (and optionally H0); outputs o and H_T."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, logits, f, K, H0=None):
+        res = forward(q, k, v, logits, f, K, H0)
+        ctx.K = K
+        ctx.save_for_backward(q, k, v, logits, f, H0 if H0 is not None else torch.empty(0, device=q.device))
+        ctx.has_h0 = H0 is not None
+        return res["o"], res["HT"]
+
+    @staticmethod
+    def backward(ctx, dO, dHT):
+        q, k, v, logits, f, H0 = ctx.saved_tensors
+        g = backward(q, k, v, logits, f, ctx.K, None if dO is None else dO.float().contiguous(),
+                     None if dHT is None else dHT.float().contiguous(), H0 if ctx.has_h0 else None)
+        cast = lambda t, like: t.to(like.dtype)
+        return (cast(g["dq"], q), cast(g["dk"], k), cast(g["dv"], v), g["dlogits"], g["df"], None,
+                g["dH0"] if ctx.has_h0 else None)

@@ -247,6 +247,73 @@ rsm_status rsm_decode_step(const rsm_decode_args* a, void* stream) {
   return e == cudaSuccess ? RSM_OK : cuda_fail(e, "rsm_decode_step launch");
 }
 
+static rsm_status check_backward(const rsm_backward_args* a) {
+  if (!a) return fail(RSM_ERR_INVALID_ARG, "args must not be NULL");
+  if (a->B < 0 || a->T < 0 || a->H < 0) return fail(RSM_ERR_INVALID_ARG, "B, T, H must be >= 0");
+  rsm_status s = check_sizes(a->M, a->K, a->Dv);
+  if (s != RSM_OK) return s;
+  if (a->qkv_dtype != RSM_F32 && a->qkv_dtype != RSM_BF16)
+    return fail(RSM_ERR_INVALID_ARG, "unknown qkv_dtype %d", (int)a->qkv_dtype);
+  if (a->decay != RSM_DECAY_HEAD && a->decay != RSM_DECAY_SLOT)
+    return fail(RSM_ERR_INVALID_ARG, "unknown decay %d", (int)a->decay);
+  if (!valid_router(a->router)) return fail(RSM_ERR_INVALID_ARG, "unknown router %d", (int)a->router);
+  if (a->router != RSM_ROUTER_SIGMOID)
+    return fail(RSM_ERR_UNSUPPORTED, "the backward supports the sigmoid router only");
+  if ((int64_t)a->M * a->Dv > 24576)
+    return fail(RSM_ERR_UNSUPPORTED, "the backward keeps the state in shared memory: M*Dv <= 24576 (got %d)",
+                a->M * a->Dv);
+  if ((int64_t)a->B * a->H > (int64_t)0x7fffffff) return fail(RSM_ERR_UNSUPPORTED, "B*H too large");
+  if ((int64_t)a->B * a->T * a->H > 0) {
+    RSM_REQUIRE_PTR(a->q, "q");
+    RSM_REQUIRE_PTR(a->k, "k");
+    RSM_REQUIRE_PTR(a->v, "v");
+    RSM_REQUIRE_PTR(a->logits, "logits");
+    RSM_REQUIRE_PTR(a->f, "f");
+  }
+  RSM_OPTIONAL_PTR(a->H0, "H0");
+  RSM_OPTIONAL_PTR(a->dO, "dO");
+  RSM_OPTIONAL_PTR(a->dHT, "dHT");
+  RSM_OPTIONAL_PTR(a->dq, "dq");
+  RSM_OPTIONAL_PTR(a->dk, "dk");
+  RSM_OPTIONAL_PTR(a->dv, "dv");
+  RSM_OPTIONAL_PTR(a->dlogits, "dlogits");
+  RSM_OPTIONAL_PTR(a->df, "df");
+  RSM_OPTIONAL_PTR(a->dH0, "dH0");
+  return RSM_OK;
+}
+
+size_t rsm_backward_workspace_size(const rsm_backward_args* a) {
+  if (check_backward(a) != RSM_OK) return (size_t)-1;
+  if ((int64_t)a->B * a->T * a->H == 0) return 0;
+  return rsm::backward_workspace_bytes(*a);
+}
+
+rsm_status rsm_backward(const rsm_backward_args* a, void* stream) {
+  g_err[0] = 0;
+  rsm_status s = check_backward(a);
+  if (s != RSM_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((int64_t)a->B * a->H == 0) return RSM_OK;
+  if (a->T == 0) {
+    // no tokens: dL/dH0 = dL/dH_T
+    if (a->dH0) {
+      const size_t bytes = (size_t)a->B * a->H * a->M * a->Dv * sizeof(float);
+      cudaError_t e = a->dHT ? cudaMemcpyAsync(a->dH0, a->dHT, bytes, cudaMemcpyDeviceToDevice, st)
+                             : cudaMemsetAsync(a->dH0, 0, bytes, st);
+      if (e != cudaSuccess) return cuda_fail(e, "rsm_backward (T=0)");
+    }
+    return RSM_OK;
+  }
+  const size_t need = rsm::backward_workspace_bytes(*a);
+  if (!a->workspace || a->workspace_bytes < need)
+    return fail(RSM_ERR_WORKSPACE, "workspace of %zu bytes required (got %zu)", need,
+                a->workspace ? a->workspace_bytes : (size_t)0);
+  if ((reinterpret_cast<uintptr_t>(a->workspace) & 255u) != 0)
+    return fail(RSM_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  cudaError_t e = rsm::launch_backward(*a, st);
+  return e == cudaSuccess ? RSM_OK : cuda_fail(e, "rsm_backward launch");
+}
+
 rsm_status rsm_get_device_status(void* stream) {
   g_err[0] = 0;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

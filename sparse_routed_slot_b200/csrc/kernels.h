@@ -27,6 +27,11 @@ cudaError_t launch_record_counts(const unsigned char* rec, int64_t pairs, int64_
 
 cudaError_t launch_decode(const rsm_decode_args& a, cudaStream_t stream);
 
+// Gradients on CUDA cores (backward.cu).
+size_t backward_smem_bytes(int M, int K, int Dv);
+size_t backward_workspace_bytes(const rsm_backward_args& a);
+cudaError_t launch_backward(const rsm_backward_args& a, cudaStream_t stream);
+
 // CUDA-core fp32 chunked prefill (any supported size).
 cudaError_t launch_prefill_simt(const rsm_forward_args& a, cudaStream_t stream);
 size_t prefill_simt_smem_bytes(int M, int Dv);
