@@ -103,8 +103,9 @@ constexpr int kSmemBytes = kOffSmall + kSmallBytes + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 struct Maps {
-  CUtensorMap v;  // v [B,T,H,Dv] bf16, box: one (b,h), 64 tokens
-  CUtensorMap o;  // o [B,T,H,Dv] fp32, box: one (b,h), 32 tokens (output stores)
+  CUtensorMap v;    // v [B,T,H,Dv] bf16, box: one (b,h), 64 tokens
+  CUtensorMap vsw;  // v [B,T,H,Dv] bf16, box: 64 value columns of one (b,h), 64 tokens, 128B swizzle
+  CUtensorMap o;    // o [B,T,H,Dv] fp32, box: one (b,h), 32 tokens (output stores)
 };
 
 struct Params {
@@ -116,8 +117,10 @@ struct Params {
   float* o;
   float* HT;
   int nseg, seg_chunks;
-  float* ws_state;  // [pairs][nseg][M][Dv]: slot 0 = start state, slot j+1 = summary of segment j
-  float* ws_D;      // [pairs][nseg][M]
+  int sub, piece_chunks;  // summary pieces per segment and their length in chunks
+  int nslot;              // 1 + (nseg - 1) * sub
+  float* ws_state;  // [pairs][nslot][M][Dv]: slot 0 = start state, slot 1 + k = summary of piece k
+  float* ws_D;      // [pairs][nslot][M]
 };
 
 RSM_DEV float4 bf16x4_to_f32(uint2 r) {
@@ -658,7 +661,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
 
     // the state of chunk ck's item into TMEM (H0, a segment start state, or zeros)
     auto load_state = [&](const Chunk& ck) {
-      const float* Hs = p.nseg > 1 ? p.ws_state + ((int64_t)ck.pair * p.nseg + ck.seg) * kM * kDV
+      const float* Hs = p.nseg > 1 ? p.ws_state + ((int64_t)ck.pair * p.nslot + ck.seg * p.sub) * kM * kDV
                                    : (p.H0 ? p.H0 + (int64_t)ck.pair * kM * kDV : nullptr);
 #pragma unroll 1
       for (int c = 0; c < kM; c += 32) {
@@ -816,46 +819,63 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
 //   U    = sum_t Wr_t^T v_t,  Wr_{t,i} = w_{t,i} e^{sum of lam_{s,i} over the segment's tokens s > t}
 // Referenced to the segment end, every exponent is <= 0: no division, no fast/exact split, and no
 // decay of an accumulator between chunks, so U is a single accumulation of V^T Wr over the
-// segment (one TMEM accumulator, chunk tiles double-buffered). The chunks are visited from the
+// segment (one TMEM accumulator). The chunks are visited from the
 // segment's last to its first, so the exponent of a token is the running sum of the lam of the
 // tokens after it.
 //
-// Warp roles (one CTA per segment at a time, 13 warps):
+// The products run on bf16 operands (kind::f16): v as stored (its TMA tile, used MN-major), and Wr
+// split into a bf16 high part and a bf16 low part (two MMAs, about 16 significant bits together),
+// accumulated in fp32.
+//
+// Warp roles (two CTAs per SM, each on one segment at a time, 9 warps):
 //   warps 0-7  row workers; warp w owns tokens 8w..8w+7 of the chunk, lane l slots 4l..4l+3 of
 //              the lam table. Per chunk: scatter the rows' lam into the table, walk the rows from
 //              the last to the first (exclusive in-warp suffix sums in place), exchange the warp
-//              totals, write Wr^T at the selected entries; at the segment's end read U out of TMEM
-//              and write U and D.
-//   warp 8     MMA issuer (one thread): the v tile loads (two chunks ahead) and the 8 MMAs of
-//              each chunk, U^T += V^T Wr (M = value columns, N = slots, K = tokens).
-//   warps 9-12 converters: each chunk's v tile into V^T (warp c: tokens 16c..16c+15), beside the
-//              row workers' chain instead of at its end.
-constexpr int kSumConvWarps = 4;
-constexpr int kSumConvThreads = kSumConvWarps * 32;
-constexpr int kSumThreads = (kRWarps + 1 + kSumConvWarps) * 32;
-constexpr int kSumOffRawV = 0;                       // v tiles from TMA, [2][64 t][128 dv] bf16
-constexpr int kSumOffVt = kSumOffRawV + 32768;       // V^T  [2][128 dv][64 t] (A)
-constexpr int kSumOffWt = kSumOffVt + 2 * 32768;     // Wr^T [2][128 slot][64 t] (B)
-constexpr int kSumOffTab = kSumOffWt + 2 * 32768;    // lam table [64 t][128 slot], then exponents
+//              totals, write Wr (high and low tiles) at the selected entries; at the segment's end
+//              read U out of TMEM and write U and D.
+//   warp 8     MMA issuer (lane 0 issues): the v tile loads (one chunk ahead) and the 8 MMAs of
+//              each chunk, U^T += V^T Wr (M = value columns, N = slots, K = 16 tokens per step,
+//              high and low part).
+// One Wr tile pair: the row workers build a chunk's table and exponents while the MMAs of the
+// chunk before run, and write its Wr once they are done.
+constexpr int kSumThreads = (kRWarps + 1) * 32;
+constexpr int kSumOffV = 0;                          // v tiles [2][2 halves][64 t][64 dv] bf16, 128B swizzled
+constexpr int kSumOffWb = kSumOffV + 2 * 16384;      // Wr high, low [2][64 t][128 slot] bf16, MN-major
+constexpr int kSumOffTab = kSumOffWb + 32768;        // lam table [64 t][128 slot], then exponents
 constexpr int kSumOffTot = kSumOffTab + 32768;       // per-warp lam sums [2][8][128]
 constexpr int kSumOffSuf = kSumOffTot + 2 * kRWarps * kM * 4;  // per-warp exponent offsets [8][128]
 constexpr int kSumSmemBytes = kSumOffSuf + kRWarps * kM * 4 + 1024;
+constexpr int kSumCtasPerSm = 2;
 constexpr int kSumTmemCols = 128;
-static_assert(kSumSmemBytes <= 232448, "shared memory budget");
+static_assert(kSumCtasPerSm * (kSumSmemBytes + 1024) <= 233472, "two summary CTAs per SM");
 
-// The summary kernel visits item (pair, seg) = blockIdx.x + j*gridDim.x, seg < nseg - 1, and the
-// item's chunks from the last to the first; first/last refer to that visiting order.
+// The bf16 high and low tiles of Wr ([64 t][128 slot] each, MN-major, 16 KB apart): row t, slot i.
+RSM_DEV void put_wr_bf16(unsigned char* sWb, int t, int i, float x) {
+  uint16_t hi, lo;
+  tc::split_bf16(x, hi, lo);
+  const uint32_t off = tc::swz16_offset(kC, t, i);
+  *reinterpret_cast<uint16_t*>(sWb + off) = hi;
+  *reinterpret_cast<uint16_t*>(sWb + 16384 + off) = lo;
+}
+
+// The summary kernel visits item (pair, piece) = blockIdx.x + j*gridDim.x, piece < (nseg - 1) * sub
+// (piece q of segment j is piece j*sub + q; a segment's pieces split its chunks evenly), and the
+// item's chunks from the last to the first; first/last refer to that visiting order. A chunk's
+// `seg` field holds the piece.
 struct SumWalker {
-  int item, pair, seg, b, h, t0, nch, i;
+  int item, pair, piece, b, h, t0, t1, nch, i;
   __device__ void set_item(const Params& p, int items) {
     if (item >= items) return;
     const int pairs = p.B * p.H;
-    seg = item / pairs;
-    pair = item - seg * pairs;
+    piece = item / pairs;
+    pair = item - piece * pairs;
     b = pair / p.H;
     h = pair - b * p.H;
-    t0 = seg * p.seg_chunks * kC;
-    const int t1 = min(p.T, t0 + p.seg_chunks * kC);
+    const int seg = piece / p.sub, q = piece - seg * p.sub;
+    const int c0 = seg * p.seg_chunks + q * p.piece_chunks;
+    const int c1 = min((seg + 1) * p.seg_chunks, c0 + p.piece_chunks);
+    t0 = c0 * kC;
+    t1 = min(p.T, c1 * kC);
     nch = (t1 - t0 + kC - 1) / kC;
     i = 0;
   }
@@ -867,11 +887,11 @@ struct SumWalker {
   __device__ Chunk get(const Params& p) const {
     Chunk c;
     c.pair = pair;
-    c.seg = seg;
+    c.seg = piece;
     c.b = b;
     c.h = h;
     c.c0 = t0 + (nch - 1 - i) * kC;
-    c.nrows = min(kC, min(p.T, t0 + p.seg_chunks * kC) - c.c0);
+    c.nrows = min(kC, t1 - c.c0);
     c.first = i == 0;
     c.last = i == nch - 1;
     return c;
@@ -885,44 +905,41 @@ struct SumWalker {
 };
 
 template <int KP>
-__global__ void __launch_bounds__(kSumThreads, 1) segment_summary_kernel(const __grid_constant__ Maps maps,
-                                                                          const Params p) {
+__global__ void __launch_bounds__(kSumThreads, kSumCtasPerSm) segment_summary_kernel(const __grid_constant__ Maps maps,
+                                                                                     const Params p) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  unsigned char* sRawV = sm + kSumOffRawV;
-  unsigned char* sVt = sm + kSumOffVt;
-  unsigned char* sWt = sm + kSumOffWt;
+  unsigned char* sV = sm + kSumOffV;
+  unsigned char* sWb = sm + kSumOffWb;  // [high | low]
   float* sTab = reinterpret_cast<float*>(sm + kSumOffTab);
   float* sTot = reinterpret_cast<float*>(sm + kSumOffTot);
   float* sSuf = reinterpret_cast<float*>(sm + kSumOffSuf);
 
-  __shared__ __align__(8) uint64_t bar_rdy[2],  // Wr^T of chunk n in buffer n&1 written (row threads)
-      bar_vt[2],                                 // V^T of chunk n in buffer n&1 written  (converters)
-      bar_tma[2],                                // raw v tile of chunk n landed          (TMA)
-      bar_mma[2],                                // MMAs of chunk n done, buffer n&1 free (MMA commit)
-      bar_out,                                   // U of an item read out of TMEM         (row threads)
-      bar_fin;                                   // issuer only: every MMA issued is done (MMA commit)
+  // mbarriers (phase k of a barrier = its k-th completion)
+  __shared__ __align__(8) uint64_t bar_rdy,  // Wr of chunk n written                  (row threads)
+      bar_tma[2],                             // v tile of chunk n landed, buffer n&1   (TMA)
+      bar_mma,                                // MMAs of chunk n done                   (MMA commit)
+      bar_out,                                // U of an item read out of TMEM          (row threads)
+      bar_fin;                                // issuer only: every MMA issued is done  (MMA commit)
   __shared__ uint32_t s_tbase;
   __shared__ int s_abort;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int K = p.K;
-  const int items = p.B * p.H * (p.nseg - 1);
+  const int items = p.B * p.H * (p.nslot - 1);
 
   if (warp == kIssuerWarp) tc::tmem_alloc(&s_tbase, kSumTmemCols);
   if (tid == 0) {
-    for (int b = 0; b < 2; ++b) {
-      tc::mbar_init(&bar_rdy[b], kRThreads);
-      tc::mbar_init(&bar_vt[b], kSumConvThreads);
-      tc::mbar_init(&bar_tma[b], 1);
-      tc::mbar_init(&bar_mma[b], 1);
-    }
+    tc::mbar_init(&bar_rdy, kRThreads);
+    tc::mbar_init(&bar_tma[0], 1);
+    tc::mbar_init(&bar_tma[1], 1);
+    tc::mbar_init(&bar_mma, 1);
     tc::mbar_init(&bar_out, kRThreads);
     tc::mbar_init(&bar_fin, 1);
     tc::fence_mbar_init();
     s_abort = 0;
   }
-  if (warp == kIssuerWarp && lane == 0) tc::tma_prefetch_desc(&maps.v);
+  if (warp == kIssuerWarp && lane == 0) tc::tma_prefetch_desc(&maps.vsw);
   tc::tmem_fence_before();
   __syncthreads();
   tc::tmem_fence_after();
@@ -937,25 +954,20 @@ __global__ void __launch_bounds__(kSumThreads, 1) segment_summary_kernel(const _
     const int w = warp;
     float* tab = sTab + w * kRowsPerWarp * kM;  // this warp's rows of the table
     float lamS[4] = {0.f, 0.f, 0.f, 0.f};      // Lam of the item's tokens after this chunk (slots 4l..)
-    // The table rows and the warp's token columns of both Wr^T buffers start at zero; afterwards each
+    // The table rows and the warp's token rows of the Wr tiles start at zero; afterwards each
     // entry's owner clears what it wrote (sparse), so no chunk fills them densely.
-    uint32_t es2[RowInputs<KP>::kGroups], es1[RowInputs<KP>::kGroups];  // entry slots of chunks n-2, n-1
+    uint32_t es1[RowInputs<KP>::kGroups];  // entry slots of the chunk before
 #pragma unroll
     for (int i = 0; i < kRowsPerWarp; ++i)
       reinterpret_cast<float4*>(tab)[lane + 32 * i] = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int b = 0; b < 2; ++b) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int slot = lane + 32 * e;
-        unsigned char* wt = sWt + b * 32768;
-        *reinterpret_cast<float4*>(wt + tc::swz_offset(kM, slot, w * kRowsPerWarp)) = make_float4(0.f, 0.f, 0.f, 0.f);
-        *reinterpret_cast<float4*>(wt + tc::swz_offset(kM, slot, w * kRowsPerWarp + 4)) =
-            make_float4(0.f, 0.f, 0.f, 0.f);
-      }
+    for (int r = 0; r < kRowsPerWarp; ++r) {
+      const uint32_t off = tc::swz16_offset(kC, w * kRowsPerWarp + r, lane * 4);
+      *reinterpret_cast<uint2*>(sWb + off) = make_uint2(0u, 0u);
+      *reinterpret_cast<uint2*>(sWb + 16384 + off) = make_uint2(0u, 0u);
     }
 #pragma unroll
-    for (int g = 0; g < RowInputs<KP>::kGroups; ++g) es2[g] = es1[g] = 0u;
+    for (int g = 0; g < RowInputs<KP>::kGroups; ++g) es1[g] = 0u;
     __syncwarp();
     RowInputs<KP> cur;
     if (wk.valid(items)) load_rows<true, KP>(p, wk.get(p), w, lane, cur);
@@ -1003,11 +1015,9 @@ __global__ void __launch_bounds__(kSumThreads, 1) segment_summary_kernel(const _
 #pragma unroll
       for (int e = 0; e < 4; ++e) lamS[e] += tot[e];
       reinterpret_cast<float4*>(sSuf + w * kM)[lane] = make_float4(suf[0], suf[1], suf[2], suf[3]);
-      // ---- Wr^T buffer `buf` is free once the MMAs of chunk n-2 are done
-      if (n >= 2) wait_or_abort(&bar_mma[buf], ((n - 2) >> 1) & 1, abort_flag);
-      unsigned char* wt = sWt + buf * 32768;
-      // the entries of chunk n-2 leave this buffer (rows past a chunk's end hold slot 0, which
-      // clears a zero)
+      // ---- the Wr tiles are free once the MMAs of the chunk before are done; that chunk's entries
+      // leave them (rows past a chunk's end hold slot 0, which clears a zero)
+      if (n >= 1) wait_or_abort(&bar_mma, (n - 1) & 1, abort_flag);
 #pragma unroll
       for (int g = 0; g < RowInputs<KP>::kGroups; ++g) {
         int r, j0;
@@ -1015,11 +1025,11 @@ __global__ void __launch_bounds__(kSumThreads, 1) segment_summary_kernel(const _
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           if (r < kRowsPerWarp && j0 + e < K) {
-            const int slot = (int)((es2[g] >> (8 * e)) & 255u);
-            *reinterpret_cast<float*>(wt + tc::swz_offset(kM, slot, w * kRowsPerWarp + r)) = 0.f;
+            const uint32_t off = tc::swz16_offset(kC, w * kRowsPerWarp + r, (int)((es1[g] >> (8 * e)) & 255u));
+            *reinterpret_cast<uint16_t*>(sWb + off) = 0;
+            *reinterpret_cast<uint16_t*>(sWb + 16384 + off) = 0;
           }
         }
-        es2[g] = es1[g];
         es1[g] = cur.es[g];
       }
       __syncwarp();
@@ -1027,16 +1037,16 @@ __global__ void __launch_bounds__(kSumThreads, 1) segment_summary_kernel(const _
       for_entries(cur, lane, K, nrows_w, [&](int r, int slot, float, float wv) {
         const float x = tab[r * kM + slot] + sSuf[w * kM + slot];
         tab[r * kM + slot] = 0.f;
-        *reinterpret_cast<float*>(wt + tc::swz_offset(kM, slot, w * kRowsPerWarp + r)) = tc::to_tf32(wv * expf(x));
+        put_wr_bf16(sWb, w * kRowsPerWarp + r, slot, wv * expf(x));
       });
       tc::fence_async_smem();
-      mbar_arrive(&bar_rdy[buf]);
+      mbar_arrive(&bar_rdy);
       // ---- the item's last chunk: U out of TMEM (warp w: lanes 32(w%4).., slot columns
       // 64(w/4)..), D = e^Lam
       if (ck.last) {
-        wait_or_abort(&bar_mma[buf], (n >> 1) & 1, abort_flag);
+        wait_or_abort(&bar_mma, n & 1, abort_flag);
         tc::tmem_fence_after();
-        const int64_t slot_base = ((int64_t)ck.pair * p.nseg + ck.seg + 1);
+        const int64_t slot_base = ((int64_t)ck.pair * p.nslot + ck.seg + 1);
         float* dst = p.ws_state + slot_base * kM * kDV;
         const int dv = (w & 3) * 32 + lane;
         const int c0 = (w >> 2) * 64;
@@ -1058,50 +1068,54 @@ __global__ void __launch_bounds__(kSumThreads, 1) segment_summary_kernel(const _
       }
       cur = nxt;
     }
-  } else if (warp == kIssuerWarp) {
+  } else {
     // =========================================================================== MMA issuer
     // The whole warp runs the issuer's loop, so that its descriptors and addresses are
     // warp-uniform values; lane 0 alone issues the copies, the MMAs and their commits.
     const bool leader = lane == 0;
     {
       uint32_t n = 0, n_tma = 0, n_items = 0;
-      auto load_v = [&](const SumWalker& at, uint32_t j) {  // v tile of the walker's chunk, as chunk j
+      // v tile of the walker's chunk, as chunk j, into buffer j&1: two 64-column halves, each
+      // [64 t][64 dv] bf16 with 128-byte swizzle (the MN-major operand layout); rows past the
+      // sequence end are zero
+      auto load_v = [&](const SumWalker& at, uint32_t j) {
         if (!at.valid(items)) return;
         const Chunk c = at.get(p);
         if (leader) {
           tc::mbar_arrive_expect_tx(&bar_tma[j & 1], kC * kDV * 2);
-          tc::tma_load_4d(sRawV + (j & 1) * (kC * kDV * 2), &maps.v, &bar_tma[j & 1], 0, c.h, c.c0, c.b);
+          tc::tma_load_4d(sV + (j & 1) * 16384, &maps.vsw, &bar_tma[j & 1], 0, c.h, c.c0, c.b);
+          tc::tma_load_4d(sV + (j & 1) * 16384 + 8192, &maps.vsw, &bar_tma[j & 1], 64, c.h, c.c0, c.b);
         }
         ++n_tma;
       };
-      {
-        SumWalker nx = wk;
-        load_v(nx, 0);
-        nx.next(p, items);
-        load_v(nx, 1);
-      }
-      auto kstep = [](int R, int j) -> uint64_t { return (uint64_t)(((j >> 2) * (R * 128) + (j & 3) * 32) >> 4); };
-      constexpr uint32_t kIdC = tc::idesc_tf32(kDV, kM, 0, 0);
-      const uint64_t dVt0 = tc::smem_desc(tc::smem_u32(sVt), 16, 1024), dWt0 = tc::smem_desc(tc::smem_u32(sWt), 16, 1024);
+      load_v(wk, 0);
+      // v: 64-column halves 8 KB apart, groups of 8 token rows 1 KB apart; Wr: 64-slot halves 8 KB
+      // apart, the same row groups; a K step of 16 tokens advances both by 2 KB
+      const uint64_t dV0 = tc::smem_desc(tc::smem_u32(sV), 8192, 1024), dWb = tc::smem_desc(tc::smem_u32(sWb), 8192, 1024);
+      constexpr uint32_t kIdC = tc::idesc_bf16(kDV, kM, 1, 1);
       for (; wk.valid(items) && !*abort_flag; ++n, wk.next(p, items)) {
         const Chunk ck = wk.get(p);
-        const int buf = n & 1;
-        wait_or_abort(&bar_rdy[buf], (n >> 1) & 1, abort_flag);  // Wr^T written
-        wait_or_abort(&bar_vt[buf], (n >> 1) & 1, abort_flag);   // V^T written, raw v consumed
         {
-          SumWalker nx = wk;  // the raw v buffer is free again: the chunk two ahead
+          // buffer (n+1)&1 is free once the MMAs of chunk n-1 are done: the next chunk's v into it
+          if (n >= 1) wait_or_abort(&bar_mma, (n - 1) & 1, abort_flag);
+          SumWalker nx = wk;
           nx.next(p, items);
-          nx.next(p, items);
-          load_v(nx, n + 2);
+          load_v(nx, n + 1);
         }
+        wait_or_abort(&bar_rdy, n & 1, abort_flag);                   // Wr written
+        wait_or_abort(&bar_tma[n & 1], (n >> 1) & 1, abort_flag);     // v landed
         // the accumulator of the item before has been read out
         if (ck.first && n_items > 0) wait_or_abort(&bar_out, (n_items - 1) & 1, abort_flag);
         tc::tmem_fence_after();
-        const uint64_t dVt = dVt0 + (uint64_t)((buf * 32768) >> 4), dWt = dWt0 + (uint64_t)((buf * 32768) >> 4);
+        const uint64_t dVn = dV0 + (uint64_t)(((n & 1) * 16384) >> 4);
 #pragma unroll
-        for (int j = 0; j < kC / 8; ++j)
-          if (leader) tc::mma_tf32_ss(tb, dVt + kstep(kDV, j), dWt + kstep(kM, j), kIdC, (ck.first && j == 0) ? 0u : 1u);
-        if (leader) tc::mma_commit(&bar_mma[buf]);
+        for (int j = 0; j < kC / 16; ++j)
+#pragma unroll
+          for (int part = 0; part < 2; ++part)
+            if (leader)
+              tc::mma_bf16_ss(tb, dVn + (uint64_t)((j * 2048) >> 4), dWb + (uint64_t)((part * 16384 + j * 2048) >> 4),
+                              kIdC, (ck.first && j == 0 && part == 0) ? 0u : 1u);
+        if (leader) tc::mma_commit(&bar_mma);
         if (ck.last) ++n_items;
       }
       // nothing may still be running when the CTA releases its memory
@@ -1110,32 +1124,6 @@ __global__ void __launch_bounds__(kSumThreads, 1) segment_summary_kernel(const _
       for (uint32_t j = n; j < n_tma; ++j) tc::mbar_wait(&bar_tma[j & 1], (j >> 1) & 1);
     }
     __syncwarp();
-  } else {
-    // =========================================================================== converters
-    const int c = warp - (kRWarps + 1);  // tokens 16c..16c+15 of each chunk
-    for (uint32_t n = 0; wk.valid(items) && !*abort_flag; ++n, wk.next(p, items)) {
-      const int buf = n & 1;
-      if (n >= 2) wait_or_abort(&bar_mma[buf], ((n - 2) >> 1) & 1, abort_flag);  // V^T buffer free
-      wait_or_abort(&bar_tma[buf], (n >> 1) & 1, abort_flag);                    // v tile landed
-      const uint16_t* raw = reinterpret_cast<const uint16_t*>(sRawV + buf * (kC * kDV * 2));
-      unsigned char* vt = sVt + buf * 32768;
-      // value columns lane + 32e (8 consecutive rows per 8 lanes: 4-way stores); rows past the
-      // sequence end are zero in the tile
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int dv = lane + 32 * e;
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const int t0 = 16 * c + 4 * g;
-          float x[4];
-#pragma unroll
-          for (int r = 0; r < 4; ++r) x[r] = __uint_as_float((uint32_t)raw[(t0 + r) * kDV + dv] << 16);
-          *reinterpret_cast<float4*>(vt + tc::swz_offset(kDV, dv, t0)) = make_float4(x[0], x[1], x[2], x[3]);
-        }
-      }
-      tc::fence_async_smem();
-      mbar_arrive(&bar_vt[buf]);
-    }
   }
 
   tc::tmem_fence_before();
@@ -1144,20 +1132,20 @@ __global__ void __launch_bounds__(kSumThreads, 1) segment_summary_kernel(const _
   if (warp == kIssuerWarp) tc::tmem_dealloc(tb, kSumTmemCols);
 }
 
-// Combines the segment summaries of each (b,h) into start states:
-// state[0] = H0 (or 0); state[j] = D_{j-1} * state[j-1] + U_{j-1} (the summary of segment j-1 is
-// stored in slot j and is replaced in place). A slot with D = 1 and U = 0 (not selected in the
-// segment) keeps its bits.
+// Combines the piece summaries of each (b,h) into states:
+// state[0] = H0 (or 0); state[k] = D_{k-1} * state[k-1] + U_{k-1} (the summary of piece k-1 is
+// stored in slot k and is replaced in place), so slot j*sub ends up holding the start state of
+// segment j. A slot with D = 1 and U = 0 (not selected in the piece) keeps its bits.
 __global__ void __launch_bounds__(256) segment_scan_kernel(const Params p) {
   const int pair = blockIdx.y;
   const int e = blockIdx.x * blockDim.x + threadIdx.x;  // element (slot, column)
   if (e >= kM * kDV) return;
   const int i = e / kDV;
-  float* st = p.ws_state + (int64_t)pair * p.nseg * kM * kDV;
-  const float* D = p.ws_D + (int64_t)pair * p.nseg * kM;
+  float* st = p.ws_state + (int64_t)pair * p.nslot * kM * kDV;
+  const float* D = p.ws_D + (int64_t)pair * p.nslot * kM;
   float hcur = p.H0 ? p.H0[(int64_t)pair * kM * kDV + e] : 0.f;
   st[e] = hcur;
-  for (int j = 1; j < p.nseg; ++j) {
+  for (int j = 1; j < p.nslot; ++j) {
     const float d = D[j * kM + i], u = st[(int64_t)j * kM * kDV + e];
     if (d != 1.f || u != 0.f) hcur = fmaf(d, hcur, u);
     st[(int64_t)j * kM * kDV + e] = hcur;
@@ -1185,16 +1173,18 @@ EncodeTiledFn encode_fn() {
 }
 
 // 4-D map over [B, T, H, C] (C innermost) with a box of one (b, h) and `box_t` tokens.
-bool make_map(CUtensorMap* m, const void* base, int B, int T, int H, int C, bool fp32, int box_t) {
+bool make_map(CUtensorMap* m, const void* base, int B, int T, int H, int C, bool fp32, int box_t, int box_c = 0,
+              bool swizzle128 = false) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t es = fp32 ? 4 : 2;
   cuuint64_t dims[4] = {(cuuint64_t)C, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
   cuuint64_t strides[3] = {(cuuint64_t)C * es, (cuuint64_t)H * C * es, (cuuint64_t)T * H * C * es};
-  cuuint32_t box[4] = {(cuuint32_t)C, 1, (cuuint32_t)box_t, 1};
+  cuuint32_t box[4] = {(cuuint32_t)(box_c > 0 ? box_c : C), 1, (cuuint32_t)box_t, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   return fn(m, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base),
-            dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -1202,6 +1192,7 @@ int sm_count() { return device_sm_count(); }
 
 struct Plan {
   int nseg, seg_chunks;
+  int sub, piece_chunks, nslot;
 };
 
 Plan plan_for(const rsm_forward_args& a, int sms) {
@@ -1214,7 +1205,12 @@ Plan plan_for(const rsm_forward_args& a, int sms) {
   int seg_chunks = (nchunks + nseg - 1) / nseg;
   if (seg_chunks < 1) seg_chunks = 1;
   nseg = std::max(1, (nchunks + seg_chunks - 1) / seg_chunks);
-  return {nseg, seg_chunks};
+  // the summary pass runs two CTAs per SM: each segment it summarises is split into that many
+  // pieces (of at least 4 chunks), combined by the scan
+  int sub = seg_chunks >= 4 * kSumCtasPerSm ? kSumCtasPerSm : 1;
+  const int piece_chunks = (seg_chunks + sub - 1) / sub;
+  sub = (seg_chunks + piece_chunks - 1) / piece_chunks;
+  return {nseg, seg_chunks, sub, piece_chunks, 1 + (nseg - 1) * sub};
 }
 
 size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -1230,7 +1226,7 @@ WsLayout ws_layout(const rsm_forward_args& a, const Plan& pl) {
   size_t off = up256(rows * (size_t)route_record_bytes(a.K));
   l.state = l.D = off;
   if (pl.nseg > 1) {
-    const size_t per = (size_t)a.B * a.H * pl.nseg;
+    const size_t per = (size_t)a.B * a.H * pl.nslot;
     l.state = off;
     off += up256(per * kM * kDV * 4);
     l.D = off;
@@ -1250,8 +1246,8 @@ cudaError_t launch_passes(const Maps& maps, const Params& p, const Plan& pl, int
   if (pl.nseg > 1) {
     e = set_smem_limit<segment_summary_kernel<KP>>(kSumSmemBytes);
     if (e != cudaSuccess) return e;
-    const int items = (int)(pairs * (pl.nseg - 1));
-    segment_summary_kernel<KP><<<std::min(items, sms), kSumThreads, kSumSmemBytes, stream>>>(maps, p);
+    const int items = (int)(pairs * (pl.nslot - 1));
+    segment_summary_kernel<KP><<<std::min(items, kSumCtasPerSm * sms), kSumThreads, kSumSmemBytes, stream>>>(maps, p);
     e = cudaGetLastError();
     if (e == cudaSuccess) e = profile_mark(stream);
     if (e != cudaSuccess) return e;
@@ -1301,6 +1297,7 @@ cudaError_t launch_prefill_tc(const rsm_forward_args& a, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   Maps maps;
   if (!make_map(&maps.v, a.v, a.B, a.T, a.H, kDV, false, kC)) return cudaErrorInvalidValue;
+  if (!make_map(&maps.vsw, a.v, a.B, a.T, a.H, kDV, false, kC, 64, true)) return cudaErrorInvalidValue;
   if (!make_map(&maps.o, a.o, a.B, a.T, a.H, kDV, true, kC / 2)) return cudaErrorInvalidValue;
   Params p;
   p.B = a.B; p.T = a.T; p.H = a.H; p.K = a.K;
@@ -1310,6 +1307,7 @@ cudaError_t launch_prefill_tc(const rsm_forward_args& a, cudaStream_t stream) {
   p.H0 = a.H0;
   p.o = a.o; p.HT = a.HT;
   p.nseg = pl.nseg; p.seg_chunks = pl.seg_chunks;
+  p.sub = pl.sub; p.piece_chunks = pl.piece_chunks; p.nslot = pl.nslot;
   p.ws_state = nullptr; p.ws_D = nullptr;
   if (pl.nseg > 1) {
     p.ws_state = reinterpret_cast<float*>(ws + wl.state);

@@ -9,6 +9,7 @@
 // transposed instead.
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -190,6 +191,53 @@ __host__ __device__ constexpr uint32_t idesc_tf32(int M, int N, int a_mn, int b_
          | ((uint32_t)b_mn << 16)       // B major
          | ((uint32_t)(N >> 3) << 17)   // N / 8
          | ((uint32_t)(M >> 4) << 24);  // M / 16
+}
+
+// Instruction descriptor: bf16 x bf16 -> f32 (kind::f16), dense, no negation.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_mn) {
+  return (1u << 4)                      // D format f32
+         | (1u << 7)                    // A format bf16
+         | (1u << 10)                   // B format bf16
+         | ((uint32_t)a_mn << 15)       // A major
+         | ((uint32_t)b_mn << 16)       // B major
+         | ((uint32_t)(N >> 3) << 17)   // N / 8
+         | ((uint32_t)(M >> 4) << 24);  // M / 16
+}
+
+// Byte offset of 16-bit element (row, col) in a 128-byte-swizzled tile of R rows: C/64 column
+// blocks of R rows x 128 bytes (64 elements); inside a block, row r, element c (0..63) sits at
+// r*128 + (((c/8) ^ (r%8)) * 16) + (c%8)*2. Used K-major (rows = M or N, columns = K) and MN-major
+// (rows = K, columns = M or N: the layout TMA writes with 128-byte swizzle).
+__host__ __device__ __forceinline__ uint32_t swz16_offset(int R, int row, int col) {
+  return (uint32_t)((col >> 6) * (R * 128) + row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4) + ((col & 7) << 1));
+}
+
+// x as a pair of bf16 values (hi + lo = x to about 16 significant bits): hi = the upper 16 bits
+// of x (bf16 by truncation, exact to subtract), lo = bf16(x - hi) rounded to nearest. Returns the
+// raw 16-bit patterns.
+RSM_DEV void split_bf16(float x, uint16_t& hi, uint16_t& lo) {
+  const uint32_t b = __float_as_uint(x);
+  hi = (uint16_t)(b >> 16);
+  lo = __bfloat16_as_ushort(__float2bfloat16_rn(x - __uint_as_float(b & 0xffff0000u)));
+}
+
+// Two values (x0 at the lower address) as packed bf16 pairs: the high parts and the low parts.
+RSM_DEV void split_bf16x2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  const uint32_t b0 = __float_as_uint(x0), b1 = __float_as_uint(x1);
+  hi = __byte_perm(b0, b1, 0x7632);  // upper halves: x0's at bits 0..15, x1's at 16..31
+  const __nv_bfloat162 l = __floats2bfloat162_rn(x0 - __uint_as_float(b0 & 0xffff0000u),
+                                                 x1 - __uint_as_float(b1 & 0xffff0000u));
+  lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+
+// D[tmem] (+)= A[smem desc] * B[smem desc], kind::f16 (bf16 operands)
+RSM_DEV void mma_bf16_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
 }
 
 // D[tmem] (+)= A[smem desc] * B[smem desc]
