@@ -237,8 +237,8 @@ RSM_API rsm_status rsm_decode_step(const rsm_decode_args* args, void* stream);
  *   dq, dk, dlogits [B,T,H,M] fp32; dv [B,T,H,Dv] fp32; df [B,T,H] or [B,T,H,M] fp32;
  *   dH0 [B,H,M,Dv] fp32 (each output may be NULL to skip it)
  *   workspace: at least rsm_backward_workspace_size(args) bytes (256-byte aligned): the routing
- *     of every token and a tape of the K state rows each token overwrites (T*K*Dv*4 bytes per
- *     (b,h) stream).
+ *     of every token, its K entries (slot, decay, write weight, score, rate, key; 32 bytes each)
+ *     and a tape of the K state rows each token overwrites (T*K*Dv*4 bytes per (b,h) stream).
  *   Supported: the sizes of rsm_forward with M*Dv <= 24576 (the state and its gradient stay in
  *   shared memory), router RSM_ROUTER_SIGMOID. The arithmetic is fp32 on CUDA cores.
  * ------------------------------------------------------------------------------------------- */

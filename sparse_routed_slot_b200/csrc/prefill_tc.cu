@@ -1145,10 +1145,26 @@ __global__ void __launch_bounds__(256) segment_scan_kernel(const Params p) {
   const float* D = p.ws_D + (int64_t)pair * p.nslot * kM;
   float hcur = p.H0 ? p.H0[(int64_t)pair * kM * kDV + e] : 0.f;
   st[e] = hcur;
-  for (int j = 1; j < p.nslot; ++j) {
-    const float d = D[j * kM + i], u = st[(int64_t)j * kM * kDV + e];
-    if (d != 1.f || u != 0.f) hcur = fmaf(d, hcur, u);
-    st[(int64_t)j * kM * kDV + e] = hcur;
+  // the summaries are loaded 8 at a time ahead of the dependent chain (one memory round trip per 8)
+  constexpr int kBatch = 8;
+  for (int j0 = 1; j0 < p.nslot; j0 += kBatch) {
+    float d[kBatch], u[kBatch];
+#pragma unroll
+    for (int k = 0; k < kBatch; ++k) {
+      d[k] = 1.f;
+      u[k] = 0.f;
+      if (j0 + k < p.nslot) {
+        d[k] = D[(j0 + k) * kM + i];
+        u[k] = st[(int64_t)(j0 + k) * kM * kDV + e];
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kBatch; ++k) {
+      if (j0 + k < p.nslot) {
+        if (d[k] != 1.f || u[k] != 0.f) hcur = fmaf(d[k], hcur, u[k]);
+        st[(int64_t)(j0 + k) * kM * kDV + e] = hcur;
+      }
+    }
   }
 }
 

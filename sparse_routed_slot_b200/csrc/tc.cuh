@@ -88,6 +88,15 @@ RSM_DEV void tma_load_4d(void* dst, const void* tmap, uint64_t* bar, int c0, int
       : "memory");
 }
 
+// Contiguous bulk copy global -> shared (bytes a multiple of 16, both addresses 16-byte aligned),
+// completion counted on an mbarrier of the issuing CTA.
+RSM_DEV void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
 // Tile store shared -> global (bulk async group of the issuing thread); out-of-range parts of the
 // box are not written.
 RSM_DEV void tma_store_4d(const void* tmap, const void* src, int c0, int c1, int c2, int c3) {

@@ -3,7 +3,10 @@
 Run a fixed case through the public API (on cuda:0, synthetic inputs):
 
     python -m sparse_routed_slot_b200.profile_case run [--workload long_ctx_bf16] [--forwards 2]
-                                                      [--decode-steps 2]
+                                                      [--decode-steps 2] [--tokens T]
+
+--tokens replaces the workload's sequence length (a smaller case of the same kernels, for captures
+that replay each launch many times).
 
 Each forward makes rsm_forward_kernel_launches() launches (routing records, segment summary,
 segment scan, chunk scan on the tensor path); the decode steps use decode_256x16. Capture with
@@ -44,7 +47,7 @@ def sources_digest() -> str:
     return h.hexdigest()
 
 
-def run_case(workload: str, forwards: int, decode_steps: int) -> None:
+def run_case(workload: str, forwards: int, decode_steps: int, tokens: int = 0) -> None:
     import torch
 
     import sparse_routed_slot_b200 as rsm
@@ -52,7 +55,8 @@ def run_case(workload: str, forwards: int, decode_steps: int) -> None:
 
     dev = torch.device("cuda", 0)
     w = WORKLOADS[workload]
-    x = make_inputs(w.B, w.T, w.H, w.M, w.Dv, w.torch_dtype, w.decay, seed=w.seed, device=dev)
+    T = tokens if tokens > 0 else w.T
+    x = make_inputs(w.B, T, w.H, w.M, w.Dv, w.torch_dtype, w.decay, seed=w.seed, device=dev)
     for _ in range(forwards):
         out = rsm.forward(x["q"], x["k"], x["v"], x["logits"], x["f"], w.K)
     torch.cuda.synchronize()
@@ -130,13 +134,14 @@ def main(argv=None) -> None:
     r.add_argument("--workload", default="long_ctx_bf16")
     r.add_argument("--forwards", type=int, default=2)
     r.add_argument("--decode-steps", type=int, default=2)
+    r.add_argument("--tokens", type=int, default=0)
     t = sub.add_parser("traffic")
     t.add_argument("csv")
     t.add_argument("--workload", default="long_ctx_bf16")
     t.add_argument("--out", default=os.path.join(ROOT, "profiles", "traffic.json"))
     a = ap.parse_args(argv)
     if a.cmd == "run":
-        run_case(a.workload, a.forwards, a.decode_steps)
+        run_case(a.workload, a.forwards, a.decode_steps, a.tokens)
         print("ok")
     else:
         d = summarize_traffic(a.csv, a.workload, a.out)
