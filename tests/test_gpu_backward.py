@@ -49,6 +49,25 @@ def test_backward_matches_oracle(rsm, M, K, Dv, T, dtype, decay):
     assert all(e <= TOL for e in errs.values()), errs
 
 
+@pytest.mark.parametrize("M,K,Dv,T", [(256, 32, 96, 21), (256, 256, 96, 9)])
+def test_backward_large_state_layouts(rsm, M, K, Dv, T):
+    """The largest states (M*Dv = 24576): the tape rows are read from global memory instead of
+    travelling through the 8-slot ring (K = 32), and a 2-slot ring (K = M = 256)."""
+    B, H = 1, 2
+    dev = torch.device("cuda")
+    x = make_inputs(B, T, H, M, Dv, torch.bfloat16, "slot", seed=M + K, device=dev, h0=True)
+    g = torch.Generator(device=dev).manual_seed(11)
+    dO = torch.randn(B, T, H, Dv, generator=g, device=dev)
+    dHT = torch.randn(B, H, M, Dv, generator=g, device=dev)
+    out = rsm.backward(x["q"], x["k"], x["v"], x["logits"], x["f"], K, dO, dHT, x["H0"])
+    torch.cuda.synchronize()
+    c = {n: t.float().cpu().numpy() for n, t in x.items()}
+    r = oracle.backward(c["q"], c["k"], c["v"], c["logits"], c["f"], K, dO=dO.cpu().numpy(),
+                        dHT=dHT.cpu().numpy(), H0=c["H0"])
+    errs = {n: rel(out[n].cpu().numpy(), r[n]) for n in ("dq", "dk", "dv", "dlogits", "df", "dH0")}
+    assert all(e <= TOL for e in errs.values()), errs
+
+
 def test_backward_without_output_gradient_and_zero_tokens(rsm):
     """dO = None (a loss on H_T only); and T = 0 (dH0 = dHT)."""
     B, T, H, M, K, Dv = 1, 50, 2, 64, 8, 64
