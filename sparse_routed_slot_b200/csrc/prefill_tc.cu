@@ -824,8 +824,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
 // tokens after it.
 //
 // The products run on bf16 operands (kind::f16): v as stored (its TMA tile, used MN-major), and Wr
-// split into a bf16 high part and a bf16 low part (two MMAs, about 16 significant bits together),
-// accumulated in fp32.
+// split into a bf16 high part and a bf16 low part (about 16 significant bits together). One MMA of
+// N = 256 per K step takes both parts as the two halves of its B operand, so v is read once: U^T
+// accumulates in fp32 as a high-part sum (TMEM columns 0..127) and a low-part sum (128..255),
+// added when U is read out.
 //
 // Warp roles (two CTAs per SM, each on one segment at a time, 9 warps):
 //   warps 0-7  row workers; warp w owns tokens 8w..8w+7 of the chunk, lane l slots 4l..4l+3 of
@@ -833,9 +835,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
 //              the last to the first (exclusive in-warp suffix sums in place), exchange the warp
 //              totals, write Wr (high and low tiles) at the selected entries; at the segment's end
 //              read U out of TMEM and write U and D.
-//   warp 8     MMA issuer (lane 0 issues): the v tile loads (one chunk ahead) and the 8 MMAs of
-//              each chunk, U^T += V^T Wr (M = value columns, N = slots, K = 16 tokens per step,
-//              high and low part).
+//   warp 8     MMA issuer (lane 0 issues): the v tile loads (one chunk ahead) and the 4 MMAs of
+//              each chunk, U^T += V^T [Wr_high | Wr_low] (M = value columns, N = 2 x 128 slots,
+//              K = 16 tokens per step).
 // One Wr tile pair: the row workers build a chunk's table and exponents while the MMAs of the
 // chunk before run, and write its Wr once they are done.
 constexpr int kSumThreads = (kRWarps + 1) * 32;
@@ -846,7 +848,7 @@ constexpr int kSumOffTot = kSumOffTab + 32768;       // per-warp lam sums [2][8]
 constexpr int kSumOffSuf = kSumOffTot + 2 * kRWarps * kM * 4;  // per-warp exponent offsets [8][128]
 constexpr int kSumSmemBytes = kSumOffSuf + kRWarps * kM * 4 + 1024;
 constexpr int kSumCtasPerSm = 2;
-constexpr int kSumTmemCols = 128;
+constexpr int kSumTmemCols = 256;
 static_assert(kSumCtasPerSm * (kSumSmemBytes + 1024) <= 233472, "two summary CTAs per SM");
 
 // The bf16 high and low tiles of Wr ([64 t][128 slot] each, MN-major, 16 KB apart): row t, slot i.
@@ -993,8 +995,9 @@ __global__ void __launch_bounds__(kSumThreads, kSumCtasPerSm) segment_summary_ke
       for (int r = kRowsPerWarp - 1; r >= 0; --r) {
         float4* row = reinterpret_cast<float4*>(tab + r * kM) + lane;
         const float4 x = *row;
-        *row = make_float4(x.x != 0.f ? run[0] : 0.f, x.y != 0.f ? run[1] : 0.f, x.z != 0.f ? run[2] : 0.f,
-                           x.w != 0.f ? run[3] : 0.f);
+        if (x.x != 0.f || x.y != 0.f || x.z != 0.f || x.w != 0.f)  // all-zero groups stay as they are
+          *row = make_float4(x.x != 0.f ? run[0] : 0.f, x.y != 0.f ? run[1] : 0.f, x.z != 0.f ? run[2] : 0.f,
+                             x.w != 0.f ? run[3] : 0.f);
         run[0] += x.x; run[1] += x.y; run[2] += x.z; run[3] += x.w;
       }
       reinterpret_cast<float4*>(sTot + (buf * kRWarps + w) * kM)[lane] = make_float4(run[0], run[1], run[2], run[3]);
@@ -1050,14 +1053,14 @@ __global__ void __launch_bounds__(kSumThreads, kSumCtasPerSm) segment_summary_ke
         float* dst = p.ws_state + slot_base * kM * kDV;
         const int dv = (w & 3) * 32 + lane;
         const int c0 = (w >> 2) * 64;
-        float u[2][32];
-        tc::tmem_ld32(tc::tmem_addr(tb, (uint32_t)((w & 3) * 32), (uint32_t)c0), u[0]);
-        tc::tmem_ld32(tc::tmem_addr(tb, (uint32_t)((w & 3) * 32), (uint32_t)(c0 + 32)), u[1]);
-        tc::tmem_wait_ld();
+#pragma unroll 1
+        for (int g = 0; g < 8; ++g) {
+          float u[8], ul[8];  // high-part and low-part sums of 8 slots
+          tc::tmem_ld8(tc::tmem_addr(tb, (uint32_t)((w & 3) * 32), (uint32_t)(c0 + 8 * g)), u);
+          tc::tmem_ld8(tc::tmem_addr(tb, (uint32_t)((w & 3) * 32), (uint32_t)(kM + c0 + 8 * g)), ul);
+          tc::tmem_wait_ld();
 #pragma unroll
-        for (int g = 0; g < 2; ++g) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) dst[(int64_t)(c0 + 32 * g + j) * kDV + dv] = u[g][j];
+          for (int j = 0; j < 8; ++j) dst[(int64_t)(c0 + 8 * g + j) * kDV + dv] = u[j] + ul[j];
         }
         if (w == 0) {
 #pragma unroll
@@ -1089,10 +1092,11 @@ __global__ void __launch_bounds__(kSumThreads, kSumCtasPerSm) segment_summary_ke
         ++n_tma;
       };
       load_v(wk, 0);
-      // v: 64-column halves 8 KB apart, groups of 8 token rows 1 KB apart; Wr: 64-slot halves 8 KB
-      // apart, the same row groups; a K step of 16 tokens advances both by 2 KB
+      // v: 64-column halves 8 KB apart, groups of 8 token rows 1 KB apart; [Wr_high | Wr_low]: four
+      // 64-slot blocks 8 KB apart (N = 256), the same row groups; a K step of 16 tokens advances both
+      // by 2 KB
       const uint64_t dV0 = tc::smem_desc(tc::smem_u32(sV), 8192, 1024), dWb = tc::smem_desc(tc::smem_u32(sWb), 8192, 1024);
-      constexpr uint32_t kIdC = tc::idesc_bf16(kDV, kM, 1, 1);
+      constexpr uint32_t kIdC = tc::idesc_bf16(kDV, 2 * kM, 1, 1);
       for (; wk.valid(items) && !*abort_flag; ++n, wk.next(p, items)) {
         const Chunk ck = wk.get(p);
         {
@@ -1110,11 +1114,9 @@ __global__ void __launch_bounds__(kSumThreads, kSumCtasPerSm) segment_summary_ke
         const uint64_t dVn = dV0 + (uint64_t)(((n & 1) * 16384) >> 4);
 #pragma unroll
         for (int j = 0; j < kC / 16; ++j)
-#pragma unroll
-          for (int part = 0; part < 2; ++part)
-            if (leader)
-              tc::mma_bf16_ss(tb, dVn + (uint64_t)((j * 2048) >> 4), dWb + (uint64_t)((part * 16384 + j * 2048) >> 4),
-                              kIdC, (ck.first && j == 0 && part == 0) ? 0u : 1u);
+          if (leader)
+            tc::mma_bf16_ss(tb, dVn + (uint64_t)((j * 2048) >> 4), dWb + (uint64_t)((j * 2048) >> 4), kIdC,
+                            (ck.first && j == 0) ? 0u : 1u);
         if (leader) tc::mma_commit(&bar_mma);
         if (ck.last) ++n_items;
       }
