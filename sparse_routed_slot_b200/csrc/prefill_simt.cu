@@ -201,34 +201,40 @@ __global__ void __launch_bounds__(kThreads) prefill_simt_kernel(rsm_forward_args
     }
     __syncthreads();
 
-    // --- outputs of the chunk for this column tile: thread (dd, g) computes the tokens
-    // t = g + G k, so that each state and value element it loads serves all of them
+    // --- outputs of the chunk for this column tile: thread (tp, cg) computes tokens 2tp, 2tp+1 x
+    // columns 4cg..4cg+3, so each state row piece and value row piece it loads (16 bytes) serves
+    // eight products
     {
-      constexpr int kMaxNT = kC * 64 / kThreads;  // tokens per thread at DT = 64
-      const int G = kThreads / DT, dd = tid % DT, g = tid / DT, NT = kC / G;  // NT = 1 or 2
-      float acc[kMaxNT];
-#pragma unroll
-      for (int k = 0; k < kMaxNT; ++k) acc[k] = 0.f;
+      const int ncg = DT / 4;
+      if (tid < (kC / 2) * ncg) {
+        const int tp = tid / ncg, cg = tid - tp * ncg;
+        const int t0 = 2 * tp;
+        float4 o0 = make_float4(0.f, 0.f, 0.f, 0.f), o1 = o0;
 #pragma unroll 4
-      for (int i = 0; i < M; ++i) {
-        const float hv = s_H[i * DT + dd];
-#pragma unroll
-        for (int k = 0; k < kMaxNT; ++k)
-          if (k < NT) acc[k] = fmaf(s_qh[(g + G * k) * M + i], hv, acc[k]);
-      }
-#pragma unroll 4
-      for (int s = 0; s < kC; ++s) {
-        const float vv = s_v[s * DT + dd];
-#pragma unroll
-        for (int k = 0; k < kMaxNT; ++k) {
-          const int t = g + G * k;
-          if (k < NT && s <= t) acc[k] = fmaf(s_A[t * kC + s], vv, acc[k]);
+        for (int i = 0; i < M; ++i) {
+          const float4 hv = *reinterpret_cast<const float4*>(s_H + i * DT + 4 * cg);
+          const float q0 = s_qh[t0 * M + i], q1 = s_qh[(t0 + 1) * M + i];
+          o0.x = fmaf(q0, hv.x, o0.x); o0.y = fmaf(q0, hv.y, o0.y); o0.z = fmaf(q0, hv.z, o0.z); o0.w = fmaf(q0, hv.w, o0.w);
+          o1.x = fmaf(q1, hv.x, o1.x); o1.y = fmaf(q1, hv.y, o1.y); o1.z = fmaf(q1, hv.z, o1.z); o1.w = fmaf(q1, hv.w, o1.w);
         }
-      }
-#pragma unroll
-      for (int k = 0; k < kMaxNT; ++k) {
-        const int t = g + G * k;
-        if (k < NT && t < nrows && dd < DTe) a.o[(((int64_t)b * T + c0 + t) * H + h) * Dv + d0 + dd] = acc[k];
+#pragma unroll 4
+        for (int s = 0; s <= t0; ++s) {
+          const float4 vv = *reinterpret_cast<const float4*>(s_v + s * DT + 4 * cg);
+          const float a0 = s_A[t0 * kC + s], a1 = s_A[(t0 + 1) * kC + s];
+          o0.x = fmaf(a0, vv.x, o0.x); o0.y = fmaf(a0, vv.y, o0.y); o0.z = fmaf(a0, vv.z, o0.z); o0.w = fmaf(a0, vv.w, o0.w);
+          o1.x = fmaf(a1, vv.x, o1.x); o1.y = fmaf(a1, vv.y, o1.y); o1.z = fmaf(a1, vv.z, o1.z); o1.w = fmaf(a1, vv.w, o1.w);
+        }
+        {  // s = t0 + 1 reaches token t0 + 1 only
+          const float4 vv = *reinterpret_cast<const float4*>(s_v + (t0 + 1) * DT + 4 * cg);
+          const float a1 = s_A[(t0 + 1) * kC + t0 + 1];
+          o1.x = fmaf(a1, vv.x, o1.x); o1.y = fmaf(a1, vv.y, o1.y); o1.z = fmaf(a1, vv.z, o1.z); o1.w = fmaf(a1, vv.w, o1.w);
+        }
+        // Dv and the tile start are multiples of 4, so a column group is wholly inside or outside
+        if (4 * cg < DTe) {
+          float* op = a.o + (((int64_t)b * T + c0 + t0) * H + h) * Dv + d0 + 4 * cg;
+          if (t0 < nrows) *reinterpret_cast<float4*>(op) = o0;
+          if (t0 + 1 < nrows) *reinterpret_cast<float4*>(op + (int64_t)H * Dv) = o1;
+        }
       }
     }
     // --- write weights carried to the chunk end (non-positive exponents)
@@ -239,28 +245,38 @@ __global__ void __launch_bounds__(kThreads) prefill_simt_kernel(rsm_forward_args
     }
     __syncthreads();
 
-    // --- state carry; slots not selected in this chunk are left untouched. Thread (dd, g)
-    // updates the slots i = g + G j, 8 at a time, so that each value element serves all of them
+    // --- state carry; slots not selected in this chunk are left untouched. Thread (ig, cg)
+    // updates slots 4ig..4ig+3 x columns 4cg..4cg+3: per token one 16-byte weight load and one
+    // 16-byte value load serve sixteen products
     {
-      const int G = kThreads / DT, dd = tid % DT, g = tid / DT, NI = M / G;  // NI = 2 .. 8
-      for (int j0 = 0; j0 < NI; j0 += 8) {
-        float acc[8];
+      const int ncg = DT / 4;
+      for (int p = tid; p < (M / 4) * ncg; p += kThreads) {
+        const int ig = p / ncg, cg = p - ig * ncg;
+        float4 acc[4];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int i = g + G * (j0 + j);
-          acc[j] = (j0 + j < NI) ? s_D[i] * s_H[i * DT + dd] : 0.f;
+        for (int j = 0; j < 4; ++j) {
+          const int i = 4 * ig + j;
+          const float4 hv = *reinterpret_cast<const float4*>(s_H + i * DT + 4 * cg);
+          const float d = s_D[i];
+          acc[j] = make_float4(d * hv.x, d * hv.y, d * hv.z, d * hv.w);
         }
 #pragma unroll 4
         for (int t = 0; t < kC; ++t) {
-          const float vv = s_v[t * DT + dd];
+          const float4 vv = *reinterpret_cast<const float4*>(s_v + t * DT + 4 * cg);
+          const float4 w4 = *reinterpret_cast<const float4*>(s_w + t * M + 4 * ig);
+          const float wj[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-            if (j0 + j < NI) acc[j] = fmaf(s_w[t * M + g + G * (j0 + j)], vv, acc[j]);
+          for (int j = 0; j < 4; ++j) {
+            acc[j].x = fmaf(wj[j], vv.x, acc[j].x);
+            acc[j].y = fmaf(wj[j], vv.y, acc[j].y);
+            acc[j].z = fmaf(wj[j], vv.z, acc[j].z);
+            acc[j].w = fmaf(wj[j], vv.w, acc[j].w);
+          }
         }
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int i = g + G * (j0 + j);
-          if (j0 + j < NI && s_touch[i]) s_H[i * DT + dd] = acc[j];
+        for (int j = 0; j < 4; ++j) {
+          const int i = 4 * ig + j;
+          if (s_touch[i]) *reinterpret_cast<float4*>(s_H + i * DT + 4 * cg) = acc[j];
         }
       }
     }
