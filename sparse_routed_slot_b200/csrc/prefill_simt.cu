@@ -98,16 +98,34 @@ __global__ void __launch_bounds__(kThreads) prefill_simt_kernel(rsm_forward_args
     for (int i = tid; i < M; i += kThreads) s_touch[i] = 0;
     __syncthreads();
 
-    // --- routing, log-decay and write weights of the chunk's rows (one warp per row)
+    // --- routing, log-decay and write weights of the chunk's rows (one warp per row). Every load
+    // of the chunk is issued before the ranking (this thread's value elements, and at M <= 128 the
+    // row's q and k beside its logits), so the chunk waits on one memory round trip, not three.
+    constexpr int kVRegs = kC * 64 / kThreads;  // value elements per thread at DT = 64
+    constexpr bool kEarlyQK = E <= 4;
+    float vr[kVRegs];
+#pragma unroll
+    for (int j = 0; j < kVRegs; ++j) {
+      const int p = tid + j * kThreads;
+      const int t = p / DT, dd = p % DT;
+      vr[j] = (p < kC * DT && t < nrows && dd < DTe)
+                  ? In<TIn>::ld(v + (((int64_t)b * T + c0 + t) * H + h) * Dv + d0 + dd)
+                  : 0.f;
+    }
     for (int t = warp; t < kC; t += kThreads / 32) {
       if (t < nrows) {
         const int64_t row = ((int64_t)b * T + c0 + t) * H + h;
         float x[E];
         load_row_logits<M>(a.logits + row * M, lane, x);
-        float fv[E];
+        float fv[E], qv[E], kv[E];
 #pragma unroll
-        for (int e = 0; e < E; ++e)
+        for (int e = 0; e < E; ++e) {
           fv[e] = (a.decay == RSM_DECAY_SLOT) ? a.f[row * M + lane * E + e] : a.f[row];
+          if (kEarlyQK) {
+            qv[e] = In<TIn>::ld(q + row * M + lane * E + e);
+            kv[e] = In<TIn>::ld(k + row * M + lane * E + e);
+          }
+        }
         if (validate) {
           bool bad = false;
 #pragma unroll
@@ -129,12 +147,12 @@ __global__ void __launch_bounds__(kThreads) prefill_simt_kernel(rsm_forward_args
 #pragma unroll
         for (int e = 0; e < E; ++e) {
           const int i = lane * E + e;
-          s_q[t * M + i] = In<TIn>::ld(q + row * M + i);
+          s_q[t * M + i] = kEarlyQK ? qv[e] : In<TIn>::ld(q + row * M + i);
           if (sel & (1u << e)) {
             if (so) so[rank[e]] = sc[e];
             const float lam = sc[e] * fv[e];
             s_g[t * M + i] = lam;
-            s_w[t * M + i] = In<TIn>::ld(k + row * M + i) * (-expm1f(lam));
+            s_w[t * M + i] = (kEarlyQK ? kv[e] : In<TIn>::ld(k + row * M + i)) * (-expm1f(lam));
             s_touch[i] = 1;
           } else {
             s_g[t * M + i] = 0.f;
@@ -151,15 +169,15 @@ __global__ void __launch_bounds__(kThreads) prefill_simt_kernel(rsm_forward_args
         }
       }
     }
-    for (int p = tid; p < kC * DT; p += kThreads) {
-      const int t = p / DT, dd = p % DT;
-      s_v[p] = (t < nrows && dd < DTe)
-                   ? In<TIn>::ld(v + (((int64_t)b * T + c0 + t) * H + h) * Dv + d0 + dd)
-                   : 0.f;
+#pragma unroll
+    for (int j = 0; j < kVRegs; ++j) {
+      const int p = tid + j * kThreads;
+      if (p < kC * DT) s_v[p] = vr[j];
     }
     __syncthreads();
 
     // --- cumulative log-decay per slot (a prefix sum down the chunk), chunk decay
+    bool strong = false;  // some slot decays by more than e^-80 in the chunk
     for (int i = tid; i < M; i += kThreads) {
       float g = 0.f;
       for (int t = 0; t < kC; ++t) {
@@ -168,10 +186,28 @@ __global__ void __launch_bounds__(kThreads) prefill_simt_kernel(rsm_forward_args
       }
       s_gC[i] = g;
       s_D[i] = expf(g);
+      strong |= g < -80.f;
     }
-    __syncthreads();
+    // A from start-referenced factors (below) unless a slot decays too strongly for e^{-g} to stay
+    // finite; the entry table takes the raw q's memory, so K <= M/2
+    const bool factored = !__syncthreads_or(strong) && 2 * K <= M;
     // --- q scaled to the chunk start, every element in parallel
     for (int p = tid; p < kC * M; p += kThreads) s_qh[p] = s_q[p] * expf(s_g[p]);
+    float2* s_ent = reinterpret_cast<float2*>(s_q);  // [K][kC]: (slot, w e^{-g}) of entry r of token s
+    if (factored) {
+      __syncthreads();  // the raw q is consumed
+      for (int p = tid; p < kC * K; p += kThreads) {
+        const int r = p / kC, s = p - r * kC;
+        int j = 0;
+        float wh = 0.f;
+        if (s < nrows) {
+          j = s_sidx[s * M + r];
+          wh = s_w[s * M + j] * expf(-s_g[s * M + j]);
+        }
+        s_ent[p] = make_float2(__int_as_float(j), wh);
+      }
+      __syncthreads();
+    }
 
     // --- intra-chunk weights A[t][s], s <= t (sparse over the K slots written at s); each
     // thread carries its kC*kC/kThreads pairs together so that their exponentials overlap
@@ -186,13 +222,27 @@ __global__ void __launch_bounds__(kThreads) prefill_simt_kernel(rsm_forward_args
         ss[k] = p % kC;
         acc[k] = 0.f;
       }
-      for (int r = 0; r < K; ++r) {
+      if (factored) {
+        // A[t][s] = sum_r (q_{t,j} e^{g_{t,j}}) (w_{s,j} e^{-g_{s,j}}), j = slot of entry r of s
+        for (int r = 0; r < K; ++r) {
 #pragma unroll
-        for (int k = 0; k < kPairs; ++k) {
-          const int t = tt[k], s = ss[k];
-          if (s <= t && t < nrows) {
-            const int j = s_sidx[s * M + r];
-            acc[k] = fmaf(s_q[t * M + j] * s_w[s * M + j], expf(s_g[t * M + j] - s_g[s * M + j]), acc[k]);
+          for (int k = 0; k < kPairs; ++k) {
+            const int t = tt[k], s = ss[k];
+            if (s <= t && t < nrows) {
+              const float2 e = s_ent[r * kC + s];
+              acc[k] = fmaf(s_qh[t * M + __float_as_int(e.x)], e.y, acc[k]);
+            }
+          }
+        }
+      } else {
+        for (int r = 0; r < K; ++r) {
+#pragma unroll
+          for (int k = 0; k < kPairs; ++k) {
+            const int t = tt[k], s = ss[k];
+            if (s <= t && t < nrows) {
+              const int j = s_sidx[s * M + r];
+              acc[k] = fmaf(s_q[t * M + j] * s_w[s * M + j], expf(s_g[t * M + j] - s_g[s * M + j]), acc[k]);
+            }
           }
         }
       }
