@@ -184,6 +184,48 @@ def replica_seed(base: int, rank: int) -> int:
 
 # --------------------------------------------------------------------------- CPU oracle timing
 
+def pipelined_e2e(nsteps: int, warmup: int, h2d, compute, d2h, nsets: int = 2) -> float:
+    """Mean ms per end-to-end step, device-timed, over `nsteps` steps run as a serving loop would:
+    `nsets` device buffer sets and three streams, so the copies in of step i+1 and the read-back of
+    step i overlap the computation. Every step still copies its own inputs in and its own result
+    out inside the timed region. h2d(i, s), compute(i, s) and d2h(i, s) enqueue step i's work for
+    buffer set s on the current stream."""
+    import torch
+    s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(nsets)]
+    ev_comp = [torch.cuda.Event() for _ in range(nsets)]
+    ev_out = [torch.cuda.Event() for _ in range(nsets)]
+
+    def run(n, e0=None, e1=None):
+        if e0 is not None:
+            e0.record(s_in)
+        for i in range(n):
+            st = i % nsets
+            with torch.cuda.stream(s_in):
+                if i >= nsets:
+                    s_in.wait_event(ev_comp[st])  # step i - nsets has consumed this set's inputs
+                h2d(i, st)
+                ev_in[st].record(s_in)
+            with torch.cuda.stream(s_comp):
+                s_comp.wait_event(ev_in[st])
+                if i >= nsets:
+                    s_comp.wait_event(ev_out[st])  # step i - nsets's result has been read back
+                compute(i, st)
+                ev_comp[st].record(s_comp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_comp[st])
+                d2h(i, st)
+                ev_out[st].record(s_out)
+        if e1 is not None:
+            e1.record(s_out)  # after the last read-back, which follows every earlier step's work
+        torch.cuda.synchronize()
+
+    run(max(1, warmup))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    run(nsteps, e0, e1)
+    return e0.elapsed_time(e1) / nsteps
+
+
 def oracle_sample(w, seconds_target: float = 3.0) -> dict:
     """Times the fp64 CPU oracle (as it stands) on a bounded sample of the workload: all heads of
     sequence 0, over a prefix of the tokens or, when the whole sequence is quick, repeated runs of
@@ -397,33 +439,34 @@ def run_ours(args, world, rank, local):
     tokens = w.B * w.T
     value, ms_max = job_throughput(tokens, ms, world)
 
-    # end to end through the public call with host buffers: pinned inputs copied in, result out
+    # end to end through the public call with host buffers: every step copies its pinned inputs
+    # in and reads o and H_T back, pipelined over two buffer sets (pipelined_e2e)
+    import sparse_routed_slot_b200 as rsm
     host_in = {n: t.cpu().pin_memory() for n, t in case.x.items()}
-    dev_in = {n: torch.empty_like(t) for n, t in case.x.items()}
-    host_o = torch.empty(case.o.shape, dtype=case.o.dtype).pin_memory()
-    host_HT = torch.empty(case.HT.shape, dtype=case.HT.dtype).pin_memory()
+    dev_in = [{n: torch.empty_like(t) for n, t in case.x.items()} for _ in range(2)]
+    dev_out = [{"o": torch.empty_like(case.o), "HT": torch.empty_like(case.HT)} for _ in range(2)]
+    wss = [torch.empty_like(case.ws) for _ in range(2)]
+    host_out = [{"o": torch.empty(case.o.shape, dtype=case.o.dtype).pin_memory(),
+                 "HT": torch.empty(case.HT.shape, dtype=case.HT.dtype).pin_memory()} for _ in range(2)]
     h2d = sum(t.numel() * t.element_size() for t in host_in.values())
-    d2h = host_o.numel() * 4 + host_HT.numel() * 4
+    d2h = case.o.numel() * 4 + case.HT.numel() * 4
 
-    def e2e_step():
-        for n in dev_in:
-            dev_in[n].copy_(host_in[n], non_blocking=True)
-        case.step(dev_in)
-        host_o.copy_(case.o, non_blocking=True)
-        host_HT.copy_(case.HT, non_blocking=True)
+    def e2e_in(i, s):
+        for n in host_in:
+            dev_in[s][n].copy_(host_in[n], non_blocking=True)
 
-    for _ in range(max(1, args.warmup)):
-        e2e_step()
-    torch.cuda.synchronize()
+    def e2e_compute(i, s):
+        x = dev_in[s]
+        rsm.forward(x["q"], x["k"], x["v"], x["logits"], x["f"], w.K, out=dev_out[s], workspace=wss[s],
+                    path=case.path)
+
+    def e2e_out(i, s):
+        for n in ("o", "HT"):
+            host_out[s][n].copy_(dev_out[s][n], non_blocking=True)
+
     barrier(world)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
-    del host_in, dev_in
+    e2e_ms = max_over_ranks(pipelined_e2e(args.steps, args.warmup, e2e_in, e2e_compute, e2e_out), world)
+    del host_in, dev_in, dev_out, wss, host_out
 
     roof = case.roofline(ms, peaks, f"{w.name}/forward")
     roof["kernel"] = f"rsm_forward, all {case.launches} launches of the step (" + ", ".join(names) + ")"
@@ -435,8 +478,9 @@ def run_ours(args, world, rank, local):
         "roofline": roof,
         "kernels": [{"name": n, "ms": t, "share": t / sum(kms) if sum(kms) > 0 else None}
                     for n, t in zip(names, kms)],
-        "e2e": {"value": tokens * world / (e2e_ms * 1e-3), "unit": "tokens/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "e2e": {"value": tokens * world / (e2e_ms * 1e-3), "unit": "tokens/s", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "pipelining": "two buffer sets, three streams: step i+1's copies in overlap step i"},
         "gpu_launches": 2 * args.steps * case.launches,  # device-timed steps and end-to-end steps
         "clocks": clk,
     }
@@ -595,26 +639,24 @@ def run_decode(args, world, rank, local, peaks) -> dict:
     # carried state stays on the device (it is the recurrence's own memory)
     e2e_steps = min(nsteps, 256)
     host_in = {n: t[:e2e_steps].cpu().pin_memory() for n, t in d.items()}
-    dev_in = {n: torch.empty_like(t[0]) for n, t in d.items()}
-    host_o = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    dev_in = [{n: torch.empty_like(t[0]) for n, t in d.items()} for _ in range(2)]
+    dev_o = [torch.empty_like(o) for _ in range(2)]
+    host_o = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for _ in range(2)]
     h2d = sum(t[0].numel() * t.element_size() for t in host_in.values())
 
-    def e2e_step(i):
-        for n in dev_in:
-            dev_in[n].copy_(host_in[n][i], non_blocking=True)
-        rsm.decode_step(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["logits"], dev_in["f"], w.K, state, o=o)
-        host_o.copy_(o, non_blocking=True)
+    def e2e_in(i, s):
+        for n in host_in:
+            dev_in[s][n].copy_(host_in[n][i % e2e_steps], non_blocking=True)
 
-    for i in range(3):
-        e2e_step(i)
-    torch.cuda.synchronize()
+    def e2e_compute(i, s):  # the steps stay in order on one stream: the state carries between them
+        x = dev_in[s]
+        rsm.decode_step(x["q"], x["k"], x["v"], x["logits"], x["f"], w.K, state, o=dev_o[s])
+
+    def e2e_out(i, s):
+        host_o[s].copy_(dev_o[s], non_blocking=True)
+
     barrier(world)
-    e0.record(stream)
-    for i in range(e2e_steps):
-        e2e_step(i)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
+    e2e_ms = max_over_ranks(pipelined_e2e(e2e_steps, 3, e2e_in, e2e_compute, e2e_out), world)
     cpu_steps = {n: t[:8].float().cpu().numpy() for n, t in d.items()} if state0 is not None else None
     del host_in, dev_in, d
 
@@ -628,7 +670,8 @@ def run_decode(args, world, rank, local, peaks) -> dict:
                         "peak_source": peaks["source"] + " (burst copy)"},
            "e2e": {"value": sb * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s (state, all GPUs)",
                    "ms_per_step": e2e_ms, "steps": e2e_steps,
-                   "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": host_o.numel() * 4},
+                   "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": o.numel() * 4,
+                   "pipelining": "two buffer sets, three streams: step i+1's copies in overlap step i"},
            "clocks": clk, "launches_timed": nsteps + e2e_steps,
            "config": {"workload": w.name, "B": w.B, "H": w.H, "M": w.M, "K": w.K, "Dv": w.Dv,
                       "decay": w.decay, "qkv_dtype": w.dtype, "prefill_T": w.decode_prefill_T,
