@@ -283,6 +283,22 @@ def _sources_digest() -> str:
     return sources_digest()
 
 
+def stored_tensor_pipe(kernel_prefix: str):
+    """Tensor-pipe activity (% of elapsed cycles) of the first stored kernel whose name contains
+    `kernel_prefix` (profiles/traffic.json, ncu section capture), or None when missing or stale."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        d = json.load(open(p))
+    except (OSError, ValueError):
+        return None
+    if d.get("sources_sha256") != _sources_digest():
+        return None
+    for name, m in d.get("per_kernel", {}).items():
+        if kernel_prefix in name and "tensor_pipe_pct" in m:
+            return m["tensor_pipe_pct"]
+    return None
+
+
 def stored_traffic(key: str):
     """DRAM bytes per call measured by ncu for `key` (profiles/traffic.json), or None when the file
     is missing or was recorded for other kernel sources."""
@@ -409,7 +425,9 @@ class PrefillCase:
                 "algorithmic_bytes": self.nbytes, "o_fp32_extra_bytes": o_fp32_extra_bytes(w),
                 "frac_with_o_fp32": (self.nbytes + o_fp32_extra_bytes(w)) / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                 "peak_source": peaks["source"] + " (burst copy)",
-                "tensor_tflops": prefill_flops(w) / (ms * 1e-3) / 1e12}
+                "tensor_tflops": prefill_flops(w) / (ms * 1e-3) / 1e12,
+                "chunk_scan_tensor_pipe_pct": stored_tensor_pipe("prefill_tc_kernel")
+                if self.path_used == "tensor" else None}
 
 
 def config_of(w, case, world, extra=None):

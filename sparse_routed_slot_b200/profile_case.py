@@ -9,18 +9,28 @@ Run a fixed case through the public API (on cuda:0, synthetic inputs):
 that replay each launch many times).
 
 Each forward makes rsm_forward_kernel_launches() launches (routing records, segment summary,
-segment scan, chunk scan on the tensor path); the decode steps use decode_256x16. Capture with
+segment scan, chunk scan on the tensor path); the decode steps use decode_256x16. These three
+metrics take one pass (check on one launch of a --tokens case first: ncu prints "- 1 pass"), so
+the full-size case can be captured, limited to the launches that are read (the second forward and
+the two decode steps):
 
     ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum \\
-        --clock-control none --csv --log-file traffic.csv \\
-        python -m sparse_routed_slot_b200.profile_case run
+        --clock-control none -k regex:"route_rec|segment_summary|segment_scan|prefill_tc|decode_kernel" \\
+        -s 4 -c 6 --csv --log-file traffic.csv python -m sparse_routed_slot_b200.profile_case run
 
 then write the per-call DRAM bytes of the LAST forward and the LAST decode step, keyed to the
 current CUDA sources, to profiles/traffic.json:
 
     python -m sparse_routed_slot_b200.profile_case traffic traffic.csv
 
-bench.py reads that file and reports its bytes only while the sources still hash the same.
+Section captures of one kernel each on a smaller case (--tokens) add the tensor-pipe activity:
+
+    ncu --section SpeedOfLight ... --clock-control none -k regex:prefill_tc_kernel -s 1 -c 1 \
+        -o prof_tc python -m sparse_routed_slot_b200.profile_case run --tokens 8192 --decode-steps 0
+    ncu -i prof_tc.ncu-rep --page raw --csv > prof_tc.csv
+    python -m sparse_routed_slot_b200.profile_case pipes prof_tc.csv [more.csv ...]
+
+bench.py reads that file and reports its figures only while the sources still hash the same.
 """
 
 from __future__ import annotations
@@ -127,6 +137,51 @@ def summarize_traffic(csv_path: str, workload: str, out_path: str) -> dict:
     return d
 
 
+PIPE_METRIC = "sm__pipe_tensor_cycles_active.avg.pct_of_peak_sustained_elapsed"
+
+
+def read_ncu_raw_csv(path: str):
+    """[(kernel name, {metric: value})] from `ncu -i report --page raw --csv` (one row per launch,
+    one column per metric, a units row under the header)."""
+    rows = list(csv.reader(open(path)))
+    hi = next(i for i, r in enumerate(rows) if "Kernel Name" in r)
+    h = rows[hi]
+    ki = h.index("Kernel Name")
+    out = []
+    for r in rows[hi + 2:]:
+        if len(r) != len(h):
+            continue
+        m = {}
+        for name, val in zip(h, r):
+            try:
+                m[name] = float(val.replace(",", ""))
+            except ValueError:
+                pass
+        out.append((r[ki].split("(")[0].strip(), m))
+    return out
+
+
+def merge_pipes(csv_paths, out_path: str) -> dict:
+    """Adds each captured kernel's tensor-pipe activity (percent of elapsed cycles) to the traffic
+    file, under per_kernel[name]["tensor_pipe_pct"], with the case it was measured on."""
+    d = json.load(open(out_path))
+    if d.get("sources_sha256") != sources_digest():
+        raise SystemExit("the traffic file was recorded for other kernel sources; capture it again first")
+    for p in csv_paths:
+        for name, m in read_ncu_raw_csv(p):
+            if PIPE_METRIC not in m:
+                continue
+            base = name.split("::")[-1]  # e.g. prefill_tc_kernel<16>
+            key = next((k for k in d["per_kernel"] if k.split("(")[0].strip().endswith(base)), name)
+            d["per_kernel"].setdefault(key, {})["tensor_pipe_pct"] = m[PIPE_METRIC]
+    d["tensor_pipe_how"] = ("ncu section capture of one kernel per command (-k <kernel> -s 1 -c 1) on "
+                            "profile_case run --tokens 8192")
+    with open(out_path, "w") as fh:
+        json.dump(d, fh, indent=1)
+        fh.write("\n")
+    return d
+
+
 def main(argv=None) -> None:
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     sub = ap.add_subparsers(dest="cmd", required=True)
@@ -139,10 +194,16 @@ def main(argv=None) -> None:
     t.add_argument("csv")
     t.add_argument("--workload", default="long_ctx_bf16")
     t.add_argument("--out", default=os.path.join(ROOT, "profiles", "traffic.json"))
+    pp = sub.add_parser("pipes")
+    pp.add_argument("csv", nargs="+")
+    pp.add_argument("--out", default=os.path.join(ROOT, "profiles", "traffic.json"))
     a = ap.parse_args(argv)
     if a.cmd == "run":
         run_case(a.workload, a.forwards, a.decode_steps, a.tokens)
         print("ok")
+    elif a.cmd == "pipes":
+        d = merge_pipes(a.csv, a.out)
+        print(json.dumps({k: v.get("tensor_pipe_pct") for k, v in d["per_kernel"].items()}))
     else:
         d = summarize_traffic(a.csv, a.workload, a.out)
         print(json.dumps(d["bytes"]))
