@@ -93,6 +93,7 @@ __global__ void __launch_bounds__(kThreads) prefill_simt_kernel(rsm_forward_args
     s_H[p] = (dd < DTe && a.H0) ? a.H0[((int64_t)pair * M + i) * Dv + d0 + dd] : 0.f;
   }
 
+  float guess = __int_as_float(0x7fc00000);  // the warp's last threshold (none yet)
   for (int c0 = 0; c0 < T; c0 += kC) {
     const int nrows = min(kC, T - c0);
     for (int i = tid; i < M; i += kThreads) s_touch[i] = 0;
@@ -103,6 +104,7 @@ __global__ void __launch_bounds__(kThreads) prefill_simt_kernel(rsm_forward_args
     // row's q and k beside its logits), so the chunk waits on one memory round trip, not three.
     constexpr int kVRegs = kC * 64 / kThreads;  // value elements per thread at DT = 64
     constexpr bool kEarlyQK = E <= 4;
+    constexpr bool kSetSelect = E <= 4;  // at M = 256 its registers would spill
     float vr[kVRegs];
 #pragma unroll
     for (int j = 0; j < kVRegs; ++j) {
@@ -136,12 +138,39 @@ __global__ void __launch_bounds__(kThreads) prefill_simt_kernel(rsm_forward_args
         float* so = (route_owner && a.score_out) ? a.score_out + row * K : nullptr;
         int32_t* cnt = (route_owner && a.slot_counts) ? a.slot_counts + (int64_t)pair * M : nullptr;
         int rank[E];
-        const uint32_t sel = warp_topk<M>(x, K, lane, [&](int r, int slot, int e) {
-          s_sidx[t * M + r] = (unsigned char)slot;
-          if (io) io[r] = slot;
-          if (cnt) atomicAdd(cnt + slot, 1);
-          set_rank<E>(rank, e, r);
-        });
+        uint32_t sel = 0u;
+        // Without ranked outputs the entries' order is free: the exact TopK set from a threshold
+        // search seeded with the warp's previous row, listed in slot order; the ranking tournament
+        // when outputs want rank order, or when the search meets a tie at the cut
+        bool listed = false;
+        if (kSetSelect && !io && !so && K >= 2 && K < M && warp_select_guess<M>(x, K, guess, sel)) {
+          const int n = __popc(sel);
+          int before = n;  // inclusive scan of the lanes' counts
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(kFull, before, o);
+            if (lane >= o) before += y;
+          }
+          int r = before - n;
+#pragma unroll
+          for (int e = 0; e < E; ++e) {
+            if (sel & (1u << e)) {
+              const int slot = lane * E + e;
+              s_sidx[t * M + r] = (unsigned char)slot;
+              if (cnt) atomicAdd(cnt + slot, 1);
+              set_rank<E>(rank, e, r);
+              ++r;
+            }
+          }
+          listed = true;
+        }
+        if (!listed)
+          sel = warp_topk<M>(x, K, lane, [&](int r, int slot, int e) {
+            s_sidx[t * M + r] = (unsigned char)slot;
+            if (io) io[r] = slot;
+            if (cnt) atomicAdd(cnt + slot, 1);
+            set_rank<E>(rank, e, r);
+          });
         float sc[E];
         warp_router_scores<E>(x, sel, a.router, sc);
 #pragma unroll

@@ -846,7 +846,8 @@ constexpr int kSumOffWb = kSumOffV + 2 * 16384;      // Wr high, low [2][64 t][1
 constexpr int kSumOffTab = kSumOffWb + 32768;        // lam table [64 t][128 slot], then exponents
 constexpr int kSumOffTot = kSumOffTab + 32768;       // per-warp lam sums [2][8][128]
 constexpr int kSumOffSuf = kSumOffTot + 2 * kRWarps * kM * 4;  // per-warp exponent offsets [8][128]
-constexpr int kSumSmemBytes = kSumOffSuf + kRWarps * kM * 4 + 1024;
+constexpr int kSumOffLam = kSumOffSuf + kRWarps * kM * 4;       // Lam of the piece past this chunk [128]
+constexpr int kSumSmemBytes = kSumOffLam + kM * 4 + 1024;
 constexpr int kSumCtasPerSm = 2;
 constexpr int kSumTmemCols = 256;
 static_assert(kSumCtasPerSm * (kSumSmemBytes + 1024) <= 233472, "two summary CTAs per SM");
@@ -916,6 +917,7 @@ __global__ void __launch_bounds__(kSumThreads, kSumCtasPerSm) segment_summary_ke
   float* sTab = reinterpret_cast<float*>(sm + kSumOffTab);
   float* sTot = reinterpret_cast<float*>(sm + kSumOffTot);
   float* sSuf = reinterpret_cast<float*>(sm + kSumOffSuf);
+  float* sLam = reinterpret_cast<float*>(sm + kSumOffLam);
 
   // mbarriers (phase k of a barrier = its k-th completion)
   __shared__ __align__(8) uint64_t bar_rdy,  // Wr of chunk n written                  (row threads)
@@ -955,7 +957,6 @@ __global__ void __launch_bounds__(kSumThreads, kSumCtasPerSm) segment_summary_ke
     // =========================================================================== row workers
     const int w = warp;
     float* tab = sTab + w * kRowsPerWarp * kM;  // this warp's rows of the table
-    float lamS[4] = {0.f, 0.f, 0.f, 0.f};      // Lam of the item's tokens after this chunk (slots 4l..)
     // The table rows and the warp's token rows of the Wr tiles start at zero; afterwards each
     // entry's owner clears what it wrote (sparse), so no chunk fills them densely.
     uint32_t es1[RowInputs<KP>::kGroups];  // entry slots of the chunk before
@@ -977,7 +978,6 @@ __global__ void __launch_bounds__(kSumThreads, kSumCtasPerSm) segment_summary_ke
       const Chunk ck = wk.get(p);
       const int buf = n & 1;
       const int nrows_w = ck.nrows - w * kRowsPerWarp;
-      if (ck.first) lamS[0] = lamS[1] = lamS[2] = lamS[3] = 0.f;
       // the next chunk's records start loading (they have this whole chunk to arrive)
       RowInputs<KP> nxt;
       {
@@ -1002,22 +1002,23 @@ __global__ void __launch_bounds__(kSumThreads, kSumCtasPerSm) segment_summary_ke
       }
       reinterpret_cast<float4*>(sTot + (buf * kRWarps + w) * kM)[lane] = make_float4(run[0], run[1], run[2], run[3]);
       if (bar_rows_or(*abort_flag != 0)) break;  // every row worker takes the same decision
-      // ---- exponent offset of the warp's rows (lam of the later warps' rows and later chunks), and
-      // Lam past the next chunk (every row warp sums in the same order, so all hold the same value)
-      float suf[4] = {lamS[0], lamS[1], lamS[2], lamS[3]}, tot[4] = {0.f, 0.f, 0.f, 0.f};
+      // ---- exponent offsets, one slot per thread (row-worker thread j < M owns slot j): for every
+      // warp, the lam of the later warps' rows and of the piece's later chunks; then Lam past this
+      // chunk, and at the piece's end D = e^Lam
+      {
+        const int j = w * 32 + lane;
+        if (j < kM) {
+          float acc = ck.first ? 0.f : sLam[j];
 #pragma unroll
-      for (int w2 = 0; w2 < kRWarps; ++w2) {
-        const float4 t4 = reinterpret_cast<const float4*>(sTot + (buf * kRWarps + w2) * kM)[lane];
-        const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          if (w2 > w) suf[e] += tv[e];
-          tot[e] += tv[e];
+          for (int w2 = kRWarps - 1; w2 >= 0; --w2) {
+            sSuf[w2 * kM + j] = acc;
+            acc += sTot[(buf * kRWarps + w2) * kM + j];
+          }
+          sLam[j] = acc;
+          if (ck.last) p.ws_D[((int64_t)ck.pair * p.nslot + ck.seg + 1) * kM + j] = expf(acc);
         }
       }
-#pragma unroll
-      for (int e = 0; e < 4; ++e) lamS[e] += tot[e];
-      reinterpret_cast<float4*>(sSuf + w * kM)[lane] = make_float4(suf[0], suf[1], suf[2], suf[3]);
+      bar_rows();
       // ---- the Wr tiles are free once the MMAs of the chunk before are done; that chunk's entries
       // leave them (rows past a chunk's end hold slot 0, which clears a zero)
       if (n >= 1) wait_or_abort(&bar_mma, (n - 1) & 1, abort_flag);
@@ -1061,10 +1062,6 @@ __global__ void __launch_bounds__(kSumThreads, kSumCtasPerSm) segment_summary_ke
           tc::tmem_wait_ld();
 #pragma unroll
           for (int j = 0; j < 8; ++j) dst[(int64_t)(c0 + 8 * g + j) * kDV + dv] = u[j] + ul[j];
-        }
-        if (w == 0) {
-#pragma unroll
-          for (int e = 0; e < 4; ++e) p.ws_D[slot_base * kM + lane * 4 + e] = expf(lamS[e]);
         }
         tc::tmem_fence_before();
         mbar_arrive(&bar_out);
