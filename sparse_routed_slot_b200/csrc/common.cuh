@@ -160,75 +160,16 @@ RSM_DEV uint32_t warp_topk(const float (&x)[M / 32], int K, int lane, Emit emit)
   return sel;
 }
 
-// Selection of the TopK set only (no ranks), for K <= 32: finds a threshold key tau with exactly
-// K keys >= tau. Then the set {key >= tau} is the TopK set under (logit desc, index asc): every
-// member is strictly larger than every non-member, so no tie straddles the cut. The threshold is
-// bracketed on the order-preserving keys (lo: the smallest lane maximum, at least 32 keys >= it;
-// hi: the row maximum) and the bracket shrinks by interpolation alternating with bisection.
-// Returns false, without a result, when no such threshold exists (a tie at the cut) or the
-// bracket closes without one (near-ties); the caller then falls back to warp_topk.
-template <int M>
-RSM_DEV bool warp_select_set(const float (&x)[M / 32], int K, uint32_t& sel) {
-  constexpr int E = M / 32;
-  uint32_t key[E];
-  uint32_t kmax = 0u;
-#pragma unroll
-  for (int e = 0; e < E; ++e) {
-    key[e] = order_key(x[e]);
-    kmax = max(kmax, key[e]);
-  }
-  auto count_ge = [&](uint32_t t) {
-    int c = 0;
-#pragma unroll
-    for (int e = 0; e < E; ++e) c += key[e] >= t ? 1 : 0;
-    return (int)__reduce_add_sync(kFull, (unsigned)c);
-  };
-  uint32_t hi = __reduce_max_sync(kFull, kmax);
-  int chi = count_ge(hi);
-  uint32_t tau = hi;
-  bool found = chi == K;
-  if (!found) {
-    if (chi > K) return false;                   // tie at the maximum
-    uint32_t lo = __reduce_min_sync(kFull, kmax);
-    int clo = count_ge(lo);                        // >= 32 >= K
-    found = clo == K;
-    tau = lo;
-    for (int it = 0; it < 40 && !found; ++it) {
-      if (hi - lo <= 1u) return false;             // adjacent keys: no threshold in between
-      uint32_t t;
-      if (it & 1) {
-        t = lo + (hi - lo) / 2u;
-      } else {
-        const float frac = (float)(clo - K) / (float)(clo - chi);
-        t = lo + (uint32_t)((float)(hi - lo) * frac);
-        if (t <= lo || t >= hi) t = lo + (hi - lo) / 2u;
-      }
-      const int c = count_ge(t);
-      if (c == K) {
-        found = true;
-        tau = t;
-      } else if (c > K) {
-        lo = t;
-        clo = c;
-      } else {
-        hi = t;
-        chi = c;
-      }
-    }
-    if (!found) return false;
-  }
-  sel = 0u;
-#pragma unroll
-  for (int e = 0; e < E; ++e) sel |= (key[e] >= tau ? 1u : 0u) << e;
-  return true;
-}
-
-// Same contract as warp_select_set (exact TopK set or false), searching in the value domain from
-// a guess of the threshold (for example the previous row's): rows of one stream share a logit
-// distribution, so the first counts usually bracket the cut tightly and a few interpolation steps
-// on the empirical distribution land between the K-th and (K+1)-th values. The bracket always
-// stays valid: lo with more than K values >= lo, hi with fewer than K values >= hi (the row max
-// and min start it). `guess` is replaced by the threshold found. Needs 2 <= K < M.
+// Selection of the TopK set only (no ranks): finds a threshold t with exactly K values >= t. Every
+// member of {x >= t} is then strictly larger than every non-member, so it is the TopK set under any
+// tie-breaking. The search runs in the value domain from a guess (for example the previous row's
+// threshold): rows of one stream share a logit distribution, so the first counts usually bracket
+// the cut tightly and a few interpolation steps on the empirical distribution land between the
+// K-th and (K+1)-th values. The bracket always stays valid: lo with more than K values >= lo, hi
+// with fewer than K values >= hi (the row max and min start it). `guess` is replaced by the
+// threshold found. Returns false, without a result, when no such threshold exists (a tie at the
+// cut) or the bracket closes without one (near-ties); the caller then uses warp_topk. Needs
+// 2 <= K < M.
 template <int M>
 RSM_DEV bool warp_select_guess(const float (&x)[M / 32], int K, float& guess, uint32_t& sel) {
   constexpr int E = M / 32;
@@ -284,82 +225,6 @@ RSM_DEV bool warp_select_guess(const float (&x)[M / 32], int K, float& guess, ui
 #pragma unroll
   for (int e = 0; e < E; ++e) sel |= (x[e] >= t ? 1u : 0u) << e;
   return true;
-}
-
-// warp_select_guess for NR rows at once (x[r] is row r's lane slice). The rows' searches run in
-// lockstep so that their warp reductions overlap; a row that has found its cut stops updating.
-// Returns a bit mask of the rows that succeeded (the others need the exact fallback); sel[r] is
-// valid for those. `guess` seeds every row and is replaced by the last row's threshold.
-template <int M, int NR>
-RSM_DEV uint32_t warp_select_guess_rows(const float (&x)[NR][M / 32], int K, float& guess, uint32_t (&sel)[NR]) {
-  constexpr int E = M / 32;
-  auto key_to_float = [](uint32_t k) {
-    return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
-  };
-  float lo[NR], hi[NR], t[NR];
-  int clo[NR], chi[NR];
-  uint32_t live = 0u, ok = 0u;
-#pragma unroll
-  for (int r = 0; r < NR; ++r) {
-    float lmax = x[r][0], lmin = x[r][0];
-#pragma unroll
-    for (int e = 1; e < E; ++e) {
-      lmax = fmaxf(lmax, x[r][e]);
-      lmin = fminf(lmin, x[r][e]);
-    }
-    hi[r] = key_to_float(warp_max_u32(order_key(lmax)));
-    lo[r] = key_to_float(warp_min_u32(order_key(lmin)));
-  }
-#pragma unroll
-  for (int r = 0; r < NR; ++r) {
-    int c = 0;
-#pragma unroll
-    for (int e = 0; e < E; ++e) c += x[r][e] >= hi[r] ? 1 : 0;
-    chi[r] = warp_sum(c);  // multiplicity of the max
-    clo[r] = M;
-    t[r] = (guess > lo[r] && guess < hi[r]) ? guess : lo[r] + (hi[r] - lo[r]) * ((float)(M - K) / (float)M);
-    if (chi[r] < K) live |= 1u << r;  // otherwise a K-way tie at the max: fallback
-  }
-  for (int it = 0; it < 24 && live; ++it) {
-    int c[NR];
-#pragma unroll
-    for (int r = 0; r < NR; ++r) {
-      int cc = 0;
-#pragma unroll
-      for (int e = 0; e < E; ++e) cc += x[r][e] >= t[r] ? 1 : 0;
-      c[r] = warp_sum(cc);
-    }
-#pragma unroll
-    for (int r = 0; r < NR; ++r) {
-      if (!(live & (1u << r))) continue;
-      if (c[r] == K) {
-        live &= ~(1u << r);
-        ok |= 1u << r;
-        continue;
-      }
-      if (c[r] > K) {
-        lo[r] = t[r];
-        clo[r] = c[r];
-      } else {
-        hi[r] = t[r];
-        chi[r] = c[r];
-      }
-      float nt = (it % 3 == 2) ? 0.5f * (lo[r] + hi[r])
-                               : lo[r] + (hi[r] - lo[r]) * __fdividef((float)clo[r] - (float)K - 0.5f,
-                                                                      (float)(clo[r] - chi[r]));
-      if (!(nt > lo[r] && nt < hi[r])) nt = 0.5f * (lo[r] + hi[r]);
-      if (!(nt > lo[r] && nt < hi[r])) live &= ~(1u << r);  // adjacent floats: tie or near-tie
-      t[r] = nt;
-    }
-  }
-#pragma unroll
-  for (int r = 0; r < NR; ++r) {
-    sel[r] = 0u;
-#pragma unroll
-    for (int e = 0; e < E; ++e) sel[r] |= (x[r][e] >= t[r] ? 1u : 0u) << e;
-    if (ok & (1u << r)) guess = t[r];
-  }
-  return ok;
 }
 
 // Router variant scores of a row held by a warp (lane: E logits x[e]; sel: the lane's selected
