@@ -153,24 +153,32 @@ __global__ void __launch_bounds__(kBwdThreads, 1) backward_kernel(const BwdParam
   }
   // token t's copies into its slot (thread 0): the record, or its first part (entries and v) in
   // the forward sweep, and the tape rows in the reverse sweep when they travel through the ring
+  uint32_t pend = 0;  // thread 0: bit s set while slot s has copies in flight that no wait has seen
   auto issue = [&](int t, bool rev) {
     if (tid != 0 || t < 0 || t >= T || *abort_flag) return;
     unsigned char* sl = slot_of(t);
     uint64_t* br = &bar[t % R];
+    pend |= 1u << (t % R);
     const uint32_t rb = rev ? (uint32_t)RB : (uint32_t)rec_q(K, Dv);
     const uint32_t tb = (rev && tape_ring) ? (uint32_t)(K * Dv * 4) : 0u;
     tc::mbar_arrive_expect_tx(br, rb + tb);
     tc::bulk_load(sl, rec + (int64_t)t * RB, rb, br);
     if (tb) tc::bulk_load(sl + RB, tape + (int64_t)t * K * Dv, tb, br);
   };
-  uint32_t par = 0;  // bit s: parity of slot s's next completion (every thread counts alike)
+  // bit s: parity of slot s's next completion (every thread counts alike). After an expired wait
+  // the kernel stops copying and waiting, and the parity of a slot whose wait was skipped stays
+  // that of its copies in flight, which thread 0 drains (bounded) before the CTA ends.
+  uint32_t par = 0;
   auto wait_slot = [&](int t) {
     const int s = t % R;
-    if (!*abort_flag && !tc::mbar_wait(&bar[s], (par >> s) & 1u)) {
+    if (*abort_flag) return;
+    if (!tc::mbar_wait(&bar[s], (par >> s) & 1u)) {
       *abort_flag = 1;
       raise_status(RSM_ERR_TIMEOUT);
+      return;
     }
     par ^= 1u << s;
+    pend &= ~(1u << s);
   };
 
   for (int e = tid; e < M * Dv; e += kBwdThreads) sH[e] = a.H0 ? a.H0[(int64_t)pair * M * Dv + e] : 0.f;
@@ -294,6 +302,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) backward_kernel(const BwdParam
     }
   }
   __syncthreads();
+  if (tid == 0 && pend) {  // only after an expired wait: no copy may land once the CTA is gone
+    for (int sl = 0; sl < R; ++sl)
+      if (pend & (1u << sl)) tc::mbar_wait(&bar[sl], (par >> sl) & 1u);
+  }
   if (a.dH0)
     for (int e = tid; e < M * Dv; e += kBwdThreads) a.dH0[(int64_t)pair * M * Dv + e] = sG[e];
 }
