@@ -81,10 +81,13 @@ enum {
   /* Device-side check of the preconditions: a non-finite logit or a non-finite or positive f is
    * reported as RSM_ERR_NONFINITE by rsm_get_device_status (results are then undefined). */
   RSM_FLAG_VALIDATE = 1,
-  /* Testing aid for the bounded-wait error path (no counterpart on the pages; never set in normal
+  /* Testing aid for the bounded-wait error paths (no counterpart on the pages; never set in normal
    * use): in rsm_decode_step the routing warps hand over no routing slot and the warps waiting for
    * one give up after a short bound, so every CTA takes its timeout exit, the call writes neither o
-   * nor the state, and rsm_get_device_status reports RSM_ERR_TIMEOUT. Other calls ignore it. */
+   * nor the state, and rsm_get_device_status reports RSM_ERR_TIMEOUT. In rsm_backward the first token's
+   * copy is withheld and the sweeps' waits get a bound of one poll, so the first wait expires with
+   * the next tokens' copies in flight: the kernel stops, drains those copies (with the normal
+   * bound) and reports RSM_ERR_TIMEOUT; the gradients are then undefined. Other calls ignore it. */
   RSM_FLAG_TEST_STALL_ROUTING = 256
 };
 

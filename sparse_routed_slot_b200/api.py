@@ -200,10 +200,11 @@ def device_status(device=None) -> int:
 
 
 def backward(q, k, v, logits, f, K: int, dO=None, dHT=None, H0=None, *, validate: bool = False,
-             out=None, workspace=None):
+             out=None, workspace=None, flags: int = 0):
     """Gradients of rsm_forward (sigmoid router): q, k, v, logits, f, H0 as in forward();
     dO [B,T,H,Dv] fp32 and dHT [B,H,M,Dv] fp32 (None = zero). Returns dict(dq, dk, dlogits
-    [B,T,H,M], dv [B,T,H,Dv], df (f's shape), dH0 [B,H,M,Dv]), all fp32."""
+    [B,T,H,M], dv [B,T,H,Dv], df (f's shape), dH0 [B,H,M,Dv]), all fp32. `flags` are extra
+    RSM_FLAG_* bits passed through unchanged."""
     B, T, H, M = q.shape
     Dv = v.shape[-1]
     dev = q.device
@@ -228,6 +229,7 @@ def backward(q, k, v, logits, f, K: int, dO=None, dHT=None, H0=None, *, validate
         _need(out[name], name, torch.float32, shape)
         setattr(a, name, out[name].data_ptr())
     a.router = _lib.RSM_ROUTER_SIGMOID
+    a.flags = a.flags | flags
     L = _lib.load()
     need = L.rsm_backward_workspace_size(ctypes.byref(a))
     if need == ctypes.c_size_t(-1).value:

@@ -154,8 +154,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) backward_kernel(const BwdParam
   // token t's copies into its slot (thread 0): the record, or its first part (entries and v) in
   // the forward sweep, and the tape rows in the reverse sweep when they travel through the ring
   uint32_t pend = 0;  // thread 0: bit s set while slot s has copies in flight that no wait has seen
+  // test flag: the first token's copy is withheld, so its wait (bounded to one poll) expires while
+  // the copies of the tokens after it are in flight
+  const bool stall_test = (a.flags & RSM_FLAG_TEST_STALL_ROUTING) != 0;
   auto issue = [&](int t, bool rev) {
-    if (tid != 0 || t < 0 || t >= T || *abort_flag) return;
+    if (tid != 0 || t < 0 || t >= T || *abort_flag || (stall_test && t == 0 && !rev)) return;
     unsigned char* sl = slot_of(t);
     uint64_t* br = &bar[t % R];
     pend |= 1u << (t % R);
@@ -169,16 +172,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1) backward_kernel(const BwdParam
   // the kernel stops copying and waiting, and the parity of a slot whose wait was skipped stays
   // that of its copies in flight, which thread 0 drains (bounded) before the CTA ends.
   uint32_t par = 0;
-  auto wait_slot = [&](int t) {
+  // one poll under the test flag (the drain below keeps the normal bound)
+  const uint32_t wait_limit = stall_test ? 1u : (1u << 22);
+  // true when this thread has seen token t's copies land; a token is processed only when every
+  // thread has (a CTA-wide AND at the barrier that follows), so no thread ever indexes with
+  // entries from a slot that was not filled
+  auto wait_slot = [&](int t) -> bool {
     const int s = t % R;
-    if (*abort_flag) return;
-    if (!tc::mbar_wait(&bar[s], (par >> s) & 1u)) {
+    if (*abort_flag) return false;
+    if (!tc::mbar_wait(&bar[s], (par >> s) & 1u, wait_limit)) {
       *abort_flag = 1;
       raise_status(RSM_ERR_TIMEOUT);
-      return;
+      return false;
     }
     par ^= 1u << s;
     pend &= ~(1u << s);
+    return true;
   };
 
   for (int e = tid; e < M * Dv; e += kBwdThreads) sH[e] = a.H0 ? a.H0[(int64_t)pair * M * Dv + e] : 0.f;
@@ -186,9 +195,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) backward_kernel(const BwdParam
   // ---------------------------------------------------------------- forward sweep with tape
   for (int j = 0; j < R - 1; ++j) issue(j, false);
   for (int t = 0; t < T; ++t) {
-    wait_slot(t);
-    __syncthreads();  // token t-1 is finished: its slot can be refilled
+    // token t is in, and token t-1 is finished: its slot can be refilled
+    const bool ok = __syncthreads_and(wait_slot(t)) != 0;
     issue(t + R - 1, false);
+    if (!ok) continue;
     const unsigned char* sl = slot_of(t);
     const Entry* en = reinterpret_cast<const Entry*>(sl);
     const float* vr = reinterpret_cast<const float*>(sl + rec_v(K));
@@ -214,8 +224,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) backward_kernel(const BwdParam
   for (int j = 0; j < R - 1; ++j) issue(T - 1 - j, true);
   for (int t = T - 1; t >= 0; --t) {
     const int64_t row = row_of(t);
-    wait_slot(t);
-    __syncthreads();  // token t's record is in; token t+1 is finished
+    const bool ok = __syncthreads_and(wait_slot(t)) != 0;  // token t is in; token t+1 is finished
     issue(t - (R - 1), true);
     const unsigned char* sl = slot_of(t);
     const Entry* en = reinterpret_cast<const Entry*>(sl);
@@ -224,7 +233,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) backward_kernel(const BwdParam
     const float4* dO4 = reinterpret_cast<const float4*>(sl + rec_dO(M, K, Dv));
     // ---- phase A: the read. dq_i = do . H_t[i] and G[i] += q_i do, slot i by tps lanes; the slot
     // gradients of the row start at zero (the selected entries overwrite theirs after the barrier)
-    if (a.dO) {
+    if (!ok) {
+      // the token's copies did not land (an expired wait): no work, the barriers still match
+    } else if (a.dO) {
       const float qi = qr[ai];
       const float4* H4 = reinterpret_cast<const float4*>(sH + ai * Dv);
       float4* G4 = reinterpret_cast<float4*>(sG + ai * Dv);
@@ -244,7 +255,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) backward_kernel(const BwdParam
     } else if (a.dq && aj == 0) {
       a.dq[row * M + ai] = 0.f;
     }
-    if (aj == 0) {
+    if (ok && aj == 0) {
       if (a.dk) a.dk[row * M + ai] = 0.f;
       if (a.dlogits) a.dlogits[row * M + ai] = 0.f;
       if (a.df && a.decay == RSM_DECAY_SLOT) a.df[row * M + ai] = 0.f;
@@ -252,7 +263,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) backward_kernel(const BwdParam
     __syncthreads();
     // ---- phase B: gradients of the selected entries (one warp per entry; a token's slots are
     // distinct), and dv_t = sum_r w_r G[i_r] by column (the last Dv threads)
-    for (int r = warp; r < K; r += kBwdWarps) {
+    for (int r = warp; ok && r < K; r += kBwdWarps) {
       const Entry e = en[r];
       const float* Gi = sG + e.slot * Dv;
       const float* tp = tape_ring ? reinterpret_cast<const float*>(sl + RB) + r * Dv : tape + ((int64_t)t * K + r) * Dv;
@@ -272,7 +283,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) backward_kernel(const BwdParam
         sm[L.dfe + r] = e.s * dlam;
       }
     }
-    if (a.dv) {
+    if (ok && a.dv) {
       const int d = tid - (kBwdThreads - Dv);
       if (d >= 0) {
         float acc = 0.f;
@@ -283,7 +294,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) backward_kernel(const BwdParam
     __syncthreads();
     // ---- phase C: G of the selected rows decays, their state rows go back to H_{t-1}; the
     // per-head df of the token out
-    for (int r = warp; r < K; r += kBwdWarps) {
+    for (int r = warp; ok && r < K; r += kBwdWarps) {
       const int i = en[r].slot;
       const float ar = en[r].a;
       float* Gi = sG + i * Dv;
@@ -294,7 +305,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) backward_kernel(const BwdParam
         Hi[d] = tp[d];
       }
     }
-    if (a.df && a.decay == RSM_DECAY_HEAD && warp == kBwdWarps - 1) {
+    if (ok && a.df && a.decay == RSM_DECAY_HEAD && warp == kBwdWarps - 1) {
       float acc = 0.f;
       for (int r = lane; r < K; r += 32) acc += sm[L.dfe + r];
       acc = warp_sum_f(acc);

@@ -6,7 +6,10 @@
 * Bounded waits: RSM_FLAG_TEST_STALL_ROUTING makes the decode kernel's routing warps hand over
   nothing, so the consumer warps' wait for a routing slot expires after a short bound; the call
   reports RSM_ERR_TIMEOUT, leaves o and the state unwritten, and the context stays usable (a
-  normal step afterwards matches the oracle).
+  normal step afterwards matches the oracle). With the same flag rsm_backward withholds its first
+  token's copy and bounds its waits to one poll: the first wait expires with the next tokens' copies
+  in flight, the kernel drains them and reports RSM_ERR_TIMEOUT, and a normal call afterwards
+  matches the oracle.
 """
 import numpy as np
 import pytest
@@ -105,3 +108,22 @@ def test_decode_routing_stall_times_out_and_context_survives(rsm):
     assert np.array_equal(res["idx"].cpu().numpy(), r["idx"])
     assert rel(res["o"].cpu().numpy(), r["o"]) <= 1e-4
     assert rel(st.cpu().numpy(), r["state"]) <= 1e-4
+
+
+def test_backward_wait_expiry_reports_timeout_and_drains(rsm):
+    m, lib = rsm
+    B, T, H, M, K, Dv = 1, 40, 2, 64, 8, 64
+    x = make_inputs(B, T, H, M, Dv, torch.float32, "head", seed=5, device="cuda")
+    dO = torch.randn(B, T, H, Dv, generator=torch.Generator(device="cuda").manual_seed(4), device="cuda")
+    m.backward(x["q"], x["k"], x["v"], x["logits"], x["f"], K, dO, None, flags=lib.RSM_FLAG_TEST_STALL_ROUTING)
+    torch.cuda.synchronize()
+    assert m.device_status() == lib.RSM_ERR_TIMEOUT
+    assert m.device_status() == lib.RSM_OK
+    # the context is still usable: the same call without the flag matches the oracle
+    out = m.backward(x["q"], x["k"], x["v"], x["logits"], x["f"], K, dO, None)
+    torch.cuda.synchronize()
+    assert m.device_status() == lib.RSM_OK
+    c = {n: t.float().cpu().numpy() for n, t in x.items()}
+    r = oracle.backward(c["q"], c["k"], c["v"], c["logits"], c["f"], K, dO=dO.cpu().numpy())
+    for n in ("dq", "dk", "dv", "dlogits", "df", "dH0"):
+        assert rel(out[n].cpu().numpy(), r[n]) <= 1e-4, n
