@@ -391,3 +391,31 @@ def test_simt_narrow_and_ragged_value_tiles(rsm, M, Dv):
     r = oracle.forward(c["q"], c["k"], c["v"], c["logits"], c["f"], K, c["H0"])
     assert rel(out["o"].cpu().numpy(), r["o"]) <= TOL_FP32
     assert rel(out["HT"].cpu().numpy(), r["HT"]) <= TOL_FP32
+
+
+@pytest.mark.parametrize("M", [32, 64, 128])
+@pytest.mark.parametrize("K", [2, 8, 16, 31])
+def test_simt_set_selection_with_ties(rsm, M, K):
+    """Without ranked outputs the CUDA-core path takes each row's TopK set from a threshold search
+    seeded with the previous row, and the ranking tournament where the search meets a tie at the
+    cut. Logit rows with many exact ties, one-ulp near ties and plain Gaussian rows (so both ways
+    run, and the seed jumps between distributions): the per-slot selection counts, which fix every
+    row's set, are bit-exact, and o and the state match at the fp32 bar."""
+    B, T, H, Dv = 1, 96, 2, 64
+    x = make_inputs(B, T, H, M, Dv, torch.float32, "slot", seed=M * 7 + K, device="cuda", h0=True)
+    g = torch.Generator().manual_seed(M + K)
+    lg = torch.randn(B, T, H, M, generator=g)
+    lg[:, 16:48] = torch.round(3 * torch.randn(B, 32, H, M, generator=g)) / 3        # exact ties
+    near = torch.full((B, 16, H, M), 0.75)
+    bump = torch.rand(B, 16, H, M, generator=g) < 0.5
+    near[bump] = torch.nextafter(torch.tensor(0.75), torch.tensor(1.0))
+    lg[:, 48:64] = near                                                                # near ties
+    x["logits"] = lg.float().contiguous().cuda()
+    counts = torch.zeros((B, H, M), dtype=torch.int32, device="cuda")
+    out = rsm.forward(x["q"], x["k"], x["v"], x["logits"], x["f"], K, x["H0"], path="simt", slot_counts=counts)
+    torch.cuda.synchronize()
+    c = host(x)
+    r = oracle.forward(c["q"], c["k"], c["v"], c["logits"], c["f"], K, c["H0"], want_counts=True)
+    assert np.array_equal(counts.cpu().numpy(), r["counts"])
+    assert rel(out["o"].cpu().numpy(), r["o"]) <= TOL_FP32
+    assert rel(out["HT"].cpu().numpy(), r["HT"]) <= TOL_FP32
